@@ -1,0 +1,215 @@
+/*
+ * llama_b200.h - C ABI of the B200 (sm_100a) LLaMA decoder-block library.
+ *
+ * The library computes the forward pass of the LLaMA decoder with a KV-cache:
+ * token-embedding gather, per block pre-norm RMSNorm, the fused Q/K/V
+ * projection with interleaved-pair RoPE and the cache append in its epilogue,
+ * causal grouped-query attention over the cache (a flash-style prefill kernel
+ * for T > 1, a split-K flash-decode kernel for T == 1), the output projection
+ * plus residual, the second RMSNorm, the SwiGLU FFN w2(silu(w1 x) * w3 x) plus
+ * residual, and for whole-model calls the final RMSNorm and the LM head.
+ *
+ * Sources (pages), cited by title and section:
+ *  - "LLaMA: Open and Efficient Foundation Language Models" (notes,
+ *    unpurerationalist.github.io), section 3 code: ModelArgs, RMSNorm,
+ *    precompute_freqs_cis, apply_rotary_emb, repeat_kv, Attention,
+ *    FeedForward, TransformerBlock, Transformer.
+ *  - "灵哥讲llama3(中)" (blog.csdn.net), Transformer class: rope_theta and the
+ *    causal mask when the cache already holds start_pos tokens.
+ *  - LLaMA model.py walk-through (linkmax.top), section 2.3 RoPE (the
+ *    element-wise rotation) and section 3.2 model.
+ *  - "LLaMa-1/2/3 原理+源码——拆解" (aitechtogether.com), section KV-Cache.
+ *
+ * Conventions for every call:
+ *  - Pointers named *_dev are device pointers; the caller owns them and the
+ *    library only borrows them for the duration of the call. Pointers named
+ *    *_host are host pointers.
+ *  - "act" is the activation/weight storage type chosen at create time:
+ *    float (LLAMA_FP32) or bfloat16 (LLAMA_BF16). Accumulation is always fp32.
+ *    The residual stream h is always fp32.
+ *  - Calls that take a cuda_stream (a cudaStream_t, may be NULL for the
+ *    legacy default stream) are asynchronous and stream-ordered; the library
+ *    never synchronises inside them, so they can be captured in a CUDA graph
+ *    once llama_reserve has sized the workspace for the largest call.
+ *  - Every int-returning call returns LLAMA_OK (0) or a negative error code;
+ *    an error returned before any launch leaves all state unchanged.
+ *    Problems only the device can see (a token id out of range, a position
+ *    past the cache, a bounded wait that timed out) set a device flag that
+ *    llama_get_error reads back.
+ */
+#ifndef LLAMA_B200_H
+#define LLAMA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* storage types */
+#define LLAMA_FP32 0
+#define LLAMA_BF16 1
+
+/* return codes */
+#define LLAMA_OK 0
+#define LLAMA_ERR_INVALID_ARGS -1 /* a size or shape rule below is broken */
+#define LLAMA_ERR_OOM -2          /* device allocation failed */
+#define LLAMA_ERR_CUDA -3         /* a CUDA runtime/driver call failed */
+#define LLAMA_ERR_NOT_READY -4    /* weights for a needed layer/head not set */
+#define LLAMA_ERR_TOKEN_RANGE -10 /* device flag: a token id outside [0, vocab_size) */
+#define LLAMA_ERR_POS_RANGE -11   /* device flag: start_pos[b] + s outside [0, max_seq_len) */
+#define LLAMA_ERR_TIMEOUT -12     /* device flag: a bounded in-kernel wait gave up */
+
+/* GEMM path selection for llama_linear (diagnostics) */
+#define LLAMA_PATH_AUTO 0
+#define LLAMA_PATH_TCGEN05 1 /* TMA + tcgen05/TMEM tensor-core GEMM (bf16) */
+#define LLAMA_PATH_GEMV 2    /* weight-streaming split-K kernel for M <= 32 (bf16) */
+#define LLAMA_PATH_SIMT 3    /* fp32 CUDA-core tiled GEMM (fp32 or bf16) */
+
+/*
+ * ModelArgs of the notes' section 3 code plus rope_theta ("灵哥讲llama3(中)",
+ * Transformer class) and the storage type.
+ *  dim, n_layers, n_heads, n_kv_heads (n_kv_heads <= 0 means n_kv_heads = n_heads),
+ *  vocab_size (0 for single-block use), multiple_of, ffn_dim_multiplier
+ *  (<= 0 means None), norm_eps, rope_theta, max_batch_size, max_seq_len, dtype.
+ * Rules: dim % n_heads == 0; head_dim = dim / n_heads in {64, 128};
+ *  n_heads % n_kv_heads == 0; n_heads / n_kv_heads <= 8 when dtype == LLAMA_BF16,
+ *  or a multiple of 8; dim % 64 == 0; all sizes positive.
+ */
+typedef struct {
+  int32_t dim;
+  int32_t n_layers;
+  int32_t n_heads;
+  int32_t n_kv_heads;
+  int32_t vocab_size;
+  int32_t multiple_of;
+  float ffn_dim_multiplier;
+  float norm_eps;
+  float rope_theta;
+  int32_t max_batch_size;
+  int32_t max_seq_len;
+  int32_t dtype;
+} llama_args;
+
+typedef struct llama_ctx llama_ctx;
+
+/*
+ * The SwiGLU hidden width of the notes' FeedForward: two thirds of 4*dim
+ * (truncated), times ffn_dim_multiplier when set (truncated), rounded up to a
+ * multiple of multiple_of. Returns the width, or LLAMA_ERR_INVALID_ARGS.
+ */
+int llama_ffn_hidden(const llama_args* args);
+
+/*
+ * Create a model context on the current CUDA device: validates args,
+ * allocates the packed weights, the per-layer K and V caches (zeroed, as the
+ * notes' Attention.__init__ preallocates zeros), the RoPE table of
+ * 2 * max_seq_len positions (precompute_freqs_cis, cos/sin in fp32) and an
+ * empty workspace. *out receives the context. The library owns all of it
+ * until llama_destroy.
+ * Cache layout inside the library: [layer][batch][kv_head][position][head_dim]
+ * (one (batch, kv head) history is contiguous); llama_kv_read/llama_kv_write
+ * convert to and from the pages' [batch][position][kv_head][head_dim].
+ */
+int llama_create(const llama_args* args, llama_ctx** out);
+
+/* Free everything the context owns (synchronises the device first). NULL is a no-op. */
+void llama_destroy(llama_ctx* ctx);
+
+/*
+ * Copy (and pack) one block's weights from device memory in the act type,
+ * nn.Linear layout [out_features][in_features], row-major:
+ *  wq [n_heads*hd][dim], wk, wv [n_kv_heads*hd][dim], wo [dim][n_heads*hd],
+ *  w1, w3 [ffn][dim], w2 [dim][ffn]; attn_norm, ffn_norm [dim].
+ * The library packs wq|wk|wv into one matrix and interleaves the rows of w1
+ * and w3 (row 2j = w1 row j, row 2j+1 = w3 row j). Synchronous with respect
+ * to the host (the sources may be freed on return).
+ */
+int llama_set_layer(llama_ctx* ctx, int layer, const void* wq_dev, const void* wk_dev, const void* wv_dev,
+                    const void* wo_dev, const void* w1_dev, const void* w2_dev, const void* w3_dev,
+                    const void* attn_norm_dev, const void* ffn_norm_dev);
+
+/*
+ * Copy the token embedding [vocab][dim], the final norm weight [dim] and the
+ * LM head [vocab][dim] (act type, device memory). Synchronous like llama_set_layer.
+ */
+int llama_set_embed_norm_head(llama_ctx* ctx, const void* tok_embeddings_dev, const void* norm_dev,
+                              const void* output_dev);
+
+/*
+ * Size the workspace for calls of up to max_tokens tokens (B*T). Calls with
+ * more tokens grow it on demand, which allocates and therefore cannot be
+ * captured in a CUDA graph; call this first to capture.
+ */
+int llama_reserve(llama_ctx* ctx, int max_tokens);
+
+/*
+ * Transformer.forward(tokens, start_pos) of the notes: tokens_dev int32 [B][T]
+ * (row-major), the same start_pos for every sequence. Writes this call's keys
+ * and values to cache positions start_pos .. start_pos+T-1 of sequences
+ * 0..B-1 and fp32 logits to logits_dev: [B][T][vocab] when all_positions != 0,
+ * else only the last position, [B][vocab].
+ * Rules: 1 <= B <= max_batch_size, T >= 1, 0 <= start_pos, start_pos + T <= max_seq_len.
+ */
+int llama_forward(llama_ctx* ctx, const int32_t* tokens_dev, int B, int T, int start_pos, float* logits_dev,
+                  int all_positions, void* cuda_stream);
+
+/*
+ * One decode step with a per-sequence position (ragged batches): tokens_dev
+ * int32 [B] (T = 1), start_pos_dev int32 [B]; sequence b's new token goes to
+ * cache position start_pos_dev[b] and attends to positions 0..start_pos_dev[b].
+ * logits_dev fp32 [B][vocab]. A position outside [0, max_seq_len) raises
+ * LLAMA_ERR_POS_RANGE on the device flag and that token's cache write is skipped.
+ */
+int llama_forward_ragged(llama_ctx* ctx, const int32_t* tokens_dev, const int32_t* start_pos_dev, int B,
+                         float* logits_dev, void* cuda_stream);
+
+/*
+ * One TransformerBlock.forward in place on the fp32 residual stream
+ * h_dev [B][T][dim]: h <- h + attn(attention_norm(h)); h <- h + ffn(ffn_norm(h)).
+ * start_pos_dev int32 [B] gives each sequence's position of its first token
+ * (device memory); when it is NULL, host_start_pos is used for all sequences
+ * and checked on the host. Used for single-layer workloads.
+ */
+int llama_block_forward(llama_ctx* ctx, int layer, float* h_dev, int B, int T, const int32_t* start_pos_dev,
+                        int host_start_pos, void* cuda_stream);
+
+/*
+ * Copy one layer's caches out of / into the library, in the pages' logical
+ * layout [max_batch_size][max_seq_len][n_kv_heads][head_dim], act type,
+ * device memory. Stream-ordered.
+ */
+int llama_kv_read(llama_ctx* ctx, int layer, void* k_dev, void* v_dev, void* cuda_stream);
+int llama_kv_write(llama_ctx* ctx, int layer, const void* k_dev, const void* v_dev, void* cuda_stream);
+
+/* Zero every cache (synchronous). */
+int llama_reset(llama_ctx* ctx);
+
+/*
+ * Synchronise the device, then return and clear the device flags: LLAMA_OK,
+ * or the most severe of LLAMA_ERR_TIMEOUT, LLAMA_ERR_POS_RANGE,
+ * LLAMA_ERR_TOKEN_RANGE. *flags (if not NULL) receives the raw flag bits
+ * (1 token range, 2 position range, 4 timeout). A pending asynchronous CUDA
+ * error is returned as LLAMA_ERR_CUDA.
+ */
+int llama_get_error(llama_ctx* ctx, int* flags);
+
+/* A static description of an error code. */
+const char* llama_strerror(int code);
+
+/*
+ * Diagnostics: y_dev[M][N] (fp32) = x_dev[M][K] * w_dev[N][K]^T with fp32
+ * accumulation, x and w both of storage type dtype, through the chosen GEMM
+ * path (LLAMA_PATH_*). Rules: M, N, K > 0, N % 8 == 0, K % 8 == 0;
+ * LLAMA_PATH_GEMV needs M <= 32 and K % 32 == 0; LLAMA_PATH_TCGEN05 needs
+ * dtype == LLAMA_BF16. Uses a private, lazily allocated workspace; not
+ * thread-safe.
+ */
+int llama_linear(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, int dtype, int path,
+                 void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_B200_H */

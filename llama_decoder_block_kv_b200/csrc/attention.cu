@@ -1,0 +1,632 @@
+// Causal grouped-query attention over the KV-cache.
+//
+// What is computed ("LLaMA: Open and Efficient Foundation Language Models"
+// notes, Attention.forward and Transformer.forward; "灵哥讲llama3(中)", the
+// cached-mask comment): for the query of sequence b at position
+// p = start_pos[b] + s and query head h, attend over the cached keys
+// j = 0 .. p of kv head h / n_rep (repeat_kv maps kv head j to query heads
+// j*n_rep .. j*n_rep + n_rep - 1) with scores q.k / sqrt(D) and a softmax.
+// The additive mask of the pages is never built: the predicate j <= p is
+// applied inside the kernels, and key tiles that are fully masked for a warp
+// are skipped (the pages' xformers remark: masked scores are not computed).
+//
+// Kernels:
+//  - attn_prefill_kernel (T > 1): flash-style online softmax. A CTA owns one
+//    (sequence, kv head) and 128 query rows made of up to 8 query heads of
+//    that kv group times 128/heads positions, so each K/V tile is loaded once
+//    for the whole group. K/V tiles (64 keys) arrive by TMA (128-byte swizzle,
+//    no multicast) into a 3-stage ring fed by a producer warp; 8 compute warps
+//    run S = QK^T and O += PV on the warp-level bf16 tensor-core MMA.
+//  - attn_decode_kernel (T == 1): split-K flash decode. A CTA owns one
+//    (sequence, kv head, chunk of keys); the chunk streams through the same
+//    TMA ring, the 4 compute warps each take 16 keys of every 64-key tile,
+//    their (max, sum, O) states merge in shared memory and the CTA writes one
+//    partial; attn_decode_combine_kernel merges the partials of all chunks
+//    with the log-sum-exp rule m = max m_c, l = sum l_c e^(m_c - m),
+//    o = sum o_c e^(m_c - m) / l.
+//  - attn_simple_kernel: fp32 mode (tiny models), one CTA per (token, head),
+//    scores in shared memory, plain two-pass softmax.
+#include "kernels.cuh"
+
+namespace llama {
+
+namespace {
+constexpr int KT = 64;  // keys per tile
+constexpr float LOG2E = 1.4426950408889634f;
+}  // namespace
+
+// Byte address of element (row, col) inside a TMA box of 64 rows x 64 bf16
+// written with 128-byte swizzling: the 16-byte chunk index is XOR-ed with row % 8.
+__device__ __forceinline__ uint32_t sw_addr(uint32_t box_base, int row, int col) {
+  return box_base + row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2;
+}
+
+__device__ __forceinline__ float quad_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+
+template <int D>
+struct AttnSmem {
+  static constexpr int HALVES = D / 64;
+  static constexpr uint32_t TILE_BYTES = KT * D * 2;  // one K or one V tile
+};
+
+// Issue the TMA loads of one K tile and one V tile (keys row .. row+63).
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const CUtensorMap* mk, const CUtensorMap* mv, uint8_t* sk, uint8_t* sv,
+                                             uint64_t* bar, int row) {
+  mbar_arrive_expect_tx(bar, 2 * AttnSmem<D>::TILE_BYTES);
+#pragma unroll
+  for (int h = 0; h < AttnSmem<D>::HALVES; ++h) {
+    tma_load_2d(sk + h * 8192, mk, bar, h * 64, row);
+    tma_load_2d(sv + h * 8192, mv, bar, h * 64, row);
+  }
+}
+
+// ============================================================================ prefill
+
+template <int D>
+__global__ void __launch_bounds__(288, 1)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                        const bf16* __restrict__ q, bf16* __restrict__ o, const int* __restrict__ start_pos,
+                        int sp_scalar, int T, int H, int Hkv, int S_max, int hpc, int* err) {
+  constexpr int STAGES = 3;
+  constexpr uint32_t TB = AttnSmem<D>::TILE_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * 2 * TB);
+  uint64_t* empty = full + STAGES;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, qd = lane & 3;
+  const int n_rep = H / Hkv, groups = n_rep / hpc;
+  const int BQ = 128 / hpc;
+  const int qblk = gridDim.x - 1 - blockIdx.x;  // longest (latest) query blocks first
+  const int z = blockIdx.y;
+  const int b = z / (Hkv * groups);
+  const int kvh = (z / groups) % Hkv;
+  const int grp = z % groups;
+  const int q0 = qblk * BQ;
+  const int sp = start_pos ? start_pos[b] : sp_scalar;
+  const int q_last = min(q0 + BQ, T) - 1;
+  const int kv_len = min(sp + q_last + 1, S_max);
+  const int n_tiles = (kv_len + KT - 1) / KT;
+  const int row0 = (b * Hkv + kvh) * S_max;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 8);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    if (lane == 0) {
+      prefetch_tensormap(&map_k);
+      prefetch_tensormap(&map_v);
+      int j = 0;
+      for (; j < n_tiles; ++j) {
+        const int st = j % STAGES;
+        if (!mbar_wait(&empty[st], ((j / STAGES) & 1) ^ 1, err)) break;
+        load_kv_tile<D>(&map_k, &map_v, base + st * 2 * TB, base + st * 2 * TB + TB, &full[st], row0 + j * KT);
+      }
+      // the CTA must not retire while a copy into its shared memory is in flight
+      for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, err);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- compute warps
+  const int hl = (warp * 16) / BQ;           // query head inside this CTA
+  const int pl0 = (warp * 16) % BQ;          // first position (inside the block) of this warp
+  const int h = kvh * n_rep + grp * hpc + hl;
+  const int t0 = q0 + pl0 + g, t1 = t0 + 8;  // call-relative positions of this thread's two rows
+  const int c0 = min(t0, T - 1), c1 = min(t1, T - 1);
+  const int p0 = sp + c0, p1 = sp + c1;
+  const int warp_pmax = sp + min(q0 + pl0 + 15, T - 1);
+
+  uint32_t qa[D / 16][4];
+  {
+    const bf16* r0 = q + ((size_t)(b * T + c0) * H + h) * D;
+    const bf16* r1 = q + ((size_t)(b * T + c1) * H + h) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qa[kk][0] = *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd);
+      qa[kk][1] = *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd);
+      qa[kk][2] = *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd);
+      qa[kk][3] = *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd);
+    }
+  }
+  float oacc[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const float sl2 = rsqrtf((float)D) * LOG2E;
+
+  for (int j = 0; j < n_tiles; ++j) {
+    const int st = j % STAGES;
+    const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    if (j * KT <= warp_pmax) {
+      const uint32_t kb = smem_u32(base + st * 2 * TB);
+      const uint32_t vb = kb + TB;
+      float s[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+        for (int jn = 0; jn < 8; jn += 2) {
+          const int mi = lane >> 3;
+          const int key = 8 * (jn + (mi >> 1)) + (lane & 7);
+          const int d = 16 * kk + 8 * (mi & 1);
+          uint32_t bf[4];
+          ldmatrix_x4(bf, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(s[jn], qa[kk], b0);
+          mma_bf16_16816(s[jn + 1], qa[kk], b1);
+        }
+      }
+      const bool need_mask = (j * KT + KT - 1) > (sp + min(q0 + pl0, T - 1));
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int jn = 0; jn < 8; ++jn) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = s[jn][e] * sl2;
+          if (need_mask) {
+            const int key = j * KT + 8 * jn + 2 * qd + (e & 1);
+            if (key > (e < 2 ? p0 : p1)) v = -INFINITY;
+          }
+          s[jn][e] = v;
+        }
+        mx0 = fmaxf(mx0, fmaxf(s[jn][0], s[jn][1]));
+        mx1 = fmaxf(mx1, fmaxf(s[jn][2], s[jn][3]));
+      }
+      mx0 = quad_max(mx0);
+      mx1 = quad_max(mx1);
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= sc0;
+      l1 *= sc1;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        oacc[i][0] *= sc0;
+        oacc[i][1] *= sc0;
+        oacc[i][2] *= sc1;
+        oacc[i][3] *= sc1;
+      }
+#pragma unroll
+      for (int jn = 0; jn < 8; ++jn) {
+        s[jn][0] = exp2f(s[jn][0] - mn0);
+        s[jn][1] = exp2f(s[jn][1] - mn0);
+        s[jn][2] = exp2f(s[jn][2] - mn1);
+        s[jn][3] = exp2f(s[jn][3] - mn1);
+        l0 += s[jn][0] + s[jn][1];
+        l1 += s[jn][2] + s[jn][3];
+      }
+#pragma unroll
+      for (int kb2 = 0; kb2 < 4; ++kb2) {
+        const uint32_t pa[4] = {pack_bf16x2(s[2 * kb2][0], s[2 * kb2][1]), pack_bf16x2(s[2 * kb2][2], s[2 * kb2][3]),
+                                pack_bf16x2(s[2 * kb2 + 1][0], s[2 * kb2 + 1][1]),
+                                pack_bf16x2(s[2 * kb2 + 1][2], s[2 * kb2 + 1][3])};
+#pragma unroll
+        for (int jd = 0; jd < D / 8; jd += 2) {
+          const int mi = lane >> 3;
+          const int key = 16 * kb2 + 8 * (mi & 1) + (lane & 7);
+          const int d = 8 * (jd + (mi >> 1));
+          uint32_t bf[4];
+          ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(oacc[jd], pa, b0);
+          mma_bf16_16816(oacc[jd + 1], pa, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  l0 = quad_sum(l0);
+  l1 = quad_sum(l1);
+  const float i0 = 1.f / l0, i1 = 1.f / l1;
+  if (t0 < T) {
+    bf16* dst = o + ((size_t)(b * T + t0) * H + h) * D;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i)
+      *reinterpret_cast<uint32_t*>(dst + 8 * i + 2 * qd) = pack_bf16x2(oacc[i][0] * i0, oacc[i][1] * i0);
+  }
+  if (t1 < T) {
+    bf16* dst = o + ((size_t)(b * T + t1) * H + h) * D;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i)
+      *reinterpret_cast<uint32_t*>(dst + 8 * i + 2 * qd) = pack_bf16x2(oacc[i][2] * i1, oacc[i][3] * i1);
+  }
+}
+
+// ============================================================================ decode
+
+template <int D>
+__global__ void __launch_bounds__(160)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                       const bf16* __restrict__ q, float* __restrict__ part_o, float* __restrict__ part_ml,
+                       const int* __restrict__ start_pos, int sp_scalar, int H, int Hkv, int S_max, int hpc, int CK,
+                       int max_chunks, int* err) {
+  constexpr int STAGES = 3;
+  constexpr uint32_t TB = AttnSmem<D>::TILE_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * 2 * TB);
+  uint64_t* empty = full + STAGES;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, qd = lane & 3;
+  const int n_rep = H / Hkv, groups = n_rep / hpc;
+  const int chunk = blockIdx.x;
+  const int z = blockIdx.y;
+  const int b = z / (Hkv * groups);
+  const int kvh = (z / groups) % Hkv;
+  const int grp = z % groups;
+  const int sp = start_pos ? start_pos[b] : sp_scalar;
+  const int L = min(sp + 1, S_max);  // keys 0 .. sp
+  const int k_begin = chunk * CK;
+  if (k_begin >= L) return;  // ragged batches: this sequence has fewer chunks
+  const int k_end = min(L, k_begin + CK);
+  const int n_tiles = (k_end - k_begin + KT - 1) / KT;
+  const int row0 = (b * Hkv + kvh) * S_max + k_begin;
+  const int h0 = kvh * n_rep + grp * hpc;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&map_k);
+      prefetch_tensormap(&map_v);
+      int j = 0;
+      for (; j < n_tiles; ++j) {
+        const int st = j % STAGES;
+        if (!mbar_wait(&empty[st], ((j / STAGES) & 1) ^ 1, err)) break;
+        load_kv_tile<D>(&map_k, &map_v, base + st * 2 * TB, base + st * 2 * TB + TB, &full[st], row0 + j * KT);
+      }
+      for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, err);
+    }
+    return;
+  }
+
+  // query rows: g and g + 8 are heads h0 + g, h0 + g + 8 when inside the group of hpc
+  uint32_t qa[D / 16][4];
+  {
+    const bool v0 = g < hpc, v1 = g + 8 < hpc;
+    const bf16* r0 = q + ((size_t)b * H + h0 + (v0 ? g : 0)) * D;
+    const bf16* r1 = q + ((size_t)b * H + h0 + (v1 ? g + 8 : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qa[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
+      qa[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd) : 0u;
+      qa[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
+      qa[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
+    }
+  }
+  float oacc[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const float sl2 = rsqrtf((float)D) * LOG2E;
+
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) s_abort = 0;
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  for (int j = 0; j < n_tiles; ++j) {
+    const int st = j % STAGES;
+    const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) atomicExch(&s_abort, 1);
+      break;
+    }
+    const int key0 = k_begin + j * KT + 16 * warp;  // first key of this warp's 16
+    if (key0 < k_end) {
+      const uint32_t kb = smem_u32(base + st * 2 * TB);
+      const uint32_t vb = kb + TB;
+      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int mi = lane >> 3;
+        const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+        const int d = 16 * kk + 8 * (mi & 1);
+        uint32_t bf[4];
+        ldmatrix_x4(bf, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
+        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+        mma_bf16_16816(s[0], qa[kk], b0);
+        mma_bf16_16816(s[1], qa[kk], b1);
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int jn = 0; jn < 2; ++jn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = s[jn][e] * sl2;
+          if (key0 + 8 * jn + 2 * qd + (e & 1) >= k_end) v = -INFINITY;
+          s[jn][e] = v;
+          if (e < 2)
+            mx0 = fmaxf(mx0, v);
+          else
+            mx1 = fmaxf(mx1, v);
+        }
+      mx0 = quad_max(mx0);
+      mx1 = quad_max(mx1);
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= sc0;
+      l1 *= sc1;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        oacc[i][0] *= sc0;
+        oacc[i][1] *= sc0;
+        oacc[i][2] *= sc1;
+        oacc[i][3] *= sc1;
+      }
+#pragma unroll
+      for (int jn = 0; jn < 2; ++jn) {
+        s[jn][0] = exp2f(s[jn][0] - mn0);
+        s[jn][1] = exp2f(s[jn][1] - mn0);
+        s[jn][2] = exp2f(s[jn][2] - mn1);
+        s[jn][3] = exp2f(s[jn][3] - mn1);
+        l0 += s[jn][0] + s[jn][1];
+        l1 += s[jn][2] + s[jn][3];
+      }
+      const uint32_t pa[4] = {pack_bf16x2(s[0][0], s[0][1]), pack_bf16x2(s[0][2], s[0][3]),
+                              pack_bf16x2(s[1][0], s[1][1]), pack_bf16x2(s[1][2], s[1][3])};
+#pragma unroll
+      for (int jd = 0; jd < D / 8; jd += 2) {
+        const int mi = lane >> 3;
+        const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
+        const int d = 8 * (jd + (mi >> 1));
+        uint32_t bf[4];
+        ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
+        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+        mma_bf16_16816(oacc[jd], pa, b0);
+        mma_bf16_16816(oacc[jd + 1], pa, b1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // merge the 4 warps' states through shared memory (the ring is idle now)
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (*(volatile int*)&s_abort) return;  // CTA-uniform
+  l0 = quad_sum(l0);
+  l1 = quad_sum(l1);
+  float* sm_o = reinterpret_cast<float*>(base);     // [4][16][D]
+  float* sm_m = sm_o + 4 * 16 * D;                  // [4][16]
+  float* sm_l = sm_m + 4 * 16;                      // [4][16]
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd] = oacc[i][0];
+    sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd + 1] = oacc[i][1];
+    sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd] = oacc[i][2];
+    sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd + 1] = oacc[i][3];
+  }
+  if (qd == 0) {
+    sm_m[warp * 16 + g] = m0;
+    sm_m[warp * 16 + g + 8] = m1;
+    sm_l[warp * 16 + g] = l0;
+    sm_l[warp * 16 + g + 8] = l1;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  for (int e = threadIdx.x; e < hpc * D; e += 128) {
+    const int r = e / D, d = e - r * D;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mm = fmaxf(mm, sm_m[w * 16 + r]);
+    float acc = 0.f, ll = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mw = sm_m[w * 16 + r];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - mm);
+      acc += sm_o[(w * 16 + r) * D + d] * f;
+      ll += sm_l[w * 16 + r] * f;
+    }
+    const size_t slot = ((size_t)b * H + h0 + r) * max_chunks + chunk;
+    part_o[slot * D + d] = acc;
+    if (d == 0) {
+      part_ml[slot * 2] = mm;
+      part_ml[slot * 2 + 1] = ll;
+    }
+  }
+}
+
+__global__ void attn_decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                                           bf16* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar,
+                                           int H, int D, int S_max, int CK, int max_chunks) {
+  const int bh = blockIdx.x;
+  const int b = bh / H;
+  const int sp = start_pos ? start_pos[b] : sp_scalar;
+  const int L = min(sp + 1, S_max);
+  const int nc = (L + CK - 1) / CK;
+  const float* ml = part_ml + (size_t)bh * max_chunks * 2;
+  float mm = -INFINITY;
+  for (int c = 0; c < nc; ++c) mm = fmaxf(mm, ml[2 * c]);
+  float ll = 0.f;
+  for (int c = 0; c < nc; ++c) ll += ml[2 * c + 1] * exp2f(ml[2 * c] - mm);
+  const float inv = 1.f / ll;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int c = 0; c < nc; ++c) acc += part_o[((size_t)bh * max_chunks + c) * D + d] * exp2f(ml[2 * c] - mm);
+    o[(size_t)bh * D + d] = __float2bfloat16_rn(acc * inv);
+  }
+}
+
+// ============================================================================ fp32 mode
+
+template <typename T>
+__global__ void attn_simple_kernel(const T* __restrict__ q, const T* __restrict__ ck, const T* __restrict__ cv,
+                                   T* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar, int T_, int H,
+                                   int Hkv, int D, int S_max) {
+  extern __shared__ float sm[];
+  float* qs = sm;             // [D]
+  float* sc = sm + D;         // [S_max]
+  __shared__ float red[32];
+  const int t = blockIdx.x, h = blockIdx.y;
+  const int b = t / T_, s = t - b * T_;
+  const int pos = min((start_pos ? start_pos[b] : sp_scalar) + s, S_max - 1);
+  const int kvh = h / (H / Hkv);
+  const float scale = rsqrtf((float)D);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) qs[d] = to_f32(q[((size_t)t * H + h) * D + d]);
+  __syncthreads();
+  const T* K = ck + (size_t)(b * Hkv + kvh) * S_max * D;
+  const T* V = cv + (size_t)(b * Hkv + kvh) * S_max * D;
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j <= pos; j += blockDim.x) {
+    float acc = 0.f;
+    for (int d = 0; d < D; ++d) acc = fmaf(qs[d], to_f32(K[(size_t)j * D + d]), acc);
+    sc[j] = acc * scale;
+    mx = fmaxf(mx, sc[j]);
+  }
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    red[0] = m;
+  }
+  __syncthreads();
+  mx = red[0];
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = threadIdx.x; j <= pos; j += blockDim.x) {
+    const float e = expf(sc[j] - mx);
+    sc[j] = e;
+    sum += e;
+  }
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s2 = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s2 += red[w];
+    red[0] = s2;
+  }
+  __syncthreads();
+  const float inv = 1.f / red[0];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j <= pos; ++j) acc = fmaf(sc[j], to_f32(V[(size_t)j * D + d]), acc);
+    o[((size_t)t * H + h) * D + d] = from_f32<T>(acc * inv);
+  }
+}
+
+// ============================================================================ host launchers
+
+template <int D>
+static cudaError_t prefill_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
+                             int sp_scalar, int B, int T, int H, int Hkv, int S_max, int* err, cudaStream_t st) {
+  const int n_rep = H / Hkv;
+  const int hpc = n_rep < 8 ? n_rep : 8;
+  const int BQ = 128 / hpc;
+  const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((T + BQ - 1) / BQ, B * Hkv * (n_rep / hpc));
+  attn_prefill_kernel<D><<<grid, 288, smem, st>>>(mk, mv, reinterpret_cast<const bf16*>(q), reinterpret_cast<bf16*>(o),
+                                                  sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
+                                int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max, int* err,
+                                cudaStream_t st) {
+  if (D == 128) return prefill_d<128>(mk, mv, q, o, sp, sp_scalar, B, T, H, Hkv, S_max, err, st);
+  return prefill_d<64>(mk, mv, q, o, sp, sp_scalar, B, T, H, Hkv, S_max, err, st);
+}
+
+DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sms) {
+  DecodePlan p;
+  const int n_rep = H / Hkv;
+  p.hpc = n_rep < 16 ? n_rep : 16;
+  const int units = B * Hkv * (n_rep / p.hpc);
+  // chunks per unit so that the grid covers the SMs about twice (at least one tile each)
+  int want = (2 * num_sms + units - 1) / units;
+  int ck = (max_len + want - 1) / want;
+  ck = (ck + KT - 1) / KT * KT;
+  if (ck < 128) ck = 128;
+  if (ck > 1024) ck = 1024;
+  p.CK = ck;
+  p.max_chunks = (S_max + ck - 1) / ck;
+  p.part_floats = (size_t)B * H * p.max_chunks * 128 + (size_t)B * H * p.max_chunks * 2;
+  return p;
+}
+
+template <int D>
+static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
+                            const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max, const DecodePlan& p,
+                            int* err, cudaStream_t st) {
+  const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int n_rep = H / Hkv;
+  float* part_o = part;
+  float* part_ml = part + (size_t)B * H * p.max_chunks * D;
+  dim3 grid(p.max_chunks, B * Hkv * (n_rep / p.hpc));
+  attn_decode_kernel<D><<<grid, 160, smem, st>>>(mk, mv, reinterpret_cast<const bf16*>(q), part_o, part_ml, sp,
+                                                 sp_scalar, H, Hkv, S_max, p.hpc, p.CK, p.max_chunks, err);
+  attn_decode_combine_kernel<<<B * H, D, 0, st>>>(part_o, part_ml, reinterpret_cast<bf16*>(o), sp, sp_scalar, H, D,
+                                                  S_max, p.CK, p.max_chunks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
+                               const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
+                               const DecodePlan& p, int* err, cudaStream_t st) {
+  if (D == 128) return decode_d<128>(mk, mv, q, o, part, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  return decode_d<64>(mk, mv, q, o, part, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+}
+
+template <typename T>
+cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, void* o, const int* sp, int sp_scalar,
+                               int B, int T_, int H, int Hkv, int D, int S_max, cudaStream_t st) {
+  const size_t smem = (size_t)(D + S_max) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(attn_simple_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(B * T_, H);
+  attn_simple_kernel<T><<<grid, 128, smem, st>>>(reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(ck),
+                                                 reinterpret_cast<const T*>(cv), reinterpret_cast<T*>(o), sp, sp_scalar,
+                                                 T_, H, Hkv, D, S_max);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_attn_simple<float>(const void*, const void*, const void*, void*, const int*, int, int,
+                                               int, int, int, int, int, cudaStream_t);
+template cudaError_t launch_attn_simple<bf16>(const void*, const void*, const void*, void*, const int*, int, int, int,
+                                              int, int, int, int, cudaStream_t);
+
+}  // namespace llama

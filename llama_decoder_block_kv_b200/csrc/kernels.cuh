@@ -1,0 +1,54 @@
+// Launchers of the library's kernels (host-side declarations).
+#pragma once
+
+#include "common.cuh"
+
+namespace llama {
+
+// elementwise.cu
+template <typename T>
+void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int* err,
+                  cudaStream_t st);
+template <typename T>
+void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
+                    int in_row_offset, cudaStream_t st);
+template <typename T>
+void launch_pack_w13(const void* w1, const void* w3, void* out, int F, int dim, cudaStream_t st);
+template <typename T>
+void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D, int to_logical, cudaStream_t st);
+
+// gemm_simt.cu
+template <typename T>
+void launch_gemm_simt(const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st);
+
+// gemv.cu
+struct GemvPlan {
+  int row_blocks = 0, S = 1, Kc = 0;
+  size_t part_floats = 0;
+};
+GemvPlan plan_gemv(int M, int N, int K, int num_sms);
+void launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part, int* counters,
+                      const EpiParams& ep, cudaStream_t st);
+
+// gemm_tc.cu
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
+                           cudaStream_t st);
+
+// attention.cu
+struct DecodePlan {
+  int hpc = 1, CK = 256, max_chunks = 1;
+  size_t part_floats = 0;
+};
+DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sms);
+cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
+                                int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max, int* err,
+                                cudaStream_t st);
+cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
+                               const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
+                               const DecodePlan& p, int* err, cudaStream_t st);
+template <typename T>
+cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, void* o, const int* sp, int sp_scalar,
+                               int B, int T_, int H, int Hkv, int D, int S_max, cudaStream_t st);
+
+}  // namespace llama

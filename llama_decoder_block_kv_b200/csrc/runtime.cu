@@ -1,0 +1,613 @@
+// Host runtime and C ABI (include/llama_b200.h): owns the packed weights, the
+// KV-caches, the RoPE table and the workspace, validates every call, and
+// enqueues the kernels of one forward pass on the caller's stream.
+//
+// Per block ("LLaMA: Open and Efficient Foundation Language Models" notes,
+// TransformerBlock.forward):
+//   rmsnorm(h) -> xn
+//   xn * Wqkv^T  -> RoPE(q) -> q buffer; RoPE(k), v -> cache slots       (QKV epilogue)
+//   attention(q, cache) -> o                                             (prefill or split-K decode)
+//   h += o * Wo^T                                                        (residual epilogue)
+//   rmsnorm(h) -> xn
+//   xn * W13^T -> silu(a) * b -> g                                       (SwiGLU epilogue)
+//   h += g * W2^T                                                        (residual epilogue)
+// Whole-model calls add the embedding gather before and the final RMSNorm
+// plus the LM head after ("... notes", Transformer.forward).
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "kernels.cuh"
+
+using namespace llama;
+
+namespace {
+
+struct Layer {
+  void* wqkv = nullptr;
+  void* wo = nullptr;
+  void* w13 = nullptr;
+  void* w2 = nullptr;
+  void* attn_norm = nullptr;
+  void* ffn_norm = nullptr;
+  void* cache_k = nullptr;
+  void* cache_v = nullptr;
+  CUtensorMap map_k, map_v;
+  bool set = false;
+};
+
+}  // namespace
+
+struct llama_ctx {
+  llama_args a;
+  bool bf16 = true;
+  int esz = 2;
+  int dim = 0, H = 0, Hkv = 0, D = 0, n_rep = 1, F = 0, V = 0, S = 0, Bm = 0, L = 0;
+  int n_qkv = 0;
+  int device = 0, num_sms = 148;
+  std::vector<Layer> layers;
+  void* tok_emb = nullptr;
+  void* final_norm = nullptr;
+  void* output = nullptr;
+  bool head_set = false;
+  float2* rope = nullptr;
+  int* err = nullptr;
+  // workspace, sized for ws_tokens tokens
+  int ws_tokens = 0;
+  float* h = nullptr;
+  void* xn = nullptr;
+  void* q = nullptr;
+  void* o = nullptr;
+  void* g = nullptr;
+  // scratch for split-K partial sums (GEMV) and decode-attention partials
+  float* part = nullptr;
+  size_t part_floats = 0;
+  int* counters = nullptr;
+  int counters_n = 0;
+};
+
+namespace {
+
+#define CK(call)                             \
+  do {                                       \
+    cudaError_t e_ = (call);                 \
+    if (e_ != cudaSuccess) return LLAMA_ERR_CUDA; \
+  } while (0)
+
+int alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return LLAMA_OK;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    return LLAMA_ERR_OOM;
+  }
+  return e == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+void release(void*& p) {
+  if (p) cudaFree(p);
+  p = nullptr;
+}
+
+int ffn_hidden(const llama_args* a) {
+  if (a->dim <= 0 || a->multiple_of <= 0) return LLAMA_ERR_INVALID_ARGS;
+  long hidden = 4L * a->dim;
+  hidden = (long)(2.0 * (double)hidden / 3.0);
+  if (a->ffn_dim_multiplier > 0.f) hidden = (long)((double)a->ffn_dim_multiplier * (double)hidden);
+  const long mo = a->multiple_of;
+  hidden = mo * ((hidden + mo - 1) / mo);
+  if (hidden <= 0 || hidden > (1L << 30)) return LLAMA_ERR_INVALID_ARGS;
+  return (int)hidden;
+}
+
+// RoPE angles as the pages' precompute_freqs_cis: freq_i = 1 / theta^(2i/D)
+// (evaluated in double, rounded to fp32), angle = fp32(t) * freq_i (one fp32
+// multiply, like torch.outer on fp32 vectors), cos/sin evaluated in double
+// on that fp32 angle and rounded to fp32. Stored as (cos, sin) pairs.
+std::vector<float2> rope_table(int D, int end, double theta) {
+  std::vector<float2> t((size_t)end * (D / 2));
+  std::vector<float> freq(D / 2);
+  for (int i = 0; i < D / 2; ++i) freq[i] = (float)(1.0 / std::pow(theta, (double)(2 * i) / (double)D));
+  for (int p = 0; p < end; ++p)
+    for (int i = 0; i < D / 2; ++i) {
+      volatile float ang = (float)p * freq[i];
+      t[(size_t)p * (D / 2) + i] = make_float2((float)std::cos((double)ang), (float)std::sin((double)ang));
+    }
+  return t;
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+int reserve(llama_ctx* c, int tokens) {
+  if (tokens <= c->ws_tokens) return LLAMA_OK;
+  cudaDeviceSynchronize();
+  release(reinterpret_cast<void*&>(c->h));
+  release(c->xn);
+  release(c->q);
+  release(c->o);
+  release(c->g);
+  c->ws_tokens = 0;
+  const size_t T = (size_t)tokens;
+  int r;
+  if ((r = alloc(reinterpret_cast<void**>(&c->h), round256(T * c->dim * 4)))) return r;
+  if ((r = alloc(&c->xn, round256(T * c->dim * c->esz)))) return r;
+  if ((r = alloc(&c->q, round256(T * c->H * c->D * c->esz)))) return r;
+  if ((r = alloc(&c->o, round256(T * c->H * c->D * c->esz)))) return r;
+  if ((r = alloc(&c->g, round256(T * c->F * c->esz)))) return r;
+  c->ws_tokens = tokens;
+  return LLAMA_OK;
+}
+
+cudaStream_t S_(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+EpiParams epi_base(llama_ctx* c, int kind, int M, int N) {
+  EpiParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.kind = kind;
+  p.M = M;
+  p.N = N;
+  p.err = c->err;
+  return p;
+}
+
+// C[M][N] = A[M][K] * W[N][K]^T through the path that suits the shape.
+int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st) {
+  if (!c->bf16) {
+    launch_gemm_simt<float>(A, W, M, N, K, ep, st);
+    return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  }
+  if (M <= 32 && K % 32 == 0) {
+    GemvPlan p = plan_gemv(M, N, K, c->num_sms);
+    if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
+    launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, st);
+    return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  }
+  return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
+  Layer& Ly = c->layers[layer];
+  const int M = B * T;
+  const int HD = c->H * c->D;
+  int r;
+  if (c->bf16)
+    launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  else
+    launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+
+  EpiParams e = epi_base(c, EPI_QKV_ROPE, M, c->n_qkv);
+  e.q_out = c->q;
+  e.cache_k = Ly.cache_k;
+  e.cache_v = Ly.cache_v;
+  e.rope = c->rope;
+  e.start_pos = sp_dev;
+  e.start_pos_scalar = sp_host;
+  e.T = T;
+  e.H = c->H;
+  e.Hkv = c->Hkv;
+  e.D = c->D;
+  e.S_max = c->S;
+  if ((r = gemm(c, c->xn, Ly.wqkv, M, c->n_qkv, c->dim, e, st))) return r;
+
+  cudaError_t ce;
+  if (!c->bf16) {
+    ce = launch_attn_simple<float>(c->q, Ly.cache_k, Ly.cache_v, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D,
+                                   c->S, st);
+  } else if (T == 1) {
+    const int max_len = sp_dev ? c->S : sp_host + 1;
+    DecodePlan p = plan_decode(B, c->H, c->Hkv, c->S, max_len, c->num_sms);
+    if (p.part_floats > c->part_floats) return LLAMA_ERR_INVALID_ARGS;
+    ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, sp_dev, sp_host, B, c->H, c->Hkv, c->D, c->S, p,
+                            c->err, st);
+  } else {
+    ce = launch_attn_prefill(Ly.map_k, Ly.map_v, c->q, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D, c->S, c->err,
+                             st);
+  }
+  if (ce != cudaSuccess) return LLAMA_ERR_CUDA;
+
+  e = epi_base(c, EPI_RESIDUAL, M, c->dim);
+  e.out = h;
+  e.ld_out = c->dim;
+  if ((r = gemm(c, c->o, Ly.wo, M, c->dim, HD, e, st))) return r;
+
+  if (c->bf16)
+    launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  else
+    launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+
+  e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
+  e.g_out = c->g;
+  if ((r = gemm(c, c->xn, Ly.w13, M, 2 * c->F, c->dim, e, st))) return r;
+
+  e = epi_base(c, EPI_RESIDUAL, M, c->dim);
+  e.out = h;
+  e.ld_out = c->dim;
+  return gemm(c, c->g, Ly.w2, M, c->dim, c->F, e, st);
+}
+
+// embedding -> blocks -> final norm -> LM head
+int run_model(llama_ctx* c, const int32_t* tokens, int B, int T, const int* sp_dev, int sp_host, float* logits,
+              int all_positions, cudaStream_t st) {
+  if (!c->head_set) return LLAMA_ERR_NOT_READY;
+  for (int l = 0; l < c->L; ++l)
+    if (!c->layers[l].set) return LLAMA_ERR_NOT_READY;
+  const int M = B * T;
+  int r;
+  if ((r = reserve(c, M))) return r;
+  if (c->bf16)
+    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, c->err, st);
+  else
+    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, c->err, st);
+  for (int l = 0; l < c->L; ++l)
+    if ((r = run_block(c, l, c->h, B, T, sp_dev, sp_host, st))) return r;
+  const int rows = all_positions ? M : B;
+  const int stride = all_positions ? 1 : T;
+  const int offset = all_positions ? 0 : T - 1;
+  if (c->bf16)
+    launch_rmsnorm<bf16>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
+  else
+    launch_rmsnorm<float>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
+  EpiParams e = epi_base(c, EPI_STORE_F32, rows, c->V);
+  e.out = logits;
+  e.ld_out = c->V;
+  return gemm(c, c->xn, c->output, rows, c->V, c->dim, e, st);
+}
+
+int check_ctx_call(llama_ctx* c, int B, int T) {
+  if (!c) return LLAMA_ERR_INVALID_ARGS;
+  if (B < 1 || B > c->Bm || T < 1) return LLAMA_ERR_INVALID_ARGS;
+  if (cudaSetDevice(c->device) != cudaSuccess) return LLAMA_ERR_CUDA;
+  return LLAMA_OK;
+}
+
+// private workspace of llama_linear
+float* g_lin_part = nullptr;
+size_t g_lin_part_floats = 0;
+int* g_lin_counters = nullptr;
+int g_lin_counters_n = 0;
+int* g_lin_err = nullptr;
+
+}  // namespace
+
+extern "C" {
+
+int llama_ffn_hidden(const llama_args* a) {
+  if (!a) return LLAMA_ERR_INVALID_ARGS;
+  return ffn_hidden(a);
+}
+
+int llama_create(const llama_args* args, llama_ctx** out) {
+  if (!args || !out) return LLAMA_ERR_INVALID_ARGS;
+  *out = nullptr;
+  llama_args a = *args;
+  if (a.n_kv_heads <= 0) a.n_kv_heads = a.n_heads;
+  if (a.dim <= 0 || a.n_layers <= 0 || a.n_heads <= 0 || a.max_batch_size <= 0 || a.max_seq_len <= 0 ||
+      a.vocab_size < 0 || a.multiple_of <= 0 || !(a.norm_eps >= 0.f) || !(a.rope_theta > 0.f))
+    return LLAMA_ERR_INVALID_ARGS;
+  if (a.dtype != LLAMA_FP32 && a.dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
+  if (a.dim % a.n_heads || a.n_heads % a.n_kv_heads || a.dim % 64) return LLAMA_ERR_INVALID_ARGS;
+  const int D = a.dim / a.n_heads;
+  if (D != 64 && D != 128) return LLAMA_ERR_INVALID_ARGS;
+  const int n_rep = a.n_heads / a.n_kv_heads;
+  if (a.dtype == LLAMA_BF16 && n_rep > 8 && n_rep % 8) return LLAMA_ERR_INVALID_ARGS;
+  const int F = ffn_hidden(&a);
+  if (F < 0 || F % 64) return LLAMA_ERR_INVALID_ARGS;
+  if (a.dtype == LLAMA_FP32 && (size_t)(a.max_seq_len + D) * 4 > 200 * 1024) return LLAMA_ERR_INVALID_ARGS;
+  if (a.vocab_size % 8) return LLAMA_ERR_INVALID_ARGS;
+
+  llama_ctx* c = new llama_ctx();
+  c->a = a;
+  c->bf16 = a.dtype == LLAMA_BF16;
+  c->esz = c->bf16 ? 2 : 4;
+  c->dim = a.dim;
+  c->H = a.n_heads;
+  c->Hkv = a.n_kv_heads;
+  c->D = D;
+  c->n_rep = n_rep;
+  c->F = F;
+  c->V = a.vocab_size;
+  c->S = a.max_seq_len;
+  c->Bm = a.max_batch_size;
+  c->L = a.n_layers;
+  c->n_qkv = (a.n_heads + 2 * a.n_kv_heads) * D;
+  cudaGetDevice(&c->device);
+  cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  c->layers.resize(a.n_layers);
+
+  auto fail = [&](int code) {
+    llama_destroy(c);
+    return code;
+  };
+  int r;
+  const size_t es = c->esz;
+  const size_t wsz = ((size_t)c->n_qkv * c->dim + (size_t)c->dim * c->H * D + 2 * (size_t)F * c->dim +
+                      (size_t)c->dim * F) * es;
+  const size_t cache_elems = (size_t)c->Bm * c->Hkv * c->S * D;
+  for (int l = 0; l < c->L; ++l) {
+    Layer& Ly = c->layers[l];
+    void* blob;
+    if ((r = alloc(&blob, wsz + 2 * round256((size_t)c->dim * es)))) return fail(r);
+    uint8_t* p = reinterpret_cast<uint8_t*>(blob);
+    Ly.wqkv = p;
+    p += (size_t)c->n_qkv * c->dim * es;
+    Ly.wo = p;
+    p += (size_t)c->dim * c->H * D * es;
+    Ly.w13 = p;
+    p += 2 * (size_t)F * c->dim * es;
+    Ly.w2 = p;
+    p += (size_t)c->dim * F * es;
+    Ly.attn_norm = p;
+    p += round256((size_t)c->dim * es);
+    Ly.ffn_norm = p;
+    if ((r = alloc(&Ly.cache_k, cache_elems * es))) return fail(r);
+    if ((r = alloc(&Ly.cache_v, cache_elems * es))) return fail(r);
+    if (cudaMemset(Ly.cache_k, 0, cache_elems * es) != cudaSuccess) return fail(LLAMA_ERR_CUDA);
+    if (cudaMemset(Ly.cache_v, 0, cache_elems * es) != cudaSuccess) return fail(LLAMA_ERR_CUDA);
+    if (c->bf16) {
+      const uint64_t rows = (uint64_t)c->Bm * c->Hkv * c->S;
+      if (!make_tmap_bf16(&Ly.map_k, Ly.cache_k, rows, D, 64) || !make_tmap_bf16(&Ly.map_v, Ly.cache_v, rows, D, 64))
+        return fail(LLAMA_ERR_CUDA);
+    }
+  }
+  if (c->V > 0) {
+    if ((r = alloc(&c->tok_emb, (size_t)c->V * c->dim * es))) return fail(r);
+    if ((r = alloc(&c->final_norm, round256((size_t)c->dim * es)))) return fail(r);
+    if ((r = alloc(&c->output, (size_t)c->V * c->dim * es))) return fail(r);
+  }
+  std::vector<float2> rt = rope_table(D, 2 * c->S, (double)a.rope_theta);
+  if ((r = alloc(reinterpret_cast<void**>(&c->rope), rt.size() * sizeof(float2)))) return fail(r);
+  if (cudaMemcpy(c->rope, rt.data(), rt.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(LLAMA_ERR_CUDA);
+  if ((r = alloc(reinterpret_cast<void**>(&c->err), sizeof(int)))) return fail(r);
+  cudaMemset(c->err, 0, sizeof(int));
+
+  // scratch: GEMV split-K partials for up to 32 tokens and decode-attention partials
+  if (c->bf16) {
+    const int mt = c->Bm < 32 ? c->Bm : 32;
+    const int Ns[5] = {c->n_qkv, c->dim, 2 * F, c->dim, c->V};
+    const int Ks[5] = {c->dim, c->H * D, c->dim, F, c->dim};
+    size_t need = 0;
+    int rbs = 0;
+    for (int i = 0; i < 5; ++i) {
+      if (Ns[i] <= 0) continue;
+      GemvPlan p = plan_gemv(mt, Ns[i], Ks[i], c->num_sms);
+      if (p.part_floats > need) need = p.part_floats;
+      if (p.row_blocks > rbs) rbs = p.row_blocks;
+    }
+    const size_t dec = (size_t)c->Bm * c->H * ((c->S + 127) / 128) * (128 + 2);
+    if (dec > need) need = dec;
+    c->part_floats = need;
+    if ((r = alloc(reinterpret_cast<void**>(&c->part), need * sizeof(float)))) return fail(r);
+    c->counters_n = rbs;
+    if ((r = alloc(reinterpret_cast<void**>(&c->counters), (size_t)rbs * sizeof(int)))) return fail(r);
+    cudaMemset(c->counters, 0, (size_t)rbs * sizeof(int));
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLAMA_ERR_CUDA);
+  *out = c;
+  return LLAMA_OK;
+}
+
+void llama_destroy(llama_ctx* c) {
+  if (!c) return;
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  for (Layer& Ly : c->layers) {
+    release(Ly.wqkv);
+    release(Ly.cache_k);
+    release(Ly.cache_v);
+  }
+  release(c->tok_emb);
+  release(c->final_norm);
+  release(c->output);
+  release(reinterpret_cast<void*&>(c->rope));
+  release(reinterpret_cast<void*&>(c->err));
+  release(reinterpret_cast<void*&>(c->h));
+  release(c->xn);
+  release(c->q);
+  release(c->o);
+  release(c->g);
+  release(reinterpret_cast<void*&>(c->part));
+  release(reinterpret_cast<void*&>(c->counters));
+  delete c;
+}
+
+int llama_set_layer(llama_ctx* c, int layer, const void* wq, const void* wk, const void* wv, const void* wo,
+                    const void* w1, const void* w2, const void* w3, const void* attn_norm, const void* ffn_norm) {
+  if (!c || layer < 0 || layer >= c->L) return LLAMA_ERR_INVALID_ARGS;
+  if (!wq || !wk || !wv || !wo || !w1 || !w2 || !w3 || !attn_norm || !ffn_norm) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  Layer& Ly = c->layers[layer];
+  const size_t es = c->esz;
+  const size_t qb = (size_t)c->H * c->D * c->dim * es, kb = (size_t)c->Hkv * c->D * c->dim * es;
+  uint8_t* p = reinterpret_cast<uint8_t*>(Ly.wqkv);
+  CK(cudaMemcpy(p, wq, qb, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(p + qb, wk, kb, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(p + qb + kb, wv, kb, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(Ly.wo, wo, (size_t)c->dim * c->H * c->D * es, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(Ly.w2, w2, (size_t)c->dim * c->F * es, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(Ly.attn_norm, attn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(Ly.ffn_norm, ffn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
+  if (c->bf16)
+    launch_pack_w13<bf16>(w1, w3, Ly.w13, c->F, c->dim, 0);
+  else
+    launch_pack_w13<float>(w1, w3, Ly.w13, c->F, c->dim, 0);
+  CK(cudaDeviceSynchronize());
+  Ly.set = true;
+  return LLAMA_OK;
+}
+
+int llama_set_embed_norm_head(llama_ctx* c, const void* tok, const void* norm, const void* output) {
+  if (!c || c->V <= 0 || !tok || !norm || !output) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  const size_t es = c->esz;
+  CK(cudaMemcpy(c->tok_emb, tok, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(c->final_norm, norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
+  CK(cudaMemcpy(c->output, output, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
+  CK(cudaDeviceSynchronize());
+  c->head_set = true;
+  return LLAMA_OK;
+}
+
+int llama_reserve(llama_ctx* c, int max_tokens) {
+  if (!c || max_tokens < 1) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  return reserve(c, max_tokens);
+}
+
+int llama_forward(llama_ctx* c, const int32_t* tokens, int B, int T, int start_pos, float* logits, int all_positions,
+                  void* stream) {
+  int r;
+  if ((r = check_ctx_call(c, B, T))) return r;
+  if (!tokens || !logits || start_pos < 0 || (long)start_pos + T > c->S) return LLAMA_ERR_INVALID_ARGS;
+  return run_model(c, tokens, B, T, nullptr, start_pos, logits, all_positions, S_(stream));
+}
+
+int llama_forward_ragged(llama_ctx* c, const int32_t* tokens, const int32_t* start_pos, int B, float* logits,
+                         void* stream) {
+  int r;
+  if ((r = check_ctx_call(c, B, 1))) return r;
+  if (!tokens || !start_pos || !logits) return LLAMA_ERR_INVALID_ARGS;
+  return run_model(c, tokens, B, 1, start_pos, 0, logits, 1, S_(stream));
+}
+
+int llama_block_forward(llama_ctx* c, int layer, float* h, int B, int T, const int32_t* start_pos_dev,
+                        int host_start_pos, void* stream) {
+  int r;
+  if ((r = check_ctx_call(c, B, T))) return r;
+  if (!h || layer < 0 || layer >= c->L) return LLAMA_ERR_INVALID_ARGS;
+  if (!c->layers[layer].set) return LLAMA_ERR_NOT_READY;
+  if (!start_pos_dev && (host_start_pos < 0 || (long)host_start_pos + T > c->S)) return LLAMA_ERR_INVALID_ARGS;
+  if ((r = reserve(c, B * T))) return r;
+  return run_block(c, layer, h, B, T, start_pos_dev, host_start_pos, S_(stream));
+}
+
+int llama_kv_read(llama_ctx* c, int layer, void* k, void* v, void* stream) {
+  if (!c || layer < 0 || layer >= c->L || !k || !v) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  Layer& Ly = c->layers[layer];
+  if (c->bf16) {
+    launch_kv_convert<bf16>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+    launch_kv_convert<bf16>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+  } else {
+    launch_kv_convert<float>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+    launch_kv_convert<float>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+  }
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int llama_kv_write(llama_ctx* c, int layer, const void* k, const void* v, void* stream) {
+  if (!c || layer < 0 || layer >= c->L || !k || !v) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  Layer& Ly = c->layers[layer];
+  if (c->bf16) {
+    launch_kv_convert<bf16>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+    launch_kv_convert<bf16>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+  } else {
+    launch_kv_convert<float>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+    launch_kv_convert<float>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+  }
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int llama_reset(llama_ctx* c) {
+  if (!c) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  const size_t bytes = (size_t)c->Bm * c->Hkv * c->S * c->D * c->esz;
+  for (Layer& Ly : c->layers) {
+    CK(cudaMemset(Ly.cache_k, 0, bytes));
+    CK(cudaMemset(Ly.cache_v, 0, bytes));
+  }
+  CK(cudaDeviceSynchronize());
+  return LLAMA_OK;
+}
+
+int llama_get_error(llama_ctx* c, int* flags) {
+  if (flags) *flags = 0;
+  if (!c) return LLAMA_ERR_INVALID_ARGS;
+  CK(cudaSetDevice(c->device));
+  if (cudaDeviceSynchronize() != cudaSuccess) return LLAMA_ERR_CUDA;
+  int f = 0;
+  CK(cudaMemcpy(&f, c->err, sizeof(int), cudaMemcpyDeviceToHost));
+  CK(cudaMemset(c->err, 0, sizeof(int)));
+  if (flags) *flags = f;
+  if (f & LLAMA_DEV_TIMEOUT) return LLAMA_ERR_TIMEOUT;
+  if (f & LLAMA_DEV_POS_RANGE) return LLAMA_ERR_POS_RANGE;
+  if (f & LLAMA_DEV_TOKEN_RANGE) return LLAMA_ERR_TOKEN_RANGE;
+  return LLAMA_OK;
+}
+
+const char* llama_strerror(int code) {
+  switch (code) {
+    case LLAMA_OK: return "ok";
+    case LLAMA_ERR_INVALID_ARGS: return "invalid arguments";
+    case LLAMA_ERR_OOM: return "device out of memory";
+    case LLAMA_ERR_CUDA: return "CUDA error";
+    case LLAMA_ERR_NOT_READY: return "weights not set";
+    case LLAMA_ERR_TOKEN_RANGE: return "token id outside [0, vocab_size)";
+    case LLAMA_ERR_POS_RANGE: return "position outside [0, max_seq_len)";
+    case LLAMA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    default: return "unknown error";
+  }
+}
+
+int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, int dtype, int path, void* stream) {
+  if (!x || !w || !y || M <= 0 || N <= 0 || K <= 0 || N % 8 || K % 8) return LLAMA_ERR_INVALID_ARGS;
+  if (dtype != LLAMA_FP32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (path == LLAMA_PATH_AUTO) path = dtype == LLAMA_FP32 ? LLAMA_PATH_SIMT : (M <= 32 && K % 32 == 0 ? LLAMA_PATH_GEMV : LLAMA_PATH_TCGEN05);
+  if (!g_lin_err) {
+    if (alloc(reinterpret_cast<void**>(&g_lin_err), sizeof(int))) return LLAMA_ERR_OOM;
+    cudaMemset(g_lin_err, 0, sizeof(int));
+  }
+  EpiParams e;
+  std::memset(&e, 0, sizeof(e));
+  e.kind = EPI_STORE_F32;
+  e.M = M;
+  e.N = N;
+  e.out = y;
+  e.ld_out = N;
+  e.err = g_lin_err;
+  cudaStream_t st = S_(stream);
+  switch (path) {
+    case LLAMA_PATH_SIMT:
+      if (dtype == LLAMA_FP32)
+        launch_gemm_simt<float>(x, w, M, N, K, e, st);
+      else
+        launch_gemm_simt<bf16>(x, w, M, N, K, e, st);
+      break;
+    case LLAMA_PATH_GEMV: {
+      if (dtype != LLAMA_BF16 || M > 32 || K % 32) return LLAMA_ERR_INVALID_ARGS;
+      GemvPlan p = plan_gemv(M, N, K, sms);
+      if (p.part_floats > g_lin_part_floats) {
+        cudaDeviceSynchronize();
+        release(reinterpret_cast<void*&>(g_lin_part));
+        g_lin_part_floats = 0;
+        if (alloc(reinterpret_cast<void**>(&g_lin_part), p.part_floats * sizeof(float))) return LLAMA_ERR_OOM;
+        g_lin_part_floats = p.part_floats;
+      }
+      if (p.row_blocks > g_lin_counters_n) {
+        cudaDeviceSynchronize();
+        release(reinterpret_cast<void*&>(g_lin_counters));
+        g_lin_counters_n = 0;
+        if (alloc(reinterpret_cast<void**>(&g_lin_counters), (size_t)p.row_blocks * sizeof(int))) return LLAMA_ERR_OOM;
+        cudaMemset(g_lin_counters, 0, (size_t)p.row_blocks * sizeof(int));
+        g_lin_counters_n = p.row_blocks;
+      }
+      launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, st);
+      break;
+    }
+    case LLAMA_PATH_TCGEN05:
+      if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
+      if (launch_gemm_tc(x, w, M, N, K, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+      break;
+    default:
+      return LLAMA_ERR_INVALID_ARGS;
+  }
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+"""Shared set-up for the GPU parity tests: load synth weights into the library
+and into the oracle, and compare results (tolerances stated once here)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from llama_decoder_block_kv_b200 import binding as B
+from llama_decoder_block_kv_b200 import synth
+from tests.helpers import build_oracle, t2np
+
+# Tolerances: fp32 mode max relative error 1e-4 (norm-wise and element-wise
+# with a small absolute floor); bf16 mode max absolute error 2e-2 on hidden
+# states and 5e-2 on logits, fp32 accumulation on both sides.
+FP32_REL = 1e-4
+BF16_HIDDEN_ABS = 2e-2
+BF16_LOGITS_ABS = 5e-2
+
+
+def assert_fp32_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    scale = np.abs(ref).max()
+    err = np.abs(got - ref)
+    assert err.max() <= FP32_REL * scale, f"{what}: norm-wise rel err {err.max() / scale:.3g}"
+    assert np.all(err <= FP32_REL * np.abs(ref) + FP32_REL * 1e-2 * scale + 1e-6), f"{what}: element-wise"
+
+
+def assert_abs_close(got: np.ndarray, ref: np.ndarray, tol: float, what: str = ""):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref).max()
+    assert err <= tol, f"{what}: max abs err {err:.4g} > {tol}"
+
+
+class Pair:
+    """The same synthetic model loaded into the CUDA library and the oracle."""
+
+    def __init__(self, w: synth.Workload, layers=None, bits: bool = False, weights_device="cpu"):
+        self.w = w
+        self.args = B.ModelArgs.from_workload(w)
+        self.model = B.Llama(self.args)
+        n = w.n_layers if layers is None else layers
+        lws = []
+        for i in range(n):
+            lw = synth.layer_weights(w, i, device=weights_device)
+            B.llama_set_layer(self.model.ctx, i, {k: v.to("cuda").contiguous() for k, v in lw.items()})
+            lws.append({k: v.cpu() for k, v in lw.items()})
+        enh = None
+        if w.vocab_size > 0:
+            enh = synth.embed_norm_head(w, device=weights_device)
+            B.llama_set_embed_norm_head(self.model.ctx, *(enh[k].to("cuda").contiguous()
+                                                          for k in ("tok_embeddings", "norm", "output")))
+            enh = {k: v.cpu() for k, v in enh.items()}
+        self.oracle = build_oracle(w, lws, enh, bits=bits)
+        torch.cuda.synchronize()
+
+    @property
+    def ctx(self):
+        return self.model.ctx
+
+    def check_error(self):
+        code, flags = B.llama_get_error(self.ctx)
+        assert code == B.LLAMA_OK, (B.strerror(code), flags)
+
+    def kv(self, layer: int):
+        w = self.w
+        dt = torch.float32 if w.act == "fp32" else torch.bfloat16
+        shape = (w.max_batch_size, w.max_seq_len, w.n_kv_heads, w.head_dim)
+        k = torch.empty(shape, dtype=dt, device="cuda")
+        v = torch.empty(shape, dtype=dt, device="cuda")
+        B.llama_kv_read(self.ctx, layer, k, v)
+        torch.cuda.synchronize()
+        return t2np(k), t2np(v)
+
+    def close(self):
+        self.model.close()
+
+
+def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float):
+    """written: bool [B_max, S_max] of slots this test wrote; others must still be 0 (bit-exact),
+    written ones match the oracle within tol (fp32: relative)."""
+    k, v = pair.kv(layer)
+    ok_, ov_ = pair.oracle.cache_k[layer], pair.oracle.cache_v[layer]
+    for got, ref, name in ((k, ok_, "K"), (v, ov_, "V")):
+        untouched = ~written
+        assert np.all(got[untouched] == 0.0), f"cache {name} layer {layer}: a slot outside the written ones changed"
+        nz = np.any(got != 0.0, axis=(2, 3))
+        assert np.all(nz[written]), f"cache {name} layer {layer}: a written slot is still zero"
+        if pair.w.act == "fp32":
+            assert_fp32_close(got[written], ref[written], f"cache {name}")
+        else:
+            assert_abs_close(got[written], ref[written], tol, f"cache {name}")

@@ -1,0 +1,128 @@
+"""One decoder block (llama_block_forward) against the oracle at sizes that span
+several tiles and ragged tails: prefill (tcgen05 GEMMs + flash prefill),
+chunked prefill at start_pos > 0, decode (GEMV + split-K decode attention)
+with scalar and per-sequence positions, and the cache slots written."""
+import numpy as np
+import pytest
+import torch
+
+from llama_decoder_block_kv_b200 import binding as B
+from llama_decoder_block_kv_b200 import synth
+from tests.gpu_util import BF16_HIDDEN_ABS, Pair, assert_abs_close, assert_cache_matches, assert_fp32_close
+from tests.helpers import t2np
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(dim, H, Hkv, act="bf16", Bm=2, S=256, mo=256, seed=5):
+    F = O.ffn_hidden_dim(dim, mo)
+    return synth.Workload(name=f"block dim {dim} H {H}/{Hkv}", dim=dim, n_layers=1, n_heads=H, n_kv_heads=Hkv,
+                          ffn_hidden=F, vocab_size=0, multiple_of=mo, ffn_dim_multiplier=None, norm_eps=1e-5,
+                          rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act=act, batch=Bm, seed=seed)
+
+
+def _run(pair: Pair, h: torch.Tensor, start_pos, tol_hidden):
+    """One block call on both sides; returns the library's output."""
+    hd = h.to("cuda").contiguous()
+    sp = start_pos
+    if isinstance(start_pos, np.ndarray):
+        sp = torch.from_numpy(start_pos.astype(np.int32)).to("cuda")
+    B.llama_block_forward(pair.ctx, 0, hd, sp)
+    torch.cuda.synchronize()
+    pair.check_error()
+    ref = pair.oracle.block(0, t2np(h), start_pos)
+    got = t2np(hd)
+    if pair.w.act == "fp32":
+        assert_fp32_close(got, ref, "hidden")
+    else:
+        assert_abs_close(got, ref, tol_hidden, "hidden")
+    return got
+
+
+@pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 2), (512, 4, 4), (256, 4, 1), (1024, 8, 1), (1024, 8, 8)])
+def test_block_prefill_chunk_and_decode(dim, H, Hkv):
+    w = _wl(dim, H, Hkv)
+    pair = Pair(w)
+    try:
+        Bsz = 2
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        # prefill 77 tokens (ragged: 64 + 13), then a chunk of 40 at start_pos 77
+        h = synth.hidden(w, (Bsz, 77, dim), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        written[:Bsz, :77] = True
+        h = synth.hidden(w, (Bsz, 40, dim), call=1)
+        _run(pair, h, 77, BF16_HIDDEN_ABS)
+        written[:Bsz, 77:117] = True
+        # three decode steps with a scalar position
+        for i in range(3):
+            h = synth.hidden(w, (Bsz, 1, dim), call=2 + i)
+            _run(pair, h, 117 + i, BF16_HIDDEN_ABS)
+            written[:Bsz, 117 + i] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+def test_block_ragged_decode_positions():
+    w = _wl(512, 4, 2, Bm=4, S=512)
+    pair = Pair(w)
+    try:
+        lens = np.array([7, 300, 64, 129])
+        # fill each sequence's history with one prefill at its own length (T differs -> separate calls
+        # would need B=1; use the device-position path with T=1 after a shared prefill instead)
+        h = synth.hidden(w, (4, 7, 512), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        # sequences advance to different lengths by chunked prefill of sequence-specific sizes is not
+        # expressible in one call; emulate ragged histories with per-sequence positions for T = 1:
+        pos = np.array([7, 7, 7, 7])
+        for step in range(4):
+            h = synth.hidden(w, (4, 1, 512), call=10 + step)
+            _run(pair, h, pos, BF16_HIDDEN_ABS)
+            pos = pos + np.array([1, 50, 20, 30])   # jump ahead: skipped slots stay zero on both sides
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:4, :7] = True
+        p = np.array([7, 7, 7, 7])
+        for step in range(4):
+            for b in range(4):
+                written[b, p[b]] = True
+            p = p + np.array([1, 50, 20, 30])
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+def test_block_fp32_mode():
+    w = _wl(256, 4, 2, act="fp32", S=64)
+    pair = Pair(w)
+    try:
+        h = synth.hidden(w, (2, 33, 256), call=0)
+        _run(pair, h, 0, None)
+        h = synth.hidden(w, (2, 1, 256), call=1)
+        _run(pair, h, 33, None)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:2, :34] = True
+        assert_cache_matches(pair, 0, written, None)
+    finally:
+        pair.close()
+
+
+def test_position_past_cache_raises_device_flag():
+    w = _wl(512, 4, 2, Bm=2, S=128)
+    pair = Pair(w)
+    try:
+        h = torch.zeros((2, 1, 512), device="cuda")
+        sp = torch.tensor([5, 128], dtype=torch.int32, device="cuda")
+        B.llama_block_forward(pair.ctx, 0, h, sp)
+        code, flags = B.llama_get_error(pair.ctx)
+        assert code == B.LLAMA_ERR_POS_RANGE and flags & 2
+        # the flag clears after it has been read
+        assert B.llama_get_error(pair.ctx)[0] == B.LLAMA_OK
+        # host-checked scalar positions are rejected before any launch
+        with pytest.raises(B.LlamaError) as e:
+            B.llama_block_forward(pair.ctx, 0, torch.zeros((2, 4, 512), device="cuda"), 126)
+        assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
+        with pytest.raises(B.LlamaError):
+            B.llama_block_forward(pair.ctx, 0, torch.zeros((3, 1, 512), device="cuda"), 0)  # B > max_batch
+    finally:
+        pair.close()

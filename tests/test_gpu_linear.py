@@ -1,0 +1,55 @@
+"""GEMM cores through the C ABI (llama_linear) against a float64 matmul of the
+same bf16 / fp32 inputs (the library primitive the oracle uses for a linear)."""
+import numpy as np
+import pytest
+import torch
+
+from llama_decoder_block_kv_b200 import binding as B
+from llama_decoder_block_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(M, N, K, dtype, seed):
+    x = synth.normal((M, K), 1.0, seed, dtype, "cuda")
+    w = synth.normal((N, K), 0.02, seed + 1, dtype, "cuda")
+    return x, w
+
+
+def _check(x, w, y, rel=2e-5):
+    ref = x.double().cpu().numpy() @ w.double().cpu().numpy().T
+    got = y.double().cpu().numpy()
+    err = np.abs(got - ref).max()
+    scale = np.abs(ref).max()
+    assert err <= rel * scale + 1e-6, (err, scale)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (37, 384, 128), (128, 256, 4096), (129, 512, 448),
+                                   (300, 1024, 1024), (512, 12288, 4096), (77, 128, 11008), (2, 2048, 256)])
+def test_tcgen05_gemm(M, N, K):
+    x, w = _inputs(M, N, K, torch.bfloat16, 11)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    B.llama_linear(x, w, y, B.LLAMA_PATH_TCGEN05)
+    torch.cuda.synchronize()
+    _check(x, w, y)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (5, 384, 4096), (8, 4096, 4096), (16, 12288, 4096),
+                                   (17, 256, 11008), (32, 4096, 14336), (32, 28672, 4096), (3, 136, 96)])
+def test_gemv_split_k(M, N, K):
+    x, w = _inputs(M, N, K, torch.bfloat16, 21)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    for _ in range(2):  # the second call checks that the split-K counters were re-armed
+        B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+    torch.cuda.synchronize()
+    _check(x, w, y)
+
+
+@pytest.mark.parametrize("M,N,K,dt", [(33, 136, 200, torch.float32), (64, 64, 64, torch.float32),
+                                      (5, 256, 96, torch.bfloat16)])
+def test_simt_gemm(M, N, K, dt):
+    x, w = _inputs(M, N, K, dt, 31)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    B.llama_linear(x, w, y, B.LLAMA_PATH_SIMT)
+    torch.cuda.synchronize()
+    _check(x, w, y, rel=1e-5)
