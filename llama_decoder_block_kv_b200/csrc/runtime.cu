@@ -365,7 +365,7 @@ int llama_create(const llama_args* args, llama_ctx** out) {
 
   // scratch: GEMV split-K partials for up to 32 tokens and decode-attention partials
   if (c->bf16) {
-    const int mt = c->Bm < 32 ? c->Bm : 32;
+    const int mt = 32;  // the GEMV path serves any call of up to 32 tokens (B * T)
     const int Ns[5] = {c->n_qkv, c->dim, 2 * F, c->dim, c->V};
     const int Ks[5] = {c->dim, c->H * D, c->dim, F, c->dim};
     size_t need = 0;

@@ -1,0 +1,81 @@
+"""Run one kernel case repeatedly (for profilers and quick timing).
+
+  python -m llama_decoder_block_kv_b200.profile_case gemv M N K [--reps R]
+  python -m llama_decoder_block_kv_b200.profile_case tc   M N K [--reps R]
+  python -m llama_decoder_block_kv_b200.profile_case simt M N K [--reps R]
+  python -m llama_decoder_block_kv_b200.profile_case prefill-attn T   (LLaMA-7B layer shape, one block call)
+  python -m llama_decoder_block_kv_b200.profile_case decode-attn B L  (LLaMA-2-70B layer shape, one block call)
+
+GEMM cases call llama_linear on seeded bf16 inputs; the block cases call
+llama_block_forward. Prints the mean CUDA-event time per launch.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import binding as B
+from . import synth
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kind", choices=["gemv", "tc", "simt", "prefill-attn", "decode-attn"])
+    ap.add_argument("sizes", type=int, nargs="+")
+    ap.add_argument("--reps", type=int, default=5)
+    a = ap.parse_args()
+    torch.cuda.set_device(0)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if a.kind in ("gemv", "tc", "simt"):
+        M, N, K = a.sizes
+        x = synth.normal((M, K), 1.0, 1, torch.bfloat16, "cuda")
+        w = synth.normal((N, K), 0.02, 2, torch.bfloat16, "cuda")
+        y = torch.empty((M, N), device="cuda")
+        path = {"gemv": B.LLAMA_PATH_GEMV, "tc": B.LLAMA_PATH_TCGEN05, "simt": B.LLAMA_PATH_SIMT}[a.kind]
+        B.llama_linear(x, w, y, path)
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(a.reps):
+            B.llama_linear(x, w, y, path)
+        e1.record(st)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / a.reps
+        flops = 2.0 * M * N * K
+        byts = 2.0 * (M * K + N * K) + 4.0 * M * N
+        print(f"{a.kind} M={M} N={N} K={K}: {ms * 1e3:.1f} us/launch, {flops / ms / 1e9:.1f} TFLOP/s, "
+              f"{byts / ms / 1e6:.1f} GB/s")
+        return
+    if a.kind == "prefill-attn":
+        w = synth.LLAMA7B_LAYER
+        T = a.sizes[0]
+        m = B.Llama(B.ModelArgs.from_workload(w))
+        B.llama_set_layer(m.ctx, 0, synth.layer_weights(w, 0, device="cuda"))
+        h0 = synth.hidden(w, (1, T, w.dim), 0, "cuda")
+        pos = 0
+    else:
+        w = synth.LLAMA70B_LAYER
+        Bsz, L = a.sizes
+        m = B.Llama(B.ModelArgs.from_workload(w.with_(max_batch_size=Bsz)))
+        B.llama_set_layer(m.ctx, 0, synth.layer_weights(w, 0, device="cuda"))
+        h0 = synth.hidden(w, (Bsz, 1, w.dim), 0, "cuda")
+        pos = L
+    h = h0.clone()
+    B.llama_block_forward(m.ctx, 0, h, pos)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(a.reps):
+        h.copy_(h0)
+        B.llama_block_forward(m.ctx, 0, h, pos)
+    e1.record(st)
+    e1.synchronize()
+    print(f"{a.kind} {a.sizes}: {e0.elapsed_time(e1) / a.reps * 1e3:.1f} us per block call")
+    code, flags = B.llama_get_error(m.ctx)
+    m.close()
+    if code != B.LLAMA_OK:
+        raise SystemExit(f"device flag: {B.strerror(code)}")
+
+
+if __name__ == "__main__":
+    main()

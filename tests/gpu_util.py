@@ -88,3 +88,53 @@ def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float
             assert_fp32_close(got[written], ref[written], f"cache {name}")
         else:
             assert_abs_close(got[written], ref[written], tol, f"cache {name}")
+
+
+# ----------------------------------------------------------------------------- conditioning floor
+#
+# The bf16 rounding points (norm outputs, q/k/v, attention output, silu*mul)
+# make the block ill-conditioned at its full sizes: the oracle itself moves
+# by ~0.03 (LLaMA-7B layer) to ~0.08 (LLaMA-2-70B layer) in max-abs when its
+# input hidden states are perturbed by one fp32 rounding (relative 2^-24),
+# because a tiny change flips a few bf16 roundings and the flips fan out
+# through 11008 / 28672-wide sums. No fp32-accumulating implementation can be
+# held below that. At those sizes the hidden-state check is therefore: the
+# 99th percentile of |error| within the 2e-2 bound, and the maximum within
+# max(2e-2, 2 x the oracle's own floor on the same inputs).
+
+PERTURB_REL = 2.0 ** -24
+
+
+def oracle_floor(run, h: np.ndarray, seed: int = 0):
+    """(run(h), max |run(h) - run(h * (1 + 2^-24 r))|), r ~ N(0, 1).
+
+    ``run`` must start from the same state each call; the unperturbed run is made
+    last so the oracle's caches end in the unperturbed state."""
+    r = np.random.default_rng(seed).standard_normal(h.shape)
+    pert = run(h * (1.0 + PERTURB_REL * r))
+    ref = run(h)
+    return ref, float(np.abs(ref - pert).max())
+
+
+def assert_hidden_close_floor(got: np.ndarray, ref: np.ndarray, floor: float, what: str = ""):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    p99 = float(np.quantile(err, 0.99))
+    tol = max(BF16_HIDDEN_ABS, 2.0 * floor)
+    assert p99 <= BF16_HIDDEN_ABS, f"{what}: p99 abs err {p99:.4g} > {BF16_HIDDEN_ABS}"
+    assert err.max() <= tol, f"{what}: max abs err {err.max():.4g} > {tol:.4g} (oracle floor {floor:.4g})"
+    return float(err.max()), p99
+
+
+class CacheSnapshot:
+    """Save and restore an oracle's caches (so a perturbed run starts from the same state)."""
+
+    def __init__(self, model, layers):
+        self.model, self.layers = model, list(layers)
+        self.k = [model.cache_k[i].copy() for i in self.layers]
+        self.v = [model.cache_v[i].copy() for i in self.layers]
+
+    def restore(self):
+        for j, i in enumerate(self.layers):
+            self.model.cache_k[i][...] = self.k[j]
+            self.model.cache_v[i][...] = self.v[j]
