@@ -201,7 +201,7 @@ const char* llama_strerror(int code);
  * Diagnostics: y_dev[M][N] (fp32) = x_dev[M][K] * w_dev[N][K]^T with fp32
  * accumulation, x and w both of storage type dtype, through the chosen GEMM
  * path (LLAMA_PATH_*). Rules: M, N, K > 0, N % 8 == 0, K % 8 == 0;
- * LLAMA_PATH_GEMV needs M <= 32 and K % 32 == 0; LLAMA_PATH_TCGEN05 needs
+ * LLAMA_PATH_GEMV needs M <= 32 and K % 64 == 0; LLAMA_PATH_TCGEN05 needs
  * dtype == LLAMA_BF16. Uses a private, lazily allocated workspace; not
  * thread-safe.
  */

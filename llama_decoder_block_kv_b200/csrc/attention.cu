@@ -392,8 +392,13 @@ __global__ void __launch_bounds__(160)
         l0 += s[jn][0] + s[jn][1];
         l1 += s[jn][2] + s[jn][3];
       }
-      const uint32_t pa[4] = {pack_bf16x2(s[0][0], s[0][1]), pack_bf16x2(s[0][2], s[0][3]),
-                              pack_bf16x2(s[1][0], s[1][1]), pack_bf16x2(s[1][2], s[1][3])};
+      // P as a sum of two bf16 parts (hi + lo): the decode kernel is bound by
+      // the cache stream, so the second MMA is free and P keeps ~16 bits.
+      uint32_t ph[4], pl[4];
+      split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
+      split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
+      split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
+      split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
 #pragma unroll
       for (int jd = 0; jd < D / 8; jd += 2) {
         const int mi = lane >> 3;
@@ -402,8 +407,10 @@ __global__ void __launch_bounds__(160)
         uint32_t bf[4];
         ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
         const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-        mma_bf16_16816(oacc[jd], pa, b0);
-        mma_bf16_16816(oacc[jd + 1], pa, b1);
+        mma_bf16_16816(oacc[jd], ph, b0);
+        mma_bf16_16816(oacc[jd], pl, b0);
+        mma_bf16_16816(oacc[jd + 1], ph, b1);
+        mma_bf16_16816(oacc[jd + 1], pl, b1);
       }
     }
     __syncwarp();

@@ -47,6 +47,13 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
+// (a, b) = hi + lo with hi = bf16(a, b) and lo = bf16 of the remainders
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  const float2 h = unpack_bf16x2(hi);
+  lo = pack_bf16x2(a - h.x, b - h.y);
+}
+
 // store 8 consecutive values (fp32 in registers) to storage type T
 __device__ __forceinline__ void store8(float* dst, const float* v) {
   float4* d = reinterpret_cast<float4*>(dst);

@@ -27,8 +27,8 @@ struct GemvPlan {
   size_t part_floats = 0;
 };
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
-void launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part, int* counters,
-                      const EpiParams& ep, cudaStream_t st);
+cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
+                             int* counters, const EpiParams& ep, cudaStream_t st);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

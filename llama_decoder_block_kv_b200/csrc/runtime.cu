@@ -158,11 +158,11 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
     launch_gemm_simt<float>(A, W, M, N, K, ep, st);
     return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
   }
-  if (M <= 32 && K % 32 == 0) {
+  if (M <= 32 && K % 64 == 0) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, st);
-    return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+    return launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, st) == cudaSuccess ? LLAMA_OK
+                                                                                          : LLAMA_ERR_CUDA;
   }
   return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
@@ -558,7 +558,8 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (path == LLAMA_PATH_AUTO) path = dtype == LLAMA_FP32 ? LLAMA_PATH_SIMT : (M <= 32 && K % 32 == 0 ? LLAMA_PATH_GEMV : LLAMA_PATH_TCGEN05);
+  if (path == LLAMA_PATH_AUTO)
+    path = dtype == LLAMA_FP32 ? LLAMA_PATH_SIMT : (M <= 32 && K % 64 == 0 ? LLAMA_PATH_GEMV : LLAMA_PATH_TCGEN05);
   if (!g_lin_err) {
     if (alloc(reinterpret_cast<void**>(&g_lin_err), sizeof(int))) return LLAMA_ERR_OOM;
     cudaMemset(g_lin_err, 0, sizeof(int));
@@ -580,7 +581,7 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
         launch_gemm_simt<bf16>(x, w, M, N, K, e, st);
       break;
     case LLAMA_PATH_GEMV: {
-      if (dtype != LLAMA_BF16 || M > 32 || K % 32) return LLAMA_ERR_INVALID_ARGS;
+      if (dtype != LLAMA_BF16 || M > 32 || K % 64) return LLAMA_ERR_INVALID_ARGS;
       GemvPlan p = plan_gemv(M, N, K, sms);
       if (p.part_floats > g_lin_part_floats) {
         cudaDeviceSynchronize();
@@ -597,7 +598,7 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
         cudaMemset(g_lin_counters, 0, (size_t)p.row_blocks * sizeof(int));
         g_lin_counters_n = p.row_blocks;
       }
-      launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, st);
+      if (launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, st) != cudaSuccess) return LLAMA_ERR_CUDA;
       break;
     }
     case LLAMA_PATH_TCGEN05:

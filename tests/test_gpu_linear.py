@@ -35,7 +35,7 @@ def test_tcgen05_gemm(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 256), (5, 384, 4096), (8, 4096, 4096), (16, 12288, 4096),
-                                   (17, 256, 11008), (32, 4096, 14336), (32, 28672, 4096), (3, 136, 96)])
+                                   (17, 256, 11008), (32, 4096, 14336), (32, 28672, 4096), (3, 136, 192), (9, 8, 128)])
 def test_gemv_split_k(M, N, K):
     x, w = _inputs(M, N, K, torch.bfloat16, 21)
     y = torch.full((M, N), float("nan"), device="cuda")
