@@ -228,6 +228,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   }
 }
 
+// Bounded wait that also gives up as soon as another role of the CTA has given
+// up (abort_flag in shared memory), so one timeout unwinds the whole CTA quickly.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > LLAMA_WAIT_LIMIT_NS) {
+      atomicOr(err, LLAMA_DEV_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 // 2-D tiled TMA load (no multicast) into this CTA's shared memory, completing
 // on an mbarrier with a transaction-byte count.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {

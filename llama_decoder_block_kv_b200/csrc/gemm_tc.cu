@@ -43,21 +43,6 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n) 
   return {first_m + local % gm, local / gm};
 }
 
-// Bounded wait that also gives up as soon as another role has given up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > LLAMA_WAIT_LIMIT_NS) {
-      atomicOr(err, LLAMA_DEV_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
 template <typename T, int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M, int N,

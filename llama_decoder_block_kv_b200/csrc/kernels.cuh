@@ -23,12 +23,12 @@ void launch_gemm_simt(const void* A, const void* W, int M, int N, int K, const E
 
 // gemv.cu
 struct GemvPlan {
-  int row_blocks = 0, S = 1, Kc = 0;
+  int row_blocks = 0, nk = 0, total = 0, grid = 1, S = 1;  // S = most CTAs sharing one row block
   size_t part_floats = 0;
 };
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
-                             int* counters, const EpiParams& ep, cudaStream_t st);
+                             int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -161,7 +161,7 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
   if (M <= 32 && K % 64 == 0) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, st) == cudaSuccess ? LLAMA_OK
+    return launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK
                                                                                           : LLAMA_ERR_CUDA;
   }
   return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -372,9 +372,11 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     int rbs = 0;
     for (int i = 0; i < 5; ++i) {
       if (Ns[i] <= 0) continue;
-      GemvPlan p = plan_gemv(mt, Ns[i], Ks[i], c->num_sms);
-      if (p.part_floats > need) need = p.part_floats;
-      if (p.row_blocks > rbs) rbs = p.row_blocks;
+      for (int m = 1; m <= mt; ++m) {
+        GemvPlan p = plan_gemv(m, Ns[i], Ks[i], c->num_sms);
+        if (p.part_floats > need) need = p.part_floats;
+        if (p.row_blocks > rbs) rbs = p.row_blocks;
+      }
     }
     const size_t dec = (size_t)c->Bm * c->H * ((c->S + 127) / 128) * (128 + 2);
     if (dec > need) need = dec;
@@ -598,7 +600,8 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
         cudaMemset(g_lin_counters, 0, (size_t)p.row_blocks * sizeof(int));
         g_lin_counters_n = p.row_blocks;
       }
-      if (launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+      if (launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, sms, st) != cudaSuccess)
+        return LLAMA_ERR_CUDA;
       break;
     }
     case LLAMA_PATH_TCGEN05:
