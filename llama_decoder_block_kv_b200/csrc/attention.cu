@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(288, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -276,6 +278,8 @@ __global__ void __launch_bounds__(160)
   const int b = z / (Hkv * groups);
   const int kvh = (z / groups) % Hkv;
   const int grp = z % groups;
+  pdl_trigger();
+  pdl_wait();
   const int sp = start_pos ? start_pos[b] : sp_scalar;
   const int L = min(sp + 1, S_max);  // keys 0 .. sp
   const int k_begin = chunk * CK;
@@ -293,6 +297,8 @@ __global__ void __launch_bounds__(160)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 4) {
     if (lane == 0) {
@@ -464,6 +470,8 @@ __global__ void __launch_bounds__(160)
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                            bf16* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar,
                                            int H, int D, int S_max, int CK, int max_chunks) {
+  pdl_trigger();
+  pdl_wait();
   const int bh = blockIdx.x;
   const int b = bh / H;
   const int sp = start_pos ? start_pos[b] : sp_scalar;
@@ -488,6 +496,8 @@ template <typename T>
 __global__ void attn_simple_kernel(const T* __restrict__ q, const T* __restrict__ ck, const T* __restrict__ cv,
                                    T* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar, int T_, int H,
                                    int Hkv, int D, int S_max) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float sm[];
   float* qs = sm;             // [D]
   float* sc = sm + D;         // [S_max]
@@ -558,9 +568,8 @@ static cudaError_t prefill_d(const CUtensorMap& mk, const CUtensorMap& mv, const
     attr = true;
   }
   dim3 grid((T + BQ - 1) / BQ, B * Hkv * (n_rep / hpc));
-  attn_prefill_kernel<D><<<grid, 288, smem, st>>>(mk, mv, reinterpret_cast<const bf16*>(q), reinterpret_cast<bf16*>(o),
-                                                  sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
-  return cudaGetLastError();
+  return launch_pdl(attn_prefill_kernel<D>, grid, dim3(288), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
+                    reinterpret_cast<bf16*>(o), sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
 }
 
 cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
@@ -602,11 +611,12 @@ static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
   float* part_o = part;
   float* part_ml = part + (size_t)B * H * p.max_chunks * D;
   dim3 grid(p.max_chunks, B * Hkv * (n_rep / p.hpc));
-  attn_decode_kernel<D><<<grid, 160, smem, st>>>(mk, mv, reinterpret_cast<const bf16*>(q), part_o, part_ml, sp,
-                                                 sp_scalar, H, Hkv, S_max, p.hpc, p.CK, p.max_chunks, err);
-  attn_decode_combine_kernel<<<B * H, D, 0, st>>>(part_o, part_ml, reinterpret_cast<bf16*>(o), sp, sp_scalar, H, D,
-                                                  S_max, p.CK, p.max_chunks);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(attn_decode_kernel<D>, grid, dim3(160), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
+                             part_o, part_ml, sp, sp_scalar, H, Hkv, S_max, p.hpc, p.CK, p.max_chunks, err);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(attn_decode_combine_kernel, dim3(B * H), dim3(D), 0, st, (const float*)part_o,
+                    (const float*)part_ml, reinterpret_cast<bf16*>(o), sp, sp_scalar, H, D, S_max, p.CK,
+                    p.max_chunks);
 }
 
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
@@ -625,10 +635,9 @@ cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, vo
     if (e != cudaSuccess) return e;
   }
   dim3 grid(B * T_, H);
-  attn_simple_kernel<T><<<grid, 128, smem, st>>>(reinterpret_cast<const T*>(q), reinterpret_cast<const T*>(ck),
-                                                 reinterpret_cast<const T*>(cv), reinterpret_cast<T*>(o), sp, sp_scalar,
-                                                 T_, H, Hkv, D, S_max);
-  return cudaGetLastError();
+  return launch_pdl(attn_simple_kernel<T>, grid, dim3(128), smem, st, reinterpret_cast<const T*>(q),
+                    reinterpret_cast<const T*>(ck), reinterpret_cast<const T*>(cv), reinterpret_cast<T*>(o), sp,
+                    sp_scalar, T_, H, Hkv, D, S_max);
 }
 
 template cudaError_t launch_attn_simple<float>(const void*, const void*, const void*, void*, const int*, int, int,

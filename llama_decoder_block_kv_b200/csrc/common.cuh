@@ -171,6 +171,14 @@ __device__ __forceinline__ void epilogue8(const EpiParams& p, int m, int n0, flo
 
 // ---------------------------------------------------------------- PTX wrappers
 
+// Programmatic dependent launch: every kernel of the forward pass is launched
+// so that it may start while the previous one drains. pdl_trigger lets the
+// next kernel begin launching; pdl_wait blocks until the previous kernel has
+// completed and its writes are visible. Nothing before pdl_wait may read data
+// a previous kernel writes, or write global memory.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

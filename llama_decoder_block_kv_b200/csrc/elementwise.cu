@@ -12,6 +12,8 @@ namespace llama {
 template <typename T>
 __global__ void embed_gather_kernel(const int* __restrict__ tokens, const T* __restrict__ table,
                                     float* __restrict__ h, int dim, int vocab, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int id = tokens[t];
   float* dst = h + (size_t)t * dim;
@@ -48,6 +50,8 @@ template <typename T, int THREADS>
 __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restrict__ h, const T* __restrict__ w,
                                                           T* __restrict__ out, int dim, float eps, int in_row_stride_T,
                                                           int in_row_offset) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x;
   const float* x = h + ((size_t)r * in_row_stride_T + in_row_offset) * dim;
   __shared__ float red[THREADS / 32];
@@ -127,18 +131,19 @@ __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ 
 template <typename T>
 void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int* err,
                   cudaStream_t st) {
-  embed_gather_kernel<T><<<n_tok, 128, 0, st>>>(tokens, reinterpret_cast<const T*>(table), h, dim, vocab, err);
+  launch_pdl(embed_gather_kernel<T>, dim3(n_tok), dim3(128), 0, st, tokens, reinterpret_cast<const T*>(table), h, dim,
+             vocab, err);
 }
 
 template <typename T>
 void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
                     int in_row_offset, cudaStream_t st) {
   if (dim >= 4096)
-    rmsnorm_kernel<T, 256><<<rows, 256, 0, st>>>(h, reinterpret_cast<const T*>(w), reinterpret_cast<T*>(out), dim,
-                                                 eps, in_row_stride_T, in_row_offset);
+    launch_pdl(rmsnorm_kernel<T, 256>, dim3(rows), dim3(256), 0, st, h, reinterpret_cast<const T*>(w),
+               reinterpret_cast<T*>(out), dim, eps, in_row_stride_T, in_row_offset);
   else
-    rmsnorm_kernel<T, 64><<<rows, 64, 0, st>>>(h, reinterpret_cast<const T*>(w), reinterpret_cast<T*>(out), dim,
-                                               eps, in_row_stride_T, in_row_offset);
+    launch_pdl(rmsnorm_kernel<T, 64>, dim3(rows), dim3(64), 0, st, h, reinterpret_cast<const T*>(w),
+               reinterpret_cast<T*>(out), dim, eps, in_row_stride_T, in_row_offset);
 }
 
 template <typename T>

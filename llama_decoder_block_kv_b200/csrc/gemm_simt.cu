@@ -12,6 +12,8 @@ constexpr int BM = 64, BN = 64, BK = 16, THREADS = 256;
 template <typename T>
 __global__ void __launch_bounds__(THREADS)
     gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ W, int M, int N, int K, EpiParams ep) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[BK][BM + 4];
   __shared__ float Ws[BK][BN + 4];
   const int tid = threadIdx.x;
@@ -51,8 +53,8 @@ __global__ void __launch_bounds__(THREADS)
 template <typename T>
 void launch_gemm_simt(const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st) {
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-  gemm_simt_kernel<T><<<grid, THREADS, 0, st>>>(reinterpret_cast<const T*>(A), reinterpret_cast<const T*>(W), M, N,
-                                                 K, ep);
+  launch_pdl(gemm_simt_kernel<T>, grid, dim3(THREADS), 0, st, reinterpret_cast<const T*>(A),
+             reinterpret_cast<const T*>(W), M, N, K, ep);
 }
 
 template void launch_gemm_simt<float>(const void*, const void*, int, int, int, const EpiParams&, cudaStream_t);

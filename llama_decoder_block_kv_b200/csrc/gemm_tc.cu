@@ -91,6 +91,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -253,8 +255,7 @@ static cudaError_t launch_tc(const void* A, const void* B, int M, int N, int K, 
   }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<bf16, BN><<<grid, 192, TcCfg<BN>::SMEM, st>>>(ma, mb, M, N, K, ep);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<bf16, BN>, dim3(grid), dim3(192), TcCfg<BN>::SMEM, st, ma, mb, M, N, K, ep);
 }
 
 // BN = 256 unless that leaves the last wave badly filled.

@@ -86,14 +86,28 @@ __global__ void __launch_bounds__(160, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_trigger();
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       prefetch_tensormap(&map_w);
       prefetch_tensormap(&map_x);
-      int j = 0;
-      for (int x = sbeg; x < send; ++x, ++j) {
+      // The weights do not depend on the previous kernel: fill the ring with
+      // weight tiles first, then wait for the producer of X and add X tiles.
+      const int pre = min(STAGES, send - sbeg);
+      for (int i = 0; i < pre; ++i) {
+        const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
+        mbar_arrive_expect_tx(&full[i], SB);
+        tma_load_2d(base + i * SB, &map_w, &full[i], ks * KB, rb * RPC);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) {
+        const int x = sbeg + i, ks = x - (x / nk) * nk;
+        tma_load_2d(base + i * SB + W_BYTES, &map_x, &full[i], ks * KB, 0);
+      }
+      int j = pre;
+      for (int x = sbeg + pre; x < send; ++x, ++j) {
         const int st = j % STAGES;
         if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, ep.err, abort_flag)) break;
         const int rb = x / nk, ks = x - rb * nk;
@@ -109,6 +123,7 @@ __global__ void __launch_bounds__(160, 1)
   }
 
   // ------------------------------------------------------------------ consumers
+  pdl_wait();
   const int a_row = warp * 32 + (lane & 7) + 8 * ((lane >> 3) & 1);  // + 16 t
   const int a_col = 8 * (lane >> 4);                                 // + 16 kk
   int j = 0;
@@ -253,8 +268,8 @@ static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  gemv_bf16_kernel<MB><<<p.grid, 160, smem, st>>>(mw, mx, M, N, p.nk, p.total, part, counters, ep);
-  return cudaGetLastError();
+  return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, part,
+                    counters, ep);
 }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,

@@ -1,6 +1,6 @@
 """Run one kernel case repeatedly (for profilers and quick timing).
 
-  python -m llama_decoder_block_kv_b200.profile_case gemv M N K [--reps R]
+  python -m llama_decoder_block_kv_b200.profile_case gemv M N K [--reps R] [--graph]
   python -m llama_decoder_block_kv_b200.profile_case tc   M N K [--reps R]
   python -m llama_decoder_block_kv_b200.profile_case simt M N K [--reps R]
   python -m llama_decoder_block_kv_b200.profile_case prefill-attn T   (LLaMA-7B layer shape, one block call)
@@ -24,6 +24,7 @@ def main():
     ap.add_argument("kind", choices=["gemv", "tc", "simt", "prefill-attn", "decode-attn"])
     ap.add_argument("sizes", type=int, nargs="+")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--graph", action="store_true", help="time the launches inside one CUDA graph")
     a = ap.parse_args()
     torch.cuda.set_device(0)
     st = torch.cuda.current_stream()
@@ -36,10 +37,22 @@ def main():
         path = {"gemv": B.LLAMA_PATH_GEMV, "tc": B.LLAMA_PATH_TCGEN05, "simt": B.LLAMA_PATH_SIMT}[a.kind]
         B.llama_linear(x, w, y, path)
         torch.cuda.synchronize()
-        e0.record(st)
-        for _ in range(a.reps):
-            B.llama_linear(x, w, y, path)
-        e1.record(st)
+        if a.graph:
+            # a graph of `reps` back-to-back launches: no host overhead between them
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(a.reps):
+                    B.llama_linear(x, w, y, path)
+            g.replay()
+            torch.cuda.synchronize()
+            e0.record(st)
+            g.replay()
+            e1.record(st)
+        else:
+            e0.record(st)
+            for _ in range(a.reps):
+                B.llama_linear(x, w, y, path)
+            e1.record(st)
         e1.synchronize()
         ms = e0.elapsed_time(e1) / a.reps
         flops = 2.0 * M * N * K

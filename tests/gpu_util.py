@@ -30,6 +30,15 @@ def assert_abs_close(got: np.ndarray, ref: np.ndarray, tol: float, what: str = "
     assert err <= tol, f"{what}: max abs err {err:.4g} > {tol}"
 
 
+def assert_bf16_ulp(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    """Stored bf16 values (the cache) equal the oracle's up to one rounding step:
+    |got - ref| <= one bf16 spacing at |ref| (2^-7 relative at the bottom of a binade)."""
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    spacing = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+    bad = np.abs(got - ref) > spacing * 1.0000001
+    assert not bad.any(), f"{what}: {int(bad.sum())} values differ by more than one bf16 step"
+
+
 class Pair:
     """The same synthetic model loaded into the CUDA library and the oracle."""
 
@@ -87,7 +96,7 @@ def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float
         if pair.w.act == "fp32":
             assert_fp32_close(got[written], ref[written], f"cache {name}")
         else:
-            assert_abs_close(got[written], ref[written], tol, f"cache {name}")
+            assert_bf16_ulp(got[written], ref[written], f"cache {name}")
 
 
 # ----------------------------------------------------------------------------- conditioning floor
