@@ -32,17 +32,20 @@ def main():
     if a.kind in ("gemv", "tc", "simt"):
         M, N, K = a.sizes
         x = synth.normal((M, K), 1.0, 1, torch.bfloat16, "cuda")
-        w = synth.normal((N, K), 0.02, 2, torch.bfloat16, "cuda")
+        # enough weight copies that consecutive launches never find their weights in L2 (126 MB)
+        n_w = max(1, -(-400 * 2 ** 20 // (N * K * 2)))
+        ws = [synth.normal((N, K), 0.02, 2 + i, torch.bfloat16, "cuda") for i in range(n_w)]
         y = torch.empty((M, N), device="cuda")
         path = {"gemv": B.LLAMA_PATH_GEMV, "tc": B.LLAMA_PATH_TCGEN05, "simt": B.LLAMA_PATH_SIMT}[a.kind]
-        B.llama_linear(x, w, y, path)
+        for w in ws:
+            B.llama_linear(x, w, y, path)
         torch.cuda.synchronize()
         if a.graph:
             # a graph of `reps` back-to-back launches: no host overhead between them
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                for _ in range(a.reps):
-                    B.llama_linear(x, w, y, path)
+                for i in range(a.reps):
+                    B.llama_linear(x, ws[i % n_w], y, path)
             g.replay()
             torch.cuda.synchronize()
             e0.record(st)
@@ -50,8 +53,8 @@ def main():
             e1.record(st)
         else:
             e0.record(st)
-            for _ in range(a.reps):
-                B.llama_linear(x, w, y, path)
+            for i in range(a.reps):
+                B.llama_linear(x, ws[i % n_w], y, path)
             e1.record(st)
         e1.synchronize()
         ms = e0.elapsed_time(e1) / a.reps
