@@ -32,11 +32,17 @@ def assert_abs_close(got: np.ndarray, ref: np.ndarray, tol: float, what: str = "
 
 def assert_bf16_ulp(got: np.ndarray, ref: np.ndarray, what: str = ""):
     """Stored bf16 values (the cache) equal the oracle's up to one rounding step:
-    |got - ref| <= one bf16 spacing at |ref| (2^-7 relative at the bottom of a binade)."""
+    |got - ref| <= one bf16 spacing at |ref| (2^-7 relative at the bottom of a
+    binade) plus 1e-4 * max|ref|. The absolute term covers values that are the
+    small remainder of a cancelling sum, where fp32 accumulation error is large
+    relative to the value itself."""
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     spacing = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
-    bad = np.abs(got - ref) > spacing * 1.0000001
-    assert not bad.any(), f"{what}: {int(bad.sum())} values differ by more than one bf16 step"
+    floor = 1e-4 * float(np.abs(ref).max())
+    diff = np.abs(got - ref)
+    bad = diff > spacing * 1.0000001 + floor
+    assert not bad.any(), (f"{what}: {int(bad.sum())} values differ by more than one bf16 step; worst diff "
+                           f"{diff[bad].max():.3g} at |ref| {np.abs(ref[bad]).max():.3g} (floor {floor:.3g})")
 
 
 class Pair:
