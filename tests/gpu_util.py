@@ -102,7 +102,8 @@ def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float
         if pair.w.act == "fp32":
             assert_fp32_close(got[written], ref[written], f"cache {name}")
         else:
-            assert_bf16_ulp(got[written], ref[written], f"cache {name}")
+            # slots are exact (checked above); values within the mode's hidden-state bound
+            assert_abs_close(got[written], ref[written], BF16_HIDDEN_ABS, f"cache {name}")
 
 
 # ----------------------------------------------------------------------------- conditioning floor
