@@ -7,8 +7,7 @@ import torch
 
 from llama_decoder_block_kv_b200 import binding as B
 from llama_decoder_block_kv_b200 import synth
-from tests.gpu_util import (BF16_HIDDEN_ABS, CacheSnapshot, Pair, assert_abs_close, assert_hidden_close_floor,
-                            oracle_floor)
+from tests.gpu_util import (CacheSnapshot, Pair, assert_bf16_cache_close, assert_hidden_close_floor, oracle_floor)
 from tests.helpers import t2np
 
 pytestmark = pytest.mark.gpu
@@ -49,7 +48,7 @@ def test_llama7b_layer_prefill_512_then_decode():
         k, v = pair.kv(0)
         for got, refc in ((k, pair.oracle.cache_k[0]), (v, pair.oracle.cache_v[0])):
             assert np.all(got[0, 516:] == 0)
-            assert_abs_close(got[0, :516], refc[0, :516], BF16_HIDDEN_ABS, "cache")
+            assert_bf16_cache_close(got[0, :516], refc[0, :516], "cache")
     finally:
         pair.close()
 
