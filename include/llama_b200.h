@@ -56,6 +56,7 @@ extern "C" {
 #define LLAMA_ERR_OOM -2          /* device allocation failed */
 #define LLAMA_ERR_CUDA -3         /* a CUDA runtime/driver call failed */
 #define LLAMA_ERR_NOT_READY -4    /* weights for a needed layer/head not set */
+#define LLAMA_ERR_TOO_LARGE -5    /* a size needs more than llama_linear_noalloc's fixed scratch */
 #define LLAMA_ERR_TOKEN_RANGE -10 /* device flag: a token id outside [0, vocab_size) */
 #define LLAMA_ERR_POS_RANGE -11   /* device flag: start_pos[b] + s outside [0, max_seq_len) */
 #define LLAMA_ERR_TIMEOUT -12     /* device flag: a bounded in-kernel wait gave up */
@@ -207,6 +208,31 @@ const char* llama_strerror(int code);
  */
 int llama_linear(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, int dtype, int path,
                  void* cuda_stream);
+
+/*
+ * llama_linear_noalloc: the LLAMA_PATH_GEMV case of llama_linear that
+ * allocates nothing. The pages have no counterpart; this is a library
+ * convenience for callers that cannot allocate device memory when they call,
+ * e.g. an application whose device memory is all owned by its own pool
+ * allocator, or a latency-critical loop where cudaMalloc/cudaFree (which can
+ * synchronise the device) are not acceptable.
+ *
+ * y_dev[M][N] (fp32) = x_dev[M][K] * w_dev[N][K]^T, x and w bfloat16, fp32
+ * accumulation, the same kernel as llama_linear(..., LLAMA_PATH_GEMV).
+ * Rules: 1 <= M <= 32, N % 8 == 0, K % 64 == 0; the caller owns x, w, y.
+ * Scratch: a fixed array of 8 MiB + 16.25 KiB of device memory compiled into
+ * the library (held on every GPU where the library's device code is loaded,
+ * until the process exits): at most 2 Mi fp32 split-K partial sums and 4096
+ * row blocks of 128 outputs (N <= 524288). A shape that needs more returns
+ * LLAMA_ERR_TOO_LARGE before anything is launched.
+ * The first call on a device (with that device current) looks up the array's
+ * device address; make that first call before any stream capture.
+ * All calls on one device share the array and it keeps the last call's
+ * contents; calls whose kernels overlap on the GPU (different streams without
+ * ordering between them) race. The arrival counters are cleared on
+ * cuda_stream before each launch. Stream-ordered, asynchronous.
+ */
+int llama_linear_noalloc(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -23,6 +23,7 @@ LLAMA_ERR_INVALID_ARGS = -1
 LLAMA_ERR_OOM = -2
 LLAMA_ERR_CUDA = -3
 LLAMA_ERR_NOT_READY = -4
+LLAMA_ERR_TOO_LARGE = -5
 LLAMA_ERR_TOKEN_RANGE = -10
 LLAMA_ERR_POS_RANGE = -11
 LLAMA_ERR_TIMEOUT = -12
@@ -31,7 +32,8 @@ LLAMA_PATH_AUTO, LLAMA_PATH_TCGEN05, LLAMA_PATH_GEMV, LLAMA_PATH_SIMT = 0, 1, 2,
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
-            "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear")
+            "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
+            "llama_linear_noalloc")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -76,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.llama_strerror.argtypes = [i]
         L.llama_strerror.restype = ctypes.c_char_p
         L.llama_linear.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+        L.llama_linear_noalloc.argtypes = [vp, vp, vp, i, i, i, vp]
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -211,6 +214,13 @@ def llama_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, path: int = 
     N = w.shape[0]
     dt = LLAMA_BF16 if x.dtype == torch.bfloat16 else LLAMA_FP32
     _check(lib().llama_linear(_ptr(x), _ptr(w), _ptr(y), M, N, K, dt, int(path), _stream(stream)), "llama_linear")
+
+
+def llama_linear_noalloc(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, stream=None) -> int:
+    """The GEMV case of llama_linear without any allocation; returns the C return code."""
+    M, K = x.shape
+    N = w.shape[0]
+    return lib().llama_linear_noalloc(_ptr(x), _ptr(w), _ptr(y), M, N, K, _stream(stream))
 
 
 class Llama:

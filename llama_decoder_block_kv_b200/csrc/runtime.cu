@@ -547,6 +547,7 @@ const char* llama_strerror(int code) {
     case LLAMA_ERR_OOM: return "device out of memory";
     case LLAMA_ERR_CUDA: return "CUDA error";
     case LLAMA_ERR_NOT_READY: return "weights not set";
+    case LLAMA_ERR_TOO_LARGE: return "size exceeds the fixed scratch of llama_linear_noalloc";
     case LLAMA_ERR_TOKEN_RANGE: return "token id outside [0, vocab_size)";
     case LLAMA_ERR_POS_RANGE: return "position outside [0, max_seq_len)";
     case LLAMA_ERR_TIMEOUT: return "a bounded device wait timed out";
