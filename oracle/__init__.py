@@ -16,6 +16,7 @@ from .llama_oracle import (  # noqa: F401
     bf16_bits_to_f64,
     bf16_round,
     block_forward,
+    block_forward_rows,
     causal_gqa_attention,
     ffn_hidden_dim,
     rmsnorm,

@@ -290,6 +290,42 @@ def block_forward(h: np.ndarray, lw: dict, cache_k: np.ndarray, cache_v: np.ndar
     return h + g @ as_f64(lw["w2"]).T
 
 
+def block_forward_rows(h: np.ndarray, lw: dict, start_pos, args: ModelArgs, cos: np.ndarray,
+                       sin: np.ndarray, rows) -> np.ndarray:
+    """block_forward restricted to selected output rows (large prefills).
+
+    The keys and values of every token of the call are computed (attention of a
+    row needs all earlier positions); queries, the attention, the output
+    projection and the feed-forward half are computed only for ``rows``, a list
+    of (b, s) pairs. Returns [len(rows), dim]: row i equals
+    block_forward(h, ...)[b_i, s_i]. Same definition, fewer rows.
+    """
+    act = args.act
+    B, T, dim = h.shape
+    H, Hkv, D = args.n_heads, args.kv_heads, args.head_dim
+    sp = _positions(start_pos, B)
+    pos = sp[:, None] + np.arange(T)[None, :]
+    K = np.zeros((B, int(pos.max()) + 1, Hkv, D))
+    V = np.zeros_like(K)
+    xn = rmsnorm(h, lw["attn_norm"], args.norm_eps, act)
+    xk = act_round(apply_rope((xn @ as_f64(lw["wk"]).T).reshape(B, T, Hkv, D), pos, cos, sin), act)
+    xv = act_round((xn @ as_f64(lw["wv"]).T).reshape(B, T, Hkv, D), act)
+    for b in range(B):
+        K[b, sp[b]:sp[b] + T] = xk[b]
+        V[b, sp[b]:sp[b] + T] = xv[b]
+    out = np.zeros((len(rows), dim))
+    for i, (b, s) in enumerate(rows):
+        p = np.array([pos[b, s]])
+        q = act_round(apply_rope((xn[b, s] @ as_f64(lw["wq"]).T).reshape(1, 1, H, D), p[None], cos, sin), act)
+        o = causal_gqa_attention(q, K[b:b + 1], V[b:b + 1], p, args.n_rep)
+        o = act_round(o.reshape(1, H * D), act)
+        hr = h[b, s][None] + o @ as_f64(lw["wo"]).T
+        xn2 = rmsnorm(hr, lw["ffn_norm"], args.norm_eps, act)
+        g = act_round(silu(xn2 @ as_f64(lw["w1"]).T) * (xn2 @ as_f64(lw["w3"]).T), act)
+        out[i] = (hr + g @ as_f64(lw["w2"]).T)[0]
+    return out
+
+
 @dataclass
 class OracleModel:
     """The whole model of [P4] Transformer: embedding, blocks, final norm, LM head.

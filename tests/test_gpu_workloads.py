@@ -92,3 +92,107 @@ def test_llama70b_layer_decode_batch16_at_4096():
         assert torch.equal(hd, hd2)
     finally:
         pair.close()
+
+
+def _cpu_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def test_llama3_8b_ragged_decode_sampled_sequences():
+    """LLaMA-3-8B-shaped whole model, batch 32 with ragged cache lengths in
+    [1024, 8128] (N(0,1) history), one decode step through llama_forward_ragged
+    exactly as the bench launches it; the oracle recomputes sequences 0, 1 and
+    31 through all 32 layers and the LM head."""
+    import oracle as O
+    w = synth.LLAMA3_8B_DECODE
+    model = B.Llama(B.ModelArgs.from_workload(w))
+    try:
+        ctx = model.ctx
+        full = (w.max_batch_size, w.max_seq_len, w.n_kv_heads, w.head_dim)
+        for i in range(w.n_layers):
+            B.llama_set_layer(ctx, i, synth.layer_weights(w, i, device="cuda"))
+            B.llama_kv_write(ctx, i, synth.cache_values(w, i, 0, full, "cuda"), synth.cache_values(w, i, 1, full, "cuda"))
+        enh = synth.embed_norm_head(w, device="cuda")
+        B.llama_set_embed_norm_head(ctx, enh["tok_embeddings"], enh["norm"], enh["output"])
+        lens = synth.ragged_lengths(w)
+        toks = synth.tokens(w, (w.decode_steps, w.batch), 0)[0].contiguous()
+        logits = torch.full((w.batch, w.vocab_size), float("nan"), device="cuda")
+        B.llama_forward_ragged(ctx, toks.cuda(), lens.cuda(), logits)
+        torch.cuda.synchronize()
+        code, flags = B.llama_get_error(ctx)
+        assert code == B.LLAMA_OK, (code, flags)
+        got = _cpu_f64(logits)
+    finally:
+        model.close()
+
+    seqs = [0, 1, 31]
+    L = lens.numpy().astype(np.int64)[seqs]
+    args = O.ModelArgs(dim=w.dim, n_layers=1, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads, vocab_size=w.vocab_size,
+                       multiple_of=w.multiple_of, ffn_dim_multiplier=w.ffn_dim_multiplier, norm_eps=w.norm_eps,
+                       rope_theta=w.rope_theta, max_batch_size=len(seqs), max_seq_len=int(L.max()) + 1, act="bf16")
+    om = O.OracleModel(args)
+    h = _cpu_f64(enh["tok_embeddings"][toks[seqs].long().cuda()])[:, None, :]
+    n = int(L.max()) + 1
+    for i in range(w.n_layers):
+        om.layers[0] = {k: _cpu_f64(v) for k, v in synth.layer_weights(w, i, device="cuda").items()}
+        om.cache_k[0] = synth.cache_values(w, i, 0, full, "cuda")[seqs, :n].float().cpu().numpy()
+        om.cache_v[0] = synth.cache_values(w, i, 1, full, "cuda")[seqs, :n].float().cpu().numpy()
+        h = om.block(0, h, L)
+    xn = O.rmsnorm(h[:, 0], _cpu_f64(enh["norm"]), w.norm_eps, "bf16")
+    out = enh["output"]
+    ref = np.concatenate([xn @ _cpu_f64(out[v0:v0 + 16384]).T for v0 in range(0, w.vocab_size, 16384)], axis=1)
+    err = np.abs(got[seqs] - ref)
+    assert np.all(np.isfinite(got))
+    assert err.max() <= 5e-2, f"logits max abs err {err.max():.4g} > 5e-2 (p99 {np.quantile(err, 0.99):.3g})"
+
+
+def test_llama3_8b_prefill_layer0_sampled_rows():
+    """LLaMA-3-8B-shaped layer 0 over the full 4 x 8192 prefill (llama_block_forward,
+    tcgen05 GEMMs at M = 32768, flash prefill over 128 key tiles with GQA 32/8);
+    rows at positions 0, 1, 4095, 8191 of each sequence against the oracle."""
+    import oracle as O
+    w = synth.LLAMA3_8B_PREFILL
+    one = w.with_(n_layers=1, vocab_size=0)
+    pair_model = B.Llama(B.ModelArgs.from_workload(one))
+    lw_dev = synth.layer_weights(one, 0, device="cuda")
+    try:
+        B.llama_set_layer(pair_model.ctx, 0, lw_dev)
+        h = synth.hidden(one, (4, 8192, w.dim), 0, "cuda")
+        hd = h.clone()
+        B.llama_block_forward(pair_model.ctx, 0, hd, 0)
+        torch.cuda.synchronize()
+        code, flags = B.llama_get_error(pair_model.ctx)
+        assert code == B.LLAMA_OK, (code, flags)
+        rows = [(b, s) for b in range(4) for s in (0, 1, 4095, 8191)]
+        got = np.stack([_cpu_f64(hd[b, s]) for b, s in rows])
+    finally:
+        pair_model.close()
+    args = O.ModelArgs(dim=w.dim, n_layers=1, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads, vocab_size=0,
+                       multiple_of=w.multiple_of, ffn_dim_multiplier=w.ffn_dim_multiplier, norm_eps=w.norm_eps,
+                       rope_theta=w.rope_theta, max_batch_size=4, max_seq_len=8192, act="bf16")
+    cos, sin = O.rope_tables(args.head_dim, 2 * args.max_seq_len, args.rope_theta)
+    lw = {k: _cpu_f64(v) for k, v in lw_dev.items()}
+    h64 = _cpu_f64(h)
+
+    def run(x):
+        return O.block_forward_rows(x, lw, 0, args, cos, sin, rows)
+    ref, floor = oracle_floor(run, h64)
+    assert_hidden_close_floor(got, ref, floor, "prefill rows")
+
+
+def test_llama3_8b_shapes_reduced_prefill_logits():
+    """The LLaMA-3-8B shapes with 2 layers, one 1024-token prefill, last-position
+    logits (the stated reduction of the 8B prefill the oracle can run in full)."""
+    w = synth.LLAMA3_8B_PREFILL.with_(n_layers=2, max_batch_size=1, batch=1, max_seq_len=2048)
+    pair = Pair(w, weights_device="cuda", bits=True)
+    try:
+        tok = synth.tokens(w, (1, 1024))
+        out = torch.full((1, w.vocab_size), float("nan"), device="cuda")
+        B.llama_forward(pair.ctx, tok.cuda(), 0, out, False)
+        torch.cuda.synchronize()
+        pair.check_error()
+        ref = pair.oracle.forward(t2np(tok).astype(np.int64), 0, all_positions=False)
+        err = np.abs(t2np(out) - ref)
+        assert err.max() <= 5e-2, f"logits max abs err {err.max():.4g}"
+    finally:
+        pair.close()

@@ -420,3 +420,15 @@ def test_whole_model_matches_transformers_llama():
     got = build_oracle(w, lws, enh).forward(t2np(tok).astype(np.int64), 0)
     # the library keeps its RMSNorm statistics and RoPE angles in fp32
     assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def test_block_forward_rows_is_block_forward_restricted():
+    w, lws, enh = _tiny(act="bf16", n_layers=1)
+    m = build_oracle(w, lws, enh)
+    h = t2np(synth.hidden(w, (2, 7, w.dim)))
+    sp = np.array([0, 5])
+    full = m.block(0, h, sp)
+    rows = [(0, 0), (0, 6), (1, 0), (1, 3), (1, 6)]
+    got = O.block_forward_rows(h, m.layers[0], sp, m.args, m.cos, m.sin, rows)
+    for i, (b, s) in enumerate(rows):
+        np.testing.assert_allclose(got[i], full[b, s], rtol=0, atol=1e-12)
