@@ -158,6 +158,19 @@ def assert_hidden_close_floor(got: np.ndarray, ref: np.ndarray, floor: np.ndarra
     return float(err.max()), p99
 
 
+def assert_logits_close_floor(got: np.ndarray, ref: np.ndarray, floor: np.ndarray, what: str = ""):
+    """Logits of a deep model: as assert_hidden_close_floor with the 5e-2 logits bound."""
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    p99, fp99 = float(np.quantile(err, 0.99)), float(np.quantile(floor, 0.99))
+    tol_max = max(BF16_LOGITS_ABS, FLOOR_FACTOR * float(floor.max()))
+    tol_p99 = max(BF16_LOGITS_ABS, FLOOR_FACTOR * fp99)
+    assert p99 <= tol_p99, f"{what}: p99 abs err {p99:.4g} > {tol_p99:.4g} (oracle floor p99 {fp99:.4g})"
+    assert err.max() <= tol_max, \
+        f"{what}: max abs err {err.max():.4g} > {tol_max:.4g} (oracle floor max {floor.max():.4g})"
+    return float(err.max()), p99
+
+
 class CacheSnapshot:
     """Save and restore an oracle's caches (so a perturbed run starts from the same state)."""
 
