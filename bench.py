@@ -120,12 +120,18 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank takes part, rank order does not matter."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_step_per_rank: int, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step_per_rank * steps / (max_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- single-layer workloads
@@ -218,34 +224,49 @@ def time_graph(g, steps, warmup, world):
     return e0.elapsed_time(e1)
 
 
-def gemv_roofline(lb: LayerBench, peaks, reps=20):
-    """Average bandwidth of the decode GEMV kernel over the four decode linears
-    (algorithmic bytes: weights + activations in + fp32 outputs)."""
+# DRAM traffic per algorithmic byte of the decode GEMV, from the committed ncu
+# capture profiles/gemv_bf16_m1_n22016_k4096.md (dram read + write of one
+# launch / weights + activations + outputs). Valid for the kernel version that
+# capture names; set to None when the kernel changes until it is re-measured.
+GEMV_TRAFFIC_RATIO = (181.597184e6 + 5.217792e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
+
+
+def gemv_roofline(lb: LayerBench, peaks, reps=10):
+    """Average bandwidth of the decode GEMV kernel: the layer's four decode linears
+    (wqkv, wo, w1|w3, w2: 405 MB together, larger than L2) launched back to back
+    `reps` times inside one CUDA graph, timed with CUDA events around the replay.
+    Algorithmic bytes: weights + activations in + fp32 outputs."""
     pairs = lb.decode_gemms()
     ys = [torch.empty((x.shape[0], w.shape[0]), device="cuda") for x, w in pairs]
     byts = sum(w.numel() * 2 + x.numel() * 2 + x.shape[0] * w.shape[0] * 4 for x, w in pairs)
-    for _ in range(3):
-        for (x, w), y in zip(pairs, ys):
-            B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+    for (x, w), y in zip(pairs, ys):
+        B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            for (x, w), y in zip(pairs, ys):
+                B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+    g.replay()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in pairs]
-    tot = [0.0] * len(pairs)
-    for _ in range(reps):
-        for i, ((x, w), y) in enumerate(zip(pairs, ys)):
-            evs[i][0].record(st)
-            B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
-            evs[i][1].record(st)
-        torch.cuda.synchronize()
-        for i in range(len(pairs)):
-            tot[i] += evs[i][0].elapsed_time(evs[i][1])
-    t_ms = sum(tot) / reps / len(pairs)          # average launch duration
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    g.replay()
+    e1.record(st)
+    e1.synchronize()
+    launches = reps * len(pairs)
+    t_ms = e0.elapsed_time(e1) / launches          # average launch duration
     per_launch = byts / len(pairs)
     achieved = per_launch / (t_ms * 1e-3) / 1e9
+    traffic = None if GEMV_TRAFFIC_RATIO is None else int(round(GEMV_TRAFFIC_RATIO * per_launch))
     return {"kernel": "gemv_bf16_kernel (decode linears: wqkv, wo, w1|w3, w2)", "bound": "hbm",
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-            "bytes_per_launch": int(per_launch), "avg_launch_us": round(t_ms * 1e3, 2)}
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+            "traffic_source": "ncu dram read+write of the w1|w3 launch scaled by algorithmic bytes "
+                              "(profiles/gemv_bf16_m1_n22016_k4096.md)",
+            "bytes_per_launch": int(per_launch), "avg_launch_us": round(t_ms * 1e3, 2),
+            "launches_timed": launches}
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
@@ -309,7 +330,7 @@ def run_ours(args, world, rank, local):
     clocks = sampler.stop()
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
-    value = world * lb.tokens_per_step * args.steps / (ms * 1e-3)
+    value = job_throughput(lb.tokens_per_step, args.steps, ms, world)
 
     # phases, each timed the same way
     phases = {}
