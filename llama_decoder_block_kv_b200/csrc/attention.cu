@@ -21,9 +21,9 @@
 //    (sequence, kv head, chunk of keys); the chunk streams through the same
 //    TMA ring, the 4 compute warps each take 16 keys of every 64-key tile,
 //    their (max, sum, O) states merge in shared memory and the CTA writes one
-//    partial; attn_decode_combine_kernel merges the partials of all chunks
-//    with the log-sum-exp rule m = max m_c, l = sum l_c e^(m_c - m),
-//    o = sum o_c e^(m_c - m) / l.
+//    partial; the CTA that finishes last for a (sequence, head group) merges
+//    the partials of all chunks with the log-sum-exp rule m = max m_c,
+//    l = sum l_c e^(m_c - m), o = sum o_c e^(m_c - m) / l.
 //  - attn_simple_kernel: fp32 mode (tiny models), one CTA per (token, head),
 //    scores in shared memory, plain two-pass softmax.
 #include "kernels.cuh"
@@ -260,9 +260,9 @@ __global__ void __launch_bounds__(288, 1)
 template <int D>
 __global__ void __launch_bounds__(160)
     attn_decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                       const bf16* __restrict__ q, float* __restrict__ part_o, float* __restrict__ part_ml,
-                       const int* __restrict__ start_pos, int sp_scalar, int H, int Hkv, int S_max, int hpc, int CK,
-                       int max_chunks, int* err) {
+                       const bf16* __restrict__ q, bf16* __restrict__ o, float* __restrict__ part_o,
+                       float* __restrict__ part_ml, int* __restrict__ counters, const int* __restrict__ start_pos,
+                       int sp_scalar, int H, int Hkv, int S_max, int hpc, int CK, int max_chunks, int* err) {
   constexpr int STAGES = 3;
   constexpr uint32_t TB = AttnSmem<D>::TILE_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(160)
   const int k_begin = chunk * CK;
   if (k_begin >= L) return;  // ragged batches: this sequence has fewer chunks
   const int k_end = min(L, k_begin + CK);
+  const int nc = (L + CK - 1) / CK;  // chunks of this sequence
   const int n_tiles = (k_end - k_begin + KT - 1) / KT;
   const int row0 = (b * Hkv + kvh) * S_max + k_begin;
   const int h0 = kvh * n_rep + grp * hpc;
@@ -458,6 +459,10 @@ __global__ void __launch_bounds__(160)
       acc += sm_o[(w * 16 + r) * D + d] * f;
       ll += sm_l[w * 16 + r] * f;
     }
+    if (nc == 1) {  // the sequence's only chunk: normalise and store the output directly
+      o[((size_t)b * H + h0 + r) * D + d] = __float2bfloat16_rn(acc / ll);
+      continue;
+    }
     const size_t slot = ((size_t)b * H + h0 + r) * max_chunks + chunk;
     part_o[slot * D + d] = acc;
     if (d == 0) {
@@ -465,29 +470,32 @@ __global__ void __launch_bounds__(160)
       part_ml[slot * 2 + 1] = ll;
     }
   }
-}
+  if (nc == 1) return;
 
-__global__ void attn_decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                           bf16* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar,
-                                           int H, int D, int S_max, int CK, int max_chunks) {
-  pdl_trigger();
-  pdl_wait();
-  const int bh = blockIdx.x;
-  const int b = bh / H;
-  const int sp = start_pos ? start_pos[b] : sp_scalar;
-  const int L = min(sp + 1, S_max);
-  const int nc = (L + CK - 1) / CK;
-  const float* ml = part_ml + (size_t)bh * max_chunks * 2;
-  float mm = -INFINITY;
-  for (int c = 0; c < nc; ++c) mm = fmaxf(mm, ml[2 * c]);
-  float ll = 0.f;
-  for (int c = 0; c < nc; ++c) ll += ml[2 * c + 1] * exp2f(ml[2 * c] - mm);
-  const float inv = 1.f / ll;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int c = 0; c < nc; ++c) acc += part_o[((size_t)bh * max_chunks + c) * D + d] * exp2f(ml[2 * c] - mm);
-    o[(size_t)bh * D + d] = __float2bfloat16_rn(acc * inv);
+  // The CTA that finishes last for this (sequence, head group) merges every
+  // chunk's partial with the log-sum-exp rule, in chunk order (deterministic),
+  // and re-arms the counter for the next launch.
+  __threadfence();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  __shared__ int s_last;
+  if (threadIdx.x == 0) s_last = (atomicAdd(&counters[z], 1) == nc - 1);
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (!s_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < hpc * D; e += 128) {
+    const int r = e / D, d = e - r * D;
+    const size_t row = ((size_t)b * H + h0 + r) * max_chunks;
+    float mm = -INFINITY;
+    for (int c = 0; c < nc; ++c) mm = fmaxf(mm, __ldcg(part_ml + (row + c) * 2));
+    float acc = 0.f, ll = 0.f;
+    for (int c = 0; c < nc; ++c) {
+      const float f = exp2f(__ldcg(part_ml + (row + c) * 2) - mm);
+      ll += __ldcg(part_ml + (row + c) * 2 + 1) * f;
+      acc += __ldcg(part_o + (row + c) * D + d) * f;
+    }
+    o[((size_t)b * H + h0 + r) * D + d] = __float2bfloat16_rn(acc / ll);
   }
+  if (threadIdx.x == 0) counters[z] = 0;
 }
 
 // ============================================================================ fp32 mode
@@ -598,8 +606,8 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
 
 template <int D>
 static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
-                            const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max, const DecodePlan& p,
-                            int* err, cudaStream_t st) {
+                            int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max,
+                            const DecodePlan& p, int* err, cudaStream_t st) {
   const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
   static bool attr = false;
   if (!attr) {
@@ -611,19 +619,16 @@ static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
   float* part_o = part;
   float* part_ml = part + (size_t)B * H * p.max_chunks * D;
   dim3 grid(p.max_chunks, B * Hkv * (n_rep / p.hpc));
-  cudaError_t e = launch_pdl(attn_decode_kernel<D>, grid, dim3(160), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
-                             part_o, part_ml, sp, sp_scalar, H, Hkv, S_max, p.hpc, p.CK, p.max_chunks, err);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(attn_decode_combine_kernel, dim3(B * H), dim3(D), 0, st, (const float*)part_o,
-                    (const float*)part_ml, reinterpret_cast<bf16*>(o), sp, sp_scalar, H, D, S_max, p.CK,
-                    p.max_chunks);
+  return launch_pdl(attn_decode_kernel<D>, grid, dim3(160), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
+                    reinterpret_cast<bf16*>(o), part_o, part_ml, counters, sp, sp_scalar, H, Hkv, S_max, p.hpc, p.CK,
+                    p.max_chunks, err);
 }
 
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
-                               const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
+                               int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st) {
-  if (D == 128) return decode_d<128>(mk, mv, q, o, part, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
-  return decode_d<64>(mk, mv, q, o, part, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  if (D == 128) return decode_d<128>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  return decode_d<64>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
 }
 
 template <typename T>

@@ -64,7 +64,7 @@ cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, co
                                 int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max, int* err,
                                 cudaStream_t st);
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
-                               const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
+                               int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
 template <typename T>
 cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, void* o, const int* sp, int sp_scalar,

@@ -199,8 +199,9 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
     const int max_len = sp_dev ? c->S : sp_host + 1;
     DecodePlan p = plan_decode(B, c->H, c->Hkv, c->S, max_len, c->num_sms);
     if (p.part_floats > c->part_floats) return LLAMA_ERR_INVALID_ARGS;
-    ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, sp_dev, sp_host, B, c->H, c->Hkv, c->D, c->S, p,
-                            c->err, st);
+    if (B * c->Hkv * (c->n_rep / p.hpc) > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
+    ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H, c->Hkv,
+                            c->D, c->S, p, c->err, st);
   } else {
     ce = launch_attn_prefill(Ly.map_k, Ly.map_v, c->q, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D, c->S, c->err,
                              st);
@@ -382,6 +383,7 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     if (dec > need) need = dec;
     c->part_floats = need;
     if ((r = alloc(reinterpret_cast<void**>(&c->part), need * sizeof(float)))) return fail(r);
+    if (rbs < c->Bm * c->H) rbs = c->Bm * c->H;  // decode attention: one counter per (sequence, head group)
     c->counters_n = rbs;
     if ((r = alloc(reinterpret_cast<void**>(&c->counters), (size_t)rbs * sizeof(int)))) return fail(r);
     cudaMemset(c->counters, 0, (size_t)rbs * sizeof(int));
