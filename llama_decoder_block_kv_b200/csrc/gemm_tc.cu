@@ -241,6 +241,22 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over a row-major [d2][d1][d0] array with a box of
+// b0 x b1 x b2 elements (b0 * 2 bytes = 128) and 128-byte swizzling.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                       uint32_t b1, uint32_t b2) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int BN>
 static cudaError_t launch_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
                              cudaStream_t st) {

@@ -51,6 +51,8 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, 
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                       uint32_t b1, uint32_t b2);
 cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
                            cudaStream_t st);
 
@@ -66,6 +68,10 @@ cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, co
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
+// attn_tc.cu
+cudaError_t launch_attn_prefill_tc(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o,
+                                   const int* sp, int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max,
+                                   int* err, cudaStream_t st);
 template <typename T>
 cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, void* o, const int* sp, int sp_scalar,
                                int B, int T_, int H, int Hkv, int D, int S_max, cudaStream_t st);

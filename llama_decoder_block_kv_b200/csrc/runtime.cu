@@ -203,8 +203,8 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
     ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H, c->Hkv,
                             c->D, c->S, p, c->err, st);
   } else {
-    ce = launch_attn_prefill(Ly.map_k, Ly.map_v, c->q, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D, c->S, c->err,
-                             st);
+    ce = launch_attn_prefill_tc(Ly.map_k, Ly.map_v, c->q, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D, c->S,
+                                c->err, st);
   }
   if (ce != cudaSuccess) return LLAMA_ERR_CUDA;
 
