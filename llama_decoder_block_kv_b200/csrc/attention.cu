@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(288, 1)
     fence_barrier_init();
   }
   __syncthreads();
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -278,8 +278,7 @@ __global__ void __launch_bounds__(160)
   const int b = z / (Hkv * groups);
   const int kvh = (z / groups) % Hkv;
   const int grp = z % groups;
-  pdl_trigger();
-  pdl_wait();
+  // positions are inputs of the call, never written by a kernel of the forward pass
   const int sp = start_pos ? start_pos[b] : sp_scalar;
   const int L = min(sp + 1, S_max);  // keys 0 .. sp
   const int k_begin = chunk * CK;
@@ -298,14 +297,24 @@ __global__ void __launch_bounds__(160)
     fence_barrier_init();
   }
   __syncthreads();
-  pdl_trigger();
-  pdl_wait();
 
   if (warp == 4) {
+    // Cache tiles that end before this step's position were written by earlier
+    // calls, which have completed (see pdl_wait): fetch up to a ring of them
+    // while the QKV kernel that writes position sp is still finishing.
+    const int safe = (k_end - 1 < sp) ? n_tiles : (sp - k_begin) / KT;
+    const int pre = min(STAGES, safe);
     if (lane == 0) {
       prefetch_tensormap(&map_k);
       prefetch_tensormap(&map_v);
-      int j = 0;
+      for (int j = 0; j < pre; ++j)
+        load_kv_tile<D>(&map_k, &map_v, base + j * 2 * TB, base + j * 2 * TB + TB, &full[j], row0 + j * KT);
+    }
+    __syncwarp();
+    pdl_wait();
+    pdl_trigger();
+    if (lane == 0) {
+      int j = pre;
       for (; j < n_tiles; ++j) {
         const int st = j % STAGES;
         if (!mbar_wait(&empty[st], ((j / STAGES) & 1) ^ 1, err)) break;
@@ -315,6 +324,8 @@ __global__ void __launch_bounds__(160)
     }
     return;
   }
+  pdl_wait();
+  pdl_trigger();
 
   // query rows: g and g + 8 are heads h0 + g, h0 + g + 8 when inside the group of hpc
   uint32_t qa[D / 16][4];
@@ -504,8 +515,8 @@ template <typename T>
 __global__ void attn_simple_kernel(const T* __restrict__ q, const T* __restrict__ ck, const T* __restrict__ cv,
                                    T* __restrict__ o, const int* __restrict__ start_pos, int sp_scalar, int T_, int H,
                                    int Hkv, int D, int S_max) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   extern __shared__ float sm[];
   float* qs = sm;             // [D]
   float* sc = sm + D;         // [S_max]

@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
 
   const int sp = start_pos ? start_pos[b] : sp_scalar;
   const int q_last = min(q0 + BQ, T) - 1;

@@ -172,10 +172,14 @@ __device__ __forceinline__ void epilogue8(const EpiParams& p, int m, int n0, flo
 // ---------------------------------------------------------------- PTX wrappers
 
 // Programmatic dependent launch: every kernel of the forward pass is launched
-// so that it may start while the previous one drains. pdl_trigger lets the
-// next kernel begin launching; pdl_wait blocks until the previous kernel has
-// completed and its writes are visible. Nothing before pdl_wait may read data
-// a previous kernel writes, or write global memory.
+// so that it may start while the previous one drains. pdl_wait blocks until
+// the previous kernel has completed and its writes are visible; pdl_trigger
+// (always called after pdl_wait) then lets the next kernel begin launching.
+// Hence when a kernel starts, every kernel before its immediate predecessor
+// has completed. Before pdl_wait a kernel may only read data no kernel of the
+// forward pass writes (weights, tensor maps, positions) or, for the decode
+// attention, cache slots written by calls before the predecessor; it never
+// writes global memory there.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -208,6 +212,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
+}
+
+// add to the transaction bytes of the current phase without arriving
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {

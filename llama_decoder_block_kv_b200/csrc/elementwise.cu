@@ -12,8 +12,8 @@ namespace llama {
 template <typename T>
 __global__ void embed_gather_kernel(const int* __restrict__ tokens, const T* __restrict__ table,
                                     float* __restrict__ h, int dim, int vocab, int* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int id = tokens[t];
   float* dst = h + (size_t)t * dim;
@@ -50,8 +50,8 @@ template <typename T, int THREADS>
 __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restrict__ h, const T* __restrict__ w,
                                                           T* __restrict__ out, int dim, float eps, int in_row_stride_T,
                                                           int in_row_offset) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const float* x = h + ((size_t)r * in_row_stride_T + in_row_offset) * dim;
   __shared__ float red[THREADS / 32];

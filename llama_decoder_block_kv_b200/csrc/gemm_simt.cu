@@ -12,8 +12,8 @@ constexpr int BM = 64, BN = 64, BK = 16, THREADS = 256;
 template <typename T>
 __global__ void __launch_bounds__(THREADS)
     gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ W, int M, int N, int K, EpiParams ep) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float As[BK][BM + 4];
   __shared__ float Ws[BK][BN + 4];
   const int tid = threadIdx.x;

@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
