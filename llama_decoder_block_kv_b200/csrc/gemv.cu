@@ -34,8 +34,8 @@ constexpr size_t RING_BUDGET = 180 * 1024;
 // tokens' fp32 residual rows in shared memory (up to NORMX_MAX_K each), so the
 // ring is shorter.
 constexpr int NORMX_MAX_M = 2;
-constexpr int NORMX_MAX_K = 8192;
-constexpr size_t NORMX_ROWS_BYTES = (size_t)NORMX_MAX_M * NORMX_MAX_K * 4;
+constexpr int NORMX_MAX_K = 4096;
+constexpr size_t NORMX_ROWS_BYTES = (size_t)NORMX_MAX_M * NORMX_MAX_K * 4 + (size_t)NORMX_MAX_K * 2;  // rows + weight
 
 __host__ __device__ constexpr uint32_t x_bytes(int mb) { return 8u * mb * KB * 2; }
 __host__ __device__ constexpr uint32_t stage_bytes(int mb) { return W_BYTES + x_bytes(mb); }
@@ -109,37 +109,59 @@ __global__ void __launch_bounds__(160, 1)
   }
   __syncthreads();
 
-  if (NORMX && warp == 4) {
-    // ------------------------------------------------- producer computing x itself
-    const int K = nk * KB;
+  float inv[NORMX_MAX_M] = {};
+  bf16* wrow = reinterpret_cast<bf16*>(hrows + NORMX_MAX_M * NORMX_MAX_K);
+  const int K = nk * KB;
+  if (NORMX) {
+    // Weights first (they do not depend on the previous kernel); then all 160
+    // threads stage the residual rows and the norm weight in shared memory and
+    // reduce the rows' sums of squares (fp32) for the inverse RMS.
     const int pre = min(STAGES, send - sbeg);
-    if (lane == 0) {
+    if (warp == 4 && lane == 0) {
       prefetch_tensormap(&map_w);
-      for (int i = 0; i < pre; ++i) {  // weights first: they do not depend on the previous kernel
+      for (int i = 0; i < pre; ++i) {
         const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
         mbar_expect_tx(&full[i], W_BYTES);
         tma_load_2d(base + i * SB, &map_w, &full[i], ks * KB, rb * RPC);
       }
     }
-    __syncwarp();
     pdl_wait();
     pdl_trigger();
-    // residual rows into shared memory and their inverse RMS (fp32 sum of squares)
-    float inv[NORMX_MAX_M];
+    __shared__ float s_ss[NORMX_MAX_M][5];
+    float ss[NORMX_MAX_M] = {};
+    constexpr int ITERS = (NORMX_MAX_K + 160 * 4 - 1) / (160 * 4);  // every load in flight at once
 #pragma unroll
     for (int m = 0; m < NORMX_MAX_M; ++m) {
-      float ss = 0.f;
-      if (m < M) {
-        for (int k = lane * 4; k < K; k += 128) {
-          const float4 v = *reinterpret_cast<const float4*>(nx.h + (size_t)m * K + k);
-          *reinterpret_cast<float4*>(hrows + m * K + k) = v;
-          ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        }
+      if (m >= M) break;
+      float4 v[ITERS];
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        const int k = tid * 4 + it * 640;
+        v[it] = k < K ? *reinterpret_cast<const float4*>(nx.h + (size_t)m * K + k) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
-      inv[m] = rsqrtf(ss / (float)K + nx.eps);
+      for (int it = 0; it < ITERS; ++it) {
+        const int k = tid * 4 + it * 640;
+        if (k < K) *reinterpret_cast<float4*>(hrows + m * K + k) = v[it];
+        ss[m] += v[it].x * v[it].x + v[it].y * v[it].y + v[it].z * v[it].z + v[it].w * v[it].w;
+      }
     }
+    for (int k = tid * 8; k < K; k += 160 * 8)
+      *reinterpret_cast<uint4*>(wrow + k) = *reinterpret_cast<const uint4*>(nx.weight + k);
+#pragma unroll
+    for (int m = 0; m < NORMX_MAX_M; ++m) {
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) ss[m] += __shfl_xor_sync(0xffffffffu, ss[m], o2);
+      if (lane == 0) s_ss[m][warp] = ss[m];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NORMX_MAX_M; ++m)
+      inv[m] = rsqrtf((s_ss[m][0] + s_ss[m][1] + s_ss[m][2] + s_ss[m][3] + s_ss[m][4]) / (float)K + nx.eps);
+  }
+  if (NORMX && warp == 4) {
+    // ------------------------------------------------- producer computing x itself
+    const int pre = min(STAGES, send - sbeg);
     // rows M..7 of every x tile stay zero
     for (int st = 0; st < STAGES; ++st)
       for (int e = lane; e < (8 - M) * 32; e += 32)
@@ -149,13 +171,16 @@ __global__ void __launch_bounds__(160, 1)
     auto build_x = [&](int st, int ks) {
       uint8_t* xt = base + st * SB + W_BYTES;
       const int c = 2 * lane, k = ks * KB + c;
-      const float2 w2 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(nx.weight + k));
-      for (int m = 0; m < M; ++m) {
-        const float a = round_to<bf16>(hrows[m * K + k] * inv[m]) * w2.x;
-        const float b = round_to<bf16>(hrows[m * K + k + 1] * inv[m]) * w2.y;
-        *reinterpret_cast<uint32_t*>(xt + m * 128 + ((((c >> 3) ^ (m & 7)) & 7) << 4) + (c & 7) * 2) =
-            pack_bf16x2(a, b);
-      }
+      const float2 w2 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(wrow + k));
+#pragma unroll
+      for (int m = 0; m < NORMX_MAX_M; ++m)
+        if (m < M) {
+          const float2 hv = *reinterpret_cast<const float2*>(hrows + m * K + k);
+          const float a = round_to<bf16>(hv.x * inv[m]) * w2.x;
+          const float b = round_to<bf16>(hv.y * inv[m]) * w2.y;
+          *reinterpret_cast<uint32_t*>(xt + m * 128 + ((((c >> 3) ^ (m & 7)) & 7) << 4) + (c & 7) * 2) =
+              pack_bf16x2(a, b);
+        }
     };
     for (int i = 0; i < pre; ++i) {
       const int x = sbeg + i;
@@ -217,8 +242,10 @@ __global__ void __launch_bounds__(160, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  pdl_wait();
-  pdl_trigger();
+  if (!NORMX) {
+    pdl_wait();
+    pdl_trigger();
+  }
   const int a_row = warp * 32 + (lane & 7) + 8 * ((lane >> 3) & 1);  // + 16 t
   const int a_col = 8 * (lane >> 4);                                 // + 16 kk
   int j = 0;
