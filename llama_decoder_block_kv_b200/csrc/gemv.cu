@@ -30,21 +30,11 @@ constexpr uint32_t W_BYTES = RPC * KB * 2; // 16 KB
 constexpr int OS = RPC + 4;                // row stride of the fp32 output staging tile
 constexpr size_t RING_BUDGET = 180 * 1024;
 
-// With the RMSNorm folded in (NORMX, at most 2 tokens), the CTA keeps the
-// tokens' fp32 residual rows in shared memory (up to NORMX_MAX_K each), so the
-// ring is shorter.
-constexpr int NORMX_MAX_M = 2;
-constexpr int NORMX_MAX_K = 4096;
-constexpr size_t NORMX_ROWS_BYTES = (size_t)NORMX_MAX_M * NORMX_MAX_K * 4 + (size_t)NORMX_MAX_K * 2;  // rows + weight
-
 __host__ __device__ constexpr uint32_t x_bytes(int mb) { return 8u * mb * KB * 2; }
 __host__ __device__ constexpr uint32_t stage_bytes(int mb) { return W_BYTES + x_bytes(mb); }
-__host__ __device__ constexpr int stages(int mb, bool normx) {
-  return (int)((RING_BUDGET - (normx ? NORMX_ROWS_BYTES : 0)) / stage_bytes(mb));
-}
-__host__ __device__ constexpr size_t gemv_smem(int mb, bool normx) {
-  return 1024 + (size_t)stages(mb, normx) * stage_bytes(mb) + (size_t)8 * mb * OS * 4 + 2 * stages(mb, normx) * 8 +
-         16 + (normx ? NORMX_ROWS_BYTES : 0);
+__host__ __device__ constexpr int stages(int mb) { return (int)(RING_BUDGET / stage_bytes(mb)); }
+__host__ __device__ constexpr size_t gemv_smem(int mb) {
+  return 1024 + (size_t)stages(mb) * stage_bytes(mb) + (size_t)8 * mb * OS * 4 + 2 * stages(mb) * 8 + 16;
 }
 }  // namespace
 
@@ -67,29 +57,17 @@ __host__ __device__ __forceinline__ int sk_owner(int x, int total, int grid) {
   return c;
 }
 
-// NORMX: x is not read from memory; the producer warp computes it as the
-// RMSNorm of the fp32 residual rows (statistics in fp32, rounded to bf16,
-// times the bf16 weight, rounded again: the rmsnorm_kernel arithmetic) and
-// writes each stage's x tile into the ring itself.
-struct NormX {
-  const float* h;      // [M][K] residual rows
-  const bf16* weight;  // [K]
-  float eps;
-};
-
-template <int MB, bool NORMX>
+template <int MB>
 __global__ void __launch_bounds__(160, 1)
     gemv_bf16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
-                     int N, int nk, int total, float* __restrict__ part, int* __restrict__ counters, EpiParams ep,
-                     NormX nx) {
-  constexpr int STAGES = stages(MB, NORMX);
+                     int N, int nk, int total, float* __restrict__ part, int* __restrict__ counters, EpiParams ep) {
+  constexpr int STAGES = stages(MB);
   constexpr uint32_t SB = stage_bytes(MB);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* os = reinterpret_cast<float*>(base + STAGES * SB);
   uint64_t* full = reinterpret_cast<uint64_t*>(os + 8 * MB * OS);
   uint64_t* empty = full + STAGES;
-  float* hrows = reinterpret_cast<float*>(empty + STAGES + 2);  // NORMX only: [M][K]
   __shared__ int s_last;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
@@ -109,103 +87,6 @@ __global__ void __launch_bounds__(160, 1)
   }
   __syncthreads();
 
-  float inv[NORMX_MAX_M] = {};
-  bf16* wrow = reinterpret_cast<bf16*>(hrows + NORMX_MAX_M * NORMX_MAX_K);
-  const int K = nk * KB;
-  if (NORMX) {
-    // Weights first (they do not depend on the previous kernel); then all 160
-    // threads stage the residual rows and the norm weight in shared memory and
-    // reduce the rows' sums of squares (fp32) for the inverse RMS.
-    const int pre = min(STAGES, send - sbeg);
-    if (warp == 4 && lane == 0) {
-      prefetch_tensormap(&map_w);
-      for (int i = 0; i < pre; ++i) {
-        const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
-        mbar_expect_tx(&full[i], W_BYTES);
-        tma_load_2d(base + i * SB, &map_w, &full[i], ks * KB, rb * RPC);
-      }
-    }
-    pdl_wait();
-    pdl_trigger();
-    __shared__ float s_ss[NORMX_MAX_M][5];
-    float ss[NORMX_MAX_M] = {};
-    constexpr int ITERS = (NORMX_MAX_K + 160 * 4 - 1) / (160 * 4);  // every load in flight at once
-#pragma unroll
-    for (int m = 0; m < NORMX_MAX_M; ++m) {
-      if (m >= M) break;
-      float4 v[ITERS];
-#pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        const int k = tid * 4 + it * 640;
-        v[it] = k < K ? *reinterpret_cast<const float4*>(nx.h + (size_t)m * K + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int it = 0; it < ITERS; ++it) {
-        const int k = tid * 4 + it * 640;
-        if (k < K) *reinterpret_cast<float4*>(hrows + m * K + k) = v[it];
-        ss[m] += v[it].x * v[it].x + v[it].y * v[it].y + v[it].z * v[it].z + v[it].w * v[it].w;
-      }
-    }
-    for (int k = tid * 8; k < K; k += 160 * 8)
-      *reinterpret_cast<uint4*>(wrow + k) = *reinterpret_cast<const uint4*>(nx.weight + k);
-#pragma unroll
-    for (int m = 0; m < NORMX_MAX_M; ++m) {
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) ss[m] += __shfl_xor_sync(0xffffffffu, ss[m], o2);
-      if (lane == 0) s_ss[m][warp] = ss[m];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < NORMX_MAX_M; ++m)
-      inv[m] = rsqrtf((s_ss[m][0] + s_ss[m][1] + s_ss[m][2] + s_ss[m][3] + s_ss[m][4]) / (float)K + nx.eps);
-  }
-  if (NORMX && warp == 4) {
-    // ------------------------------------------------- producer computing x itself
-    const int pre = min(STAGES, send - sbeg);
-    // rows M..7 of every x tile stay zero
-    for (int st = 0; st < STAGES; ++st)
-      for (int e = lane; e < (8 - M) * 32; e += 32)
-        *reinterpret_cast<uint32_t*>(base + st * SB + W_BYTES + M * 128 + e * 4) = 0u;
-    __syncwarp();
-    // lane l owns columns 2l, 2l+1 of the 64-wide tile, for each token row
-    auto build_x = [&](int st, int ks) {
-      uint8_t* xt = base + st * SB + W_BYTES;
-      const int c = 2 * lane, k = ks * KB + c;
-      const float2 w2 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(wrow + k));
-#pragma unroll
-      for (int m = 0; m < NORMX_MAX_M; ++m)
-        if (m < M) {
-          const float2 hv = *reinterpret_cast<const float2*>(hrows + m * K + k);
-          const float a = round_to<bf16>(hv.x * inv[m]) * w2.x;
-          const float b = round_to<bf16>(hv.y * inv[m]) * w2.y;
-          *reinterpret_cast<uint32_t*>(xt + m * 128 + ((((c >> 3) ^ (m & 7)) & 7) << 4) + (c & 7) * 2) =
-              pack_bf16x2(a, b);
-        }
-    };
-    for (int i = 0; i < pre; ++i) {
-      const int x = sbeg + i;
-      build_x(i, x - (x / nk) * nk);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[i]);
-    }
-    int j = pre;
-    for (int x = sbeg + pre; x < send; ++x, ++j) {
-      const int st = j % STAGES;
-      const bool ok = wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, ep.err, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const int rb = x / nk, ks = x - rb * nk;
-      if (lane == 0) {
-        mbar_expect_tx(&full[st], W_BYTES);
-        tma_load_2d(base + st * SB, &map_w, &full[st], ks * KB, rb * RPC);
-      }
-      build_x(st, ks);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[st]);
-    }
-    if (lane == 0)
-      for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, ep.err);
-    return;
-  }
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
@@ -242,10 +123,8 @@ __global__ void __launch_bounds__(160, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  if (!NORMX) {
-    pdl_wait();
-    pdl_trigger();
-  }
+  pdl_wait();
+  pdl_trigger();
   const int a_row = warp * 32 + (lane & 7) + 8 * ((lane >> 3) & 1);  // + 16 t
   const int a_col = 8 * (lane >> 4);                                 // + 16 kk
   int j = 0;
@@ -379,19 +258,19 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
   return p;
 }
 
-template <int MB, bool NORMX>
+template <int MB>
 static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
-                             float* part, int* counters, const EpiParams& ep, const NormX& nx, cudaStream_t st) {
-  constexpr size_t smem = gemv_smem(MB, NORMX);
+                             float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
+  constexpr size_t smem = gemv_smem(MB);
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
-        cudaFuncSetAttribute(gemv_bf16_kernel<MB, NORMX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(gemv_bf16_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(gemv_bf16_kernel<MB, NORMX>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total,
-                    part, counters, ep, nx);
+  return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, part,
+                    counters, ep);
 }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
@@ -400,25 +279,12 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, 
   const int MB = (M + 7) / 8;
   CUtensorMap mw, mx;
   if (!make_tmap_bf16(&mw, W, N, K, RPC) || !make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
-  const NormX nx = {nullptr, nullptr, 0.f};
   switch (MB) {
-    case 1: return launch_mb<1, false>(mw, mx, M, N, p, part, counters, ep, nx, st);
-    case 2: return launch_mb<2, false>(mw, mx, M, N, p, part, counters, ep, nx, st);
-    case 3: return launch_mb<3, false>(mw, mx, M, N, p, part, counters, ep, nx, st);
-    default: return launch_mb<4, false>(mw, mx, M, N, p, part, counters, ep, nx, st);
+    case 1: return launch_mb<1>(mw, mx, M, N, p, part, counters, ep, st);
+    case 2: return launch_mb<2>(mw, mx, M, N, p, part, counters, ep, st);
+    case 3: return launch_mb<3>(mw, mx, M, N, p, part, counters, ep, st);
+    default: return launch_mb<4>(mw, mx, M, N, p, part, counters, ep, st);
   }
-}
-
-bool gemv_norm_supported(int M, int K) { return M >= 1 && M <= NORMX_MAX_M && K % KB == 0 && K <= NORMX_MAX_K; }
-
-cudaError_t launch_gemv_norm_bf16(const float* h, const void* norm_w, float eps, const void* W, int M, int N, int K,
-                                  const GemvPlan& p, float* part, int* counters, const EpiParams& ep,
-                                  cudaStream_t st) {
-  if (!gemv_norm_supported(M, K)) return cudaErrorInvalidValue;
-  CUtensorMap mw;
-  if (!make_tmap_bf16(&mw, W, N, K, RPC)) return cudaErrorInvalidValue;
-  const NormX nx = {h, reinterpret_cast<const bf16*>(norm_w), eps};
-  return launch_mb<1, true>(mw, mw, M, N, p, part, counters, ep, nx, st);
 }
 
 }  // namespace llama

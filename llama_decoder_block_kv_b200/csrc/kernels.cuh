@@ -49,12 +49,6 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms);
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
                              int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
 
-// RMSNorm folded into the decode GEMV (x = RMSNorm(h) with weight norm_w), for up to 2 tokens
-bool gemv_norm_supported(int M, int K);
-cudaError_t launch_gemv_norm_bf16(const float* h, const void* norm_w, float eps, const void* W, int M, int N, int K,
-                                  const GemvPlan& p, float* part, int* counters, const EpiParams& ep,
-                                  cudaStream_t st);
-
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,

@@ -167,31 +167,15 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
   return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
-// x = RMSNorm(h) then C = x * W^T. For one or two tokens (bf16) the norm is
-// computed inside the decode GEMV; otherwise the rmsnorm kernel writes xn first.
-int norm_gemm(llama_ctx* c, const float* h, const void* norm_w, const void* W, int M, int N, const EpiParams& ep,
-              cudaStream_t st) {
-  const int K = c->dim;
-  if (c->bf16 && gemv_norm_supported(M, K)) {
-    GemvPlan p = plan_gemv(M, N, K, c->num_sms);
-    if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_norm_bf16(h, norm_w, c->a.norm_eps, W, M, N, K, p, c->part, c->counters, ep, st) ==
-                   cudaSuccess
-               ? LLAMA_OK
-               : LLAMA_ERR_CUDA;
-  }
-  if (c->bf16)
-    launch_rmsnorm<bf16>(h, norm_w, c->xn, M, K, c->a.norm_eps, 1, 0, st);
-  else
-    launch_rmsnorm<float>(h, norm_w, c->xn, M, K, c->a.norm_eps, 1, 0, st);
-  return gemm(c, c->xn, W, M, N, K, ep, st);
-}
-
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
   Layer& Ly = c->layers[layer];
   const int M = B * T;
   const int HD = c->H * c->D;
   int r;
+  if (c->bf16)
+    launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  else
+    launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
 
   EpiParams e = epi_base(c, EPI_QKV_ROPE, M, c->n_qkv);
   e.q_out = c->q;
@@ -205,7 +189,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.Hkv = c->Hkv;
   e.D = c->D;
   e.S_max = c->S;
-  if ((r = norm_gemm(c, h, Ly.attn_norm, Ly.wqkv, M, c->n_qkv, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.wqkv, M, c->n_qkv, c->dim, e, st))) return r;
 
   cudaError_t ce;
   if (!c->bf16) {
@@ -229,9 +213,14 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.ld_out = c->dim;
   if ((r = gemm(c, c->o, Ly.wo, M, c->dim, HD, e, st))) return r;
 
+  if (c->bf16)
+    launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  else
+    launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+
   e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
   e.g_out = c->g;
-  if ((r = norm_gemm(c, h, Ly.ffn_norm, Ly.w13, M, 2 * c->F, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.w13, M, 2 * c->F, c->dim, e, st))) return r;
 
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;
@@ -257,14 +246,13 @@ int run_model(llama_ctx* c, const int32_t* tokens, int B, int T, const int* sp_d
   const int rows = all_positions ? M : B;
   const int stride = all_positions ? 1 : T;
   const int offset = all_positions ? 0 : T - 1;
-  EpiParams e = epi_base(c, EPI_STORE_F32, rows, c->V);
-  e.out = logits;
-  e.ld_out = c->V;
-  if (stride == 1) return norm_gemm(c, c->h, c->final_norm, c->output, rows, c->V, e, st);
   if (c->bf16)
     launch_rmsnorm<bf16>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
   else
     launch_rmsnorm<float>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
+  EpiParams e = epi_base(c, EPI_STORE_F32, rows, c->V);
+  e.out = logits;
+  e.ld_out = c->V;
   return gemm(c, c->xn, c->output, rows, c->V, c->dim, e, st);
 }
 
