@@ -607,7 +607,7 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
   int want = (2 * num_sms + units - 1) / units;
   int ck = (max_len + want - 1) / want;
   ck = (ck + KT - 1) / KT * KT;
-  if (ck < 128) ck = 128;
+  if (ck < 512) ck = 512;  // below ~512 keys the merge costs more than the parallelism gains
   if (ck > 1024) ck = 1024;
   p.CK = ck;
   p.max_chunks = (S_max + ck - 1) / ck;
