@@ -72,7 +72,15 @@ extern "C" {
  * Transformer class) and the storage type.
  *  dim, n_layers, n_heads, n_kv_heads (n_kv_heads <= 0 means n_kv_heads = n_heads),
  *  vocab_size (0 for single-block use), multiple_of, ffn_dim_multiplier
- *  (<= 0 means None), norm_eps, rope_theta, max_batch_size, max_seq_len, dtype.
+ *  (<= 0 means None), norm_eps, rope_theta, max_batch_size, max_seq_len, dtype,
+ *  rope_half_split.
+ * rope_half_split = 0: RoPE rotates the interleaved pairs (2i, 2i+1) of each
+ *  head (the notes' apply_rotary_emb, complex form). rope_half_split = 1: the
+ *  weights are given in the half-split convention of the HuggingFace port
+ *  ("LLaMa-1/2/3 原理+源码——拆解", RoPE: q*cos + rotate_half(q)*sin, pairs
+ *  (i, i + head_dim/2)); the library permutes the rows of wq and wk into the
+ *  interleaved order at load time (dot products q.k are unchanged) and
+ *  llama_kv_read/llama_kv_write present K in the half-split order.
  * Rules: dim % n_heads == 0; head_dim = dim / n_heads in {64, 128};
  *  n_heads % n_kv_heads == 0; n_heads / n_kv_heads <= 8 when dtype == LLAMA_BF16,
  *  or a multiple of 8; dim % 64 == 0; all sizes positive.
@@ -90,6 +98,7 @@ typedef struct {
   int32_t max_batch_size;
   int32_t max_seq_len;
   int32_t dtype;
+  int32_t rope_half_split;
 } llama_args;
 
 typedef struct llama_ctx llama_ctx;
@@ -174,6 +183,40 @@ int llama_forward_ragged(llama_ctx* ctx, const int32_t* tokens_dev, const int32_
  */
 int llama_block_forward(llama_ctx* ctx, int layer, float* h_dev, int B, int T, const int32_t* start_pos_dev,
                         int host_start_pos, void* cuda_stream);
+
+/*
+ * Next-token selection, the LLaMA model.py walk-through (linkmax.top),
+ * section 3.3 generate / sample_top_p. logits_dev fp32 [B][V] (row-major).
+ * temperature <= 0: greedy, out_dev[b] = argmax_v logits[b][v] (lowest index
+ * on ties). Otherwise probs = softmax(logits / temperature); sorted in
+ * descending order, a token is kept when the probabilities before it sum to
+ * at most top_p (0 < top_p <= 1); the kept probabilities are renormalised and
+ * the token drawn is the first one, in descending order (ties in index
+ * order), whose cumulative renormalised probability exceeds uniforms_dev[b]
+ * (caller-supplied uniforms in [0, 1), one per sequence: the draw is
+ * reproducible). out_dev int32 [B]. Uses a private, lazily allocated
+ * scratch of B*V floats; not thread-safe. Stream-ordered.
+ */
+int llama_sample(const float* logits_dev, int B, int V, float temperature, float top_p, const float* uniforms_dev,
+                 int32_t* out_dev, void* cuda_stream);
+
+/*
+ * generate() of the same walk-through, on the device, without host
+ * round trips: tokens_dev int32 [B][total_len] holds each prompt at the
+ * start of its row; prompt_mask_dev uint8 [B][total_len] is 1 where the row
+ * holds a prompt token (the walk-through's input_text_mask). Starting at
+ * cur = min_prompt_len (the shortest prompt), each step runs
+ * Transformer.forward(tokens[:, prev:cur], prev) with last-position logits,
+ * selects the next token as llama_sample does (uniforms_dev fp32
+ * [total_len][B], row cur used at step cur; may be NULL when temperature <= 0)
+ * and writes it to tokens[:, cur] except where the prompt mask is set; then
+ * prev = cur. Cache positions 0..total_len-2 of sequences 0..B-1 are
+ * overwritten. Rules: 1 <= B <= max_batch_size, 1 <= min_prompt_len <=
+ * total_len <= max_seq_len, vocab_size > 0. Stream-ordered; tokens_dev holds
+ * the result when the stream reaches the end of the call.
+ */
+int llama_generate(llama_ctx* ctx, int32_t* tokens_dev, const uint8_t* prompt_mask_dev, int B, int total_len,
+                   int min_prompt_len, float temperature, float top_p, const float* uniforms_dev, void* cuda_stream);
 
 /*
  * Copy one layer's caches out of / into the library, in the pages' logical

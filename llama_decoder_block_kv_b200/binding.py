@@ -33,14 +33,15 @@ LLAMA_PATH_AUTO, LLAMA_PATH_TCGEN05, LLAMA_PATH_GEMV, LLAMA_PATH_SIMT = 0, 1, 2,
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
-            "llama_linear_noalloc")
+            "llama_linear_noalloc", "llama_sample", "llama_generate")
 
 
 class LlamaArgs(ctypes.Structure):
     _fields_ = [("dim", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("vocab_size", ctypes.c_int32), ("multiple_of", ctypes.c_int32),
                 ("ffn_dim_multiplier", ctypes.c_float), ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
-                ("max_batch_size", ctypes.c_int32), ("max_seq_len", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("max_batch_size", ctypes.c_int32), ("max_seq_len", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("rope_half_split", ctypes.c_int32)]
 
 
 class LlamaError(RuntimeError):
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.llama_strerror.restype = ctypes.c_char_p
         L.llama_linear.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
         L.llama_linear_noalloc.argtypes = [vp, vp, vp, i, i, i, vp]
+        L.llama_sample.argtypes = [vp, i, i, f, f, vp, vp, vp]
+        L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -124,12 +127,13 @@ class ModelArgs:
     max_batch_size: int
     max_seq_len: int
     dtype: str = "bf16"
+    rope_half_split: bool = False
 
     def c(self) -> LlamaArgs:
         return LlamaArgs(self.dim, self.n_layers, self.n_heads, self.n_kv_heads, self.vocab_size, self.multiple_of,
                          -1.0 if self.ffn_dim_multiplier is None else float(self.ffn_dim_multiplier),
                          float(self.norm_eps), float(self.rope_theta), self.max_batch_size, self.max_seq_len,
-                         LLAMA_BF16 if self.dtype == "bf16" else LLAMA_FP32)
+                         LLAMA_BF16 if self.dtype == "bf16" else LLAMA_FP32, int(bool(self.rope_half_split)))
 
     @classmethod
     def from_workload(cls, w) -> "ModelArgs":
@@ -214,6 +218,21 @@ def llama_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, path: int = 
     N = w.shape[0]
     dt = LLAMA_BF16 if x.dtype == torch.bfloat16 else LLAMA_FP32
     _check(lib().llama_linear(_ptr(x), _ptr(w), _ptr(y), M, N, K, dt, int(path), _stream(stream)), "llama_linear")
+
+
+def llama_sample(logits: torch.Tensor, out: torch.Tensor, temperature: float = 0.0, top_p: float = 1.0,
+                 uniforms: Optional[torch.Tensor] = None, stream=None) -> None:
+    B, V = logits.shape
+    _check(lib().llama_sample(_ptr(logits), B, V, float(temperature), float(top_p), _ptr(uniforms), _ptr(out),
+                              _stream(stream)), "llama_sample")
+
+
+def llama_generate(ctx, tokens: torch.Tensor, prompt_mask: torch.Tensor, min_prompt_len: int,
+                   temperature: float = 0.0, top_p: float = 1.0, uniforms: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+    B, total_len = tokens.shape
+    _check(lib().llama_generate(ctx, _ptr(tokens), _ptr(prompt_mask), B, total_len, int(min_prompt_len),
+                                float(temperature), float(top_p), _ptr(uniforms), _stream(stream)), "llama_generate")
 
 
 def llama_linear_noalloc(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, stream=None) -> int:

@@ -11,11 +11,11 @@ namespace llama {
 // outside [0, vocab) raises the token-range flag and yields a zero row.
 template <typename T>
 __global__ void embed_gather_kernel(const int* __restrict__ tokens, const T* __restrict__ table,
-                                    float* __restrict__ h, int dim, int vocab, int* err) {
+                                    float* __restrict__ h, int dim, int vocab, int T_, int tok_stride, int* err) {
   pdl_wait();
   pdl_trigger();
-  const int t = blockIdx.x;
-  const int id = tokens[t];
+  const int t = blockIdx.x;  // token b * T_ + s, read from tokens[b * tok_stride + s]
+  const int id = tokens[(t / T_) * tok_stride + t % T_];
   float* dst = h + (size_t)t * dim;
   if (id < 0 || id >= vocab) {
     if (threadIdx.x == 0) atomicOr(err, LLAMA_DEV_TOKEN_RANGE);
@@ -105,11 +105,31 @@ __global__ void pack_w13_kernel(const T* __restrict__ w1, const T* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
+// Half-split RoPE weights (pairs (i, i + D/2) of each head) into the
+// interleaved order the kernels rotate (pairs (2i, 2i+1)): row 2i of a head
+// takes row i, row 2i+1 takes row i + D/2. q.k products are unchanged.
+template <typename T>
+__global__ void rope_rows_to_interleaved_kernel(const T* __restrict__ src, T* __restrict__ dst, int D, int dim) {
+  const size_t r = blockIdx.x;  // destination row
+  const int h = r / D, j = r % D;
+  const T* s = src + ((size_t)h * D + (j & 1 ? D / 2 : 0) + (j >> 1)) * dim;
+  T* d = dst + r * dim;
+  for (int i = threadIdx.x; i < dim; i += blockDim.x) d[i] = s[i];
+}
+
+// position of element j of a head in the interleaved order, given its index j
+// in the half-split order
+__device__ __forceinline__ int half_split_to_interleaved(int j, int D) {
+  return j < D / 2 ? 2 * j : 2 * (j - D / 2) + 1;
+}
+
+// ---------------------------------------------------------------------------
 // Cache layout conversion between the library's [b][kvh][pos][D] and the
 // pages' logical [b][pos][kvh][D] (the notes' Attention cache_k shape).
+// half_split: the logical side holds the head dimension in half-split order.
 template <typename T>
 __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ dst, int Bm, int S, int Hkv, int D,
-                                     int to_logical) {
+                                     int to_logical, int half_split) {
   const size_t row = blockIdx.x;  // over Bm * S * Hkv rows of D
   const int kvh = row % Hkv;
   const size_t bp = row / Hkv;
@@ -118,10 +138,11 @@ __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ 
   const size_t lib = (((size_t)b * Hkv + kvh) * S + pos) * D;
   const size_t logi = row * D;
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    const int li = half_split ? half_split_to_interleaved(i, D) : i;  // library index of logical element i
     if (to_logical)
-      dst[logi + i] = src[lib + i];
+      dst[logi + i] = src[lib + li];
     else
-      dst[lib + i] = src[logi + i];
+      dst[lib + li] = src[logi + i];
   }
 }
 
@@ -129,10 +150,10 @@ __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ 
 // host launchers
 
 template <typename T>
-void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int* err,
-                  cudaStream_t st) {
+void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
+                  int tok_stride, int* err, cudaStream_t st) {
   launch_pdl(embed_gather_kernel<T>, dim3(n_tok), dim3(128), 0, st, tokens, reinterpret_cast<const T*>(table), h, dim,
-             vocab, err);
+             vocab, T_, tok_stride, err);
 }
 
 template <typename T>
@@ -153,17 +174,25 @@ void launch_pack_w13(const void* w1, const void* w3, void* out, int F, int dim, 
 }
 
 template <typename T>
-void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D, int to_logical, cudaStream_t st) {
+void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D, int to_logical, int half_split,
+                       cudaStream_t st) {
   const size_t rows = (size_t)Bm * S * Hkv;
   kv_to_logical_kernel<T><<<(unsigned)rows, 128, 0, st>>>(reinterpret_cast<const T*>(src), reinterpret_cast<T*>(dst),
-                                                          Bm, S, Hkv, D, to_logical);
+                                                          Bm, S, Hkv, D, to_logical, half_split);
+}
+
+template <typename T>
+void launch_rope_rows_to_interleaved(const void* src, void* dst, int heads, int D, int dim, cudaStream_t st) {
+  rope_rows_to_interleaved_kernel<T><<<heads * D, 256, 0, st>>>(reinterpret_cast<const T*>(src),
+                                                                reinterpret_cast<T*>(dst), D, dim);
 }
 
 #define INST(T)                                                                                              \
-  template void launch_embed<T>(const int*, const void*, float*, int, int, int, int*, cudaStream_t);         \
+  template void launch_embed<T>(const int*, const void*, float*, int, int, int, int, int, int*, cudaStream_t); \
   template void launch_rmsnorm<T>(const float*, const void*, void*, int, int, float, int, int, cudaStream_t); \
   template void launch_pack_w13<T>(const void*, const void*, void*, int, int, cudaStream_t);                 \
-  template void launch_kv_convert<T>(const void*, void*, int, int, int, int, int, cudaStream_t);
+  template void launch_kv_convert<T>(const void*, void*, int, int, int, int, int, int, cudaStream_t);   \
+  template void launch_rope_rows_to_interleaved<T>(const void*, void*, int, int, int, cudaStream_t);
 INST(float)
 INST(bf16)
 #undef INST

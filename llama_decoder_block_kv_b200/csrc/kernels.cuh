@@ -26,15 +26,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // elementwise.cu
 template <typename T>
-void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int* err,
-                  cudaStream_t st);
+void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
+                  int tok_stride, int* err, cudaStream_t st);
 template <typename T>
 void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
                     int in_row_offset, cudaStream_t st);
 template <typename T>
 void launch_pack_w13(const void* w1, const void* w3, void* out, int F, int dim, cudaStream_t st);
 template <typename T>
-void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D, int to_logical, cudaStream_t st);
+void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D, int to_logical, int half_split,
+                       cudaStream_t st);
+template <typename T>
+void launch_rope_rows_to_interleaved(const void* src, void* dst, int heads, int D, int dim, cudaStream_t st);
 
 // gemm_simt.cu
 template <typename T>
@@ -68,6 +71,11 @@ cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, co
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
+// sample.cu
+cudaError_t launch_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
+                          float* scratch, int32_t* out, int out_stride, const uint8_t* keep, int keep_stride,
+                          cudaStream_t st);
+
 // attn_tc.cu
 cudaError_t launch_attn_prefill_tc(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o,
                                    const int* sp, int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max,

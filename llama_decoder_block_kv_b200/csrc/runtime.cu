@@ -42,6 +42,7 @@ struct Layer {
 struct llama_ctx {
   llama_args a;
   bool bf16 = true;
+  bool half_split = false;  // weights given with half-split RoPE pairs
   int esz = 2;
   int dim = 0, H = 0, Hkv = 0, D = 0, n_rep = 1, F = 0, V = 0, S = 0, Bm = 0, L = 0;
   int n_qkv = 0;
@@ -65,6 +66,9 @@ struct llama_ctx {
   size_t part_floats = 0;
   int* counters = nullptr;
   int counters_n = 0;
+  // generation: last-position logits and sampling scratch, [max_batch][vocab] each
+  float* gen_logits = nullptr;
+  float* gen_probs = nullptr;
 };
 
 namespace {
@@ -229,8 +233,8 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
 }
 
 // embedding -> blocks -> final norm -> LM head
-int run_model(llama_ctx* c, const int32_t* tokens, int B, int T, const int* sp_dev, int sp_host, float* logits,
-              int all_positions, cudaStream_t st) {
+int run_model(llama_ctx* c, const int32_t* tokens, int tok_stride, int B, int T, const int* sp_dev, int sp_host,
+              float* logits, int all_positions, cudaStream_t st) {
   if (!c->head_set) return LLAMA_ERR_NOT_READY;
   for (int l = 0; l < c->L; ++l)
     if (!c->layers[l].set) return LLAMA_ERR_NOT_READY;
@@ -238,9 +242,9 @@ int run_model(llama_ctx* c, const int32_t* tokens, int B, int T, const int* sp_d
   int r;
   if ((r = reserve(c, M))) return r;
   if (c->bf16)
-    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, c->err, st);
+    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st);
   else
-    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, c->err, st);
+    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st);
   for (int l = 0; l < c->L; ++l)
     if ((r = run_block(c, l, c->h, B, T, sp_dev, sp_host, st))) return r;
   const int rows = all_positions ? M : B;
@@ -288,6 +292,7 @@ int llama_create(const llama_args* args, llama_ctx** out) {
       a.vocab_size < 0 || a.multiple_of <= 0 || !(a.norm_eps >= 0.f) || !(a.rope_theta > 0.f))
     return LLAMA_ERR_INVALID_ARGS;
   if (a.dtype != LLAMA_FP32 && a.dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
+  if (a.rope_half_split != 0 && a.rope_half_split != 1) return LLAMA_ERR_INVALID_ARGS;
   if (a.dim % a.n_heads || a.n_heads % a.n_kv_heads || a.dim % 64) return LLAMA_ERR_INVALID_ARGS;
   const int D = a.dim / a.n_heads;
   if (D != 64 && D != 128) return LLAMA_ERR_INVALID_ARGS;
@@ -301,6 +306,7 @@ int llama_create(const llama_args* args, llama_ctx** out) {
   llama_ctx* c = new llama_ctx();
   c->a = a;
   c->bf16 = a.dtype == LLAMA_BF16;
+  c->half_split = a.rope_half_split == 1;
   c->esz = c->bf16 ? 2 : 4;
   c->dim = a.dim;
   c->H = a.n_heads;
@@ -414,6 +420,8 @@ void llama_destroy(llama_ctx* c) {
   release(c->g);
   release(reinterpret_cast<void*&>(c->part));
   release(reinterpret_cast<void*&>(c->counters));
+  release(reinterpret_cast<void*&>(c->gen_logits));
+  release(reinterpret_cast<void*&>(c->gen_probs));
   delete c;
 }
 
@@ -426,8 +434,19 @@ int llama_set_layer(llama_ctx* c, int layer, const void* wq, const void* wk, con
   const size_t es = c->esz;
   const size_t qb = (size_t)c->H * c->D * c->dim * es, kb = (size_t)c->Hkv * c->D * c->dim * es;
   uint8_t* p = reinterpret_cast<uint8_t*>(Ly.wqkv);
-  CK(cudaMemcpy(p, wq, qb, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(p + qb, wk, kb, cudaMemcpyDeviceToDevice));
+  if (c->half_split) {  // rotate interleaved pairs on rows permuted from the half-split order
+    if (c->bf16) {
+      launch_rope_rows_to_interleaved<bf16>(wq, p, c->H, c->D, c->dim, 0);
+      launch_rope_rows_to_interleaved<bf16>(wk, p + qb, c->Hkv, c->D, c->dim, 0);
+    } else {
+      launch_rope_rows_to_interleaved<float>(wq, p, c->H, c->D, c->dim, 0);
+      launch_rope_rows_to_interleaved<float>(wk, p + qb, c->Hkv, c->D, c->dim, 0);
+    }
+    CK(cudaGetLastError());
+  } else {
+    CK(cudaMemcpy(p, wq, qb, cudaMemcpyDeviceToDevice));
+    CK(cudaMemcpy(p + qb, wk, kb, cudaMemcpyDeviceToDevice));
+  }
   CK(cudaMemcpy(p + qb + kb, wv, kb, cudaMemcpyDeviceToDevice));
   CK(cudaMemcpy(Ly.wo, wo, (size_t)c->dim * c->H * c->D * es, cudaMemcpyDeviceToDevice));
   CK(cudaMemcpy(Ly.w2, w2, (size_t)c->dim * c->F * es, cudaMemcpyDeviceToDevice));
@@ -465,7 +484,7 @@ int llama_forward(llama_ctx* c, const int32_t* tokens, int B, int T, int start_p
   int r;
   if ((r = check_ctx_call(c, B, T))) return r;
   if (!tokens || !logits || start_pos < 0 || (long)start_pos + T > c->S) return LLAMA_ERR_INVALID_ARGS;
-  return run_model(c, tokens, B, T, nullptr, start_pos, logits, all_positions, S_(stream));
+  return run_model(c, tokens, T, B, T, nullptr, start_pos, logits, all_positions, S_(stream));
 }
 
 int llama_forward_ragged(llama_ctx* c, const int32_t* tokens, const int32_t* start_pos, int B, float* logits,
@@ -473,7 +492,7 @@ int llama_forward_ragged(llama_ctx* c, const int32_t* tokens, const int32_t* sta
   int r;
   if ((r = check_ctx_call(c, B, 1))) return r;
   if (!tokens || !start_pos || !logits) return LLAMA_ERR_INVALID_ARGS;
-  return run_model(c, tokens, B, 1, start_pos, 0, logits, 1, S_(stream));
+  return run_model(c, tokens, 1, B, 1, start_pos, 0, logits, 1, S_(stream));
 }
 
 int llama_block_forward(llama_ctx* c, int layer, float* h, int B, int T, const int32_t* start_pos_dev,
@@ -487,16 +506,43 @@ int llama_block_forward(llama_ctx* c, int layer, float* h, int B, int T, const i
   return run_block(c, layer, h, B, T, start_pos_dev, host_start_pos, S_(stream));
 }
 
+int llama_generate(llama_ctx* c, int32_t* tokens, const uint8_t* prompt_mask, int B, int total_len,
+                   int min_prompt_len, float temperature, float top_p, const float* uniforms, void* stream) {
+  int r;
+  if ((r = check_ctx_call(c, B, 1))) return r;
+  if (!tokens || !prompt_mask || c->V <= 0) return LLAMA_ERR_INVALID_ARGS;
+  if (min_prompt_len < 1 || total_len > c->S || min_prompt_len > total_len) return LLAMA_ERR_INVALID_ARGS;
+  const bool greedy = !(temperature > 0.f);
+  if (!greedy && (!uniforms || !(top_p > 0.f) || !(top_p <= 1.f))) return LLAMA_ERR_INVALID_ARGS;
+  if (!c->gen_logits) {
+    const size_t n = (size_t)c->Bm * c->V * sizeof(float);
+    if ((r = alloc(reinterpret_cast<void**>(&c->gen_logits), n))) return r;
+    if ((r = alloc(reinterpret_cast<void**>(&c->gen_probs), n))) return r;
+  }
+  cudaStream_t st = S_(stream);
+  int prev = 0;
+  for (int cur = min_prompt_len; cur < total_len; ++cur) {
+    // Transformer.forward(tokens[:, prev:cur], prev), last position only
+    if ((r = run_model(c, tokens + prev, total_len, B, cur - prev, nullptr, prev, c->gen_logits, 0, st))) return r;
+    // next token unless the sequence's prompt still covers position cur
+    if (launch_sample(c->gen_logits, B, c->V, temperature, top_p, greedy ? nullptr : uniforms + (size_t)cur * B,
+                      c->gen_probs, tokens + cur, total_len, prompt_mask + cur, total_len, st) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    prev = cur;
+  }
+  return LLAMA_OK;
+}
+
 int llama_kv_read(llama_ctx* c, int layer, void* k, void* v, void* stream) {
   if (!c || layer < 0 || layer >= c->L || !k || !v) return LLAMA_ERR_INVALID_ARGS;
   CK(cudaSetDevice(c->device));
   Layer& Ly = c->layers[layer];
   if (c->bf16) {
-    launch_kv_convert<bf16>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
-    launch_kv_convert<bf16>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+    launch_kv_convert<bf16>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, c->half_split, S_(stream));
+    launch_kv_convert<bf16>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, 0, S_(stream));
   } else {
-    launch_kv_convert<float>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
-    launch_kv_convert<float>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, S_(stream));
+    launch_kv_convert<float>(Ly.cache_k, k, c->Bm, c->S, c->Hkv, c->D, 1, c->half_split, S_(stream));
+    launch_kv_convert<float>(Ly.cache_v, v, c->Bm, c->S, c->Hkv, c->D, 1, 0, S_(stream));
   }
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
@@ -506,11 +552,11 @@ int llama_kv_write(llama_ctx* c, int layer, const void* k, const void* v, void* 
   CK(cudaSetDevice(c->device));
   Layer& Ly = c->layers[layer];
   if (c->bf16) {
-    launch_kv_convert<bf16>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
-    launch_kv_convert<bf16>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+    launch_kv_convert<bf16>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, c->half_split, S_(stream));
+    launch_kv_convert<bf16>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, 0, S_(stream));
   } else {
-    launch_kv_convert<float>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
-    launch_kv_convert<float>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, S_(stream));
+    launch_kv_convert<float>(k, Ly.cache_k, c->Bm, c->S, c->Hkv, c->D, 0, c->half_split, S_(stream));
+    launch_kv_convert<float>(v, Ly.cache_v, c->Bm, c->S, c->Hkv, c->D, 0, 0, S_(stream));
   }
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
@@ -555,6 +601,26 @@ const char* llama_strerror(int code) {
     case LLAMA_ERR_TIMEOUT: return "a bounded device wait timed out";
     default: return "unknown error";
   }
+}
+
+int llama_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
+                 int32_t* out, void* stream) {
+  if (!logits || !out || B < 1 || V < 1) return LLAMA_ERR_INVALID_ARGS;
+  const bool greedy = !(temperature > 0.f);
+  if (!greedy && (!uniforms || !(top_p > 0.f) || !(top_p <= 1.f))) return LLAMA_ERR_INVALID_ARGS;
+  static float* scratch = nullptr;
+  static size_t scratch_n = 0;
+  if (!greedy && scratch_n < (size_t)B * V) {
+    cudaDeviceSynchronize();
+    release(reinterpret_cast<void*&>(scratch));
+    scratch_n = 0;
+    if (alloc(reinterpret_cast<void**>(&scratch), (size_t)B * V * sizeof(float))) return LLAMA_ERR_OOM;
+    scratch_n = (size_t)B * V;
+  }
+  return launch_sample(logits, B, V, temperature, top_p, uniforms, scratch, out, 1, nullptr, 0, S_(stream)) ==
+                 cudaSuccess
+             ? LLAMA_OK
+             : LLAMA_ERR_CUDA;
 }
 
 int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, int dtype, int path, void* stream) {

@@ -19,7 +19,9 @@ from .llama_oracle import (  # noqa: F401
     block_forward_rows,
     causal_gqa_attention,
     ffn_hidden_dim,
+    generate,
     rmsnorm,
     rope_tables,
+    select_next,
     silu,
 )

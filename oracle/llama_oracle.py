@@ -388,3 +388,54 @@ class OracleModel:
         for v0 in range(0, V, step):
             out[..., v0:v0 + step] = xn @ as_f64(w[v0:v0 + step]).T
         return out
+
+
+# ----------------------------------------------------------------------------
+# Generation ([P3] §3.3 generate and sample_top_p)
+# ----------------------------------------------------------------------------
+
+def select_next(logits: np.ndarray, temperature: float, top_p: float, u: Optional[float] = None) -> int:
+    """The next token from one row of logits.
+
+    temperature <= 0: argmax (the first maximum). Otherwise probs =
+    softmax(logits / temperature); sort descending (ties keep index order);
+    zero the tokens whose predecessors' cumulative probability exceeds top_p
+    (mask cum - p > top_p); renormalise; the multinomial draw is made with the
+    given uniform u: the first token in that order whose cumulative
+    renormalised probability exceeds u.
+    """
+    logits = np.asarray(logits, dtype=np.float64)
+    if not temperature > 0:
+        return int(np.argmax(logits))
+    z = logits / temperature
+    z = z - z.max()
+    e = np.exp(z)
+    probs = e / e.sum()
+    order = np.argsort(-probs, kind="stable")
+    ps = probs[order]
+    cum = np.cumsum(ps)
+    ps = np.where(cum - ps > top_p, 0.0, ps)
+    ps = ps / ps.sum()
+    c = np.cumsum(ps)
+    k = min(int(np.searchsorted(c, u, side="right")), len(ps) - 1)
+    return int(order[k])
+
+
+def generate(model: "OracleModel", tokens: np.ndarray, prompt_mask: np.ndarray, min_prompt_len: int,
+             temperature: float, top_p: float, uniforms: Optional[np.ndarray] = None) -> np.ndarray:
+    """[P3] §3.3 generate on token ids: from cur = the shortest prompt's length,
+    forward(tokens[:, prev:cur], prev) with last-position logits, select the
+    next token, keep the prompt's own token where the prompt mask is set, then
+    prev = cur. ``uniforms[cur, b]`` is the draw of sequence b at step cur.
+    Returns the completed token array (a copy)."""
+    tokens = np.array(tokens, dtype=np.int64, copy=True)
+    B, total_len = tokens.shape
+    prev = 0
+    for cur in range(min_prompt_len, total_len):
+        logits = model.forward(tokens[:, prev:cur], prev, all_positions=False)   # [B, V]
+        for b in range(B):
+            if not prompt_mask[b, cur]:
+                u = None if uniforms is None else float(uniforms[cur, b])
+                tokens[b, cur] = select_next(logits[b], temperature, top_p, u)
+        prev = cur
+    return tokens

@@ -432,3 +432,62 @@ def test_block_forward_rows_is_block_forward_restricted():
     got = O.block_forward_rows(h, m.layers[0], sp, m.args, m.cos, m.sin, rows)
     for i, (b, s) in enumerate(rows):
         np.testing.assert_allclose(got[i], full[b, s], rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- next-token selection
+
+def test_select_next_greedy_is_first_argmax():
+    logits = np.array([0.1, 3.0, -1.0, 3.0, 2.9])
+    assert O.select_next(logits, 0.0, 0.9) == 1          # first of the tied maxima
+    assert O.select_next(logits, -1.0, 0.9) == 1
+
+
+def test_select_next_top_p_hand_example():
+    # probabilities 0.5, 0.3, 0.2 (logits are their logs, temperature 1): with top_p = 0.6 the
+    # sorted cumulative sums are 0.5, 0.8, 1.0 and cum - p = 0, 0.5, 0.8, so the third token is
+    # dropped; the kept pair renormalises to 0.625, 0.375.
+    logits = np.log(np.array([0.2, 0.5, 0.3]))           # indices 1, 2, 0 in descending order
+    assert O.select_next(logits, 1.0, 0.6, 0.10) == 1
+    assert O.select_next(logits, 1.0, 0.6, 0.62) == 1
+    assert O.select_next(logits, 1.0, 0.6, 0.63) == 2
+    assert O.select_next(logits, 1.0, 0.6, 0.99) == 2    # token 0 never drawn
+    # top_p = 1 keeps everything: plain inverse CDF over 0.5, 0.3, 0.2
+    assert O.select_next(logits, 1.0, 1.0, 0.85) == 0
+
+
+def test_select_next_frequencies_follow_renormalised_top_p():
+    rng = np.random.default_rng(11)
+    logits = rng.standard_normal(40) * 2.0
+    T, top_p = 0.7, 0.8
+    z = np.exp((logits - logits.max()) / T)
+    probs = z / z.sum()
+    order = np.argsort(-probs, kind="stable")
+    cum = np.cumsum(probs[order])
+    keep = order[(cum - probs[order]) <= top_p]
+    target = np.zeros(40)
+    target[keep] = probs[keep] / probs[keep].sum()
+    us = (np.arange(20000) + 0.5) / 20000                 # a uniform grid of draws
+    counts = np.bincount([O.select_next(logits, T, top_p, u) for u in us], minlength=40) / len(us)
+    np.testing.assert_allclose(counts, target, atol=2e-4)
+
+
+def test_generate_keeps_prompts_and_matches_stepwise_forward():
+    w, lws, enh = _tiny(n_layers=1)
+    m = build_oracle(w, lws, enh)
+    rng = np.random.default_rng(12)
+    total = 12
+    tokens = np.zeros((2, total), dtype=np.int64)
+    tokens[0, :5] = rng.integers(0, w.vocab_size, 5)
+    tokens[1, :8] = rng.integers(0, w.vocab_size, 8)
+    mask = np.zeros((2, total), dtype=bool)
+    mask[0, :5] = True
+    mask[1, :8] = True
+    out = O.generate(m, tokens, mask, 5, 0.0, 1.0)
+    np.testing.assert_array_equal(out[0, :5], tokens[0, :5])
+    np.testing.assert_array_equal(out[1, :8], tokens[1, :8])
+    # greedy continuation of sequence 0 equals argmax of a one-sequence recompute at each step
+    m2 = build_oracle(w, lws, enh)
+    for cur in range(5, total):
+        logits = m2.forward(out[:1, :cur], 0, all_positions=False)
+        m2 = build_oracle(w, lws, enh)
+        assert out[0, cur] == int(np.argmax(logits[0]))
