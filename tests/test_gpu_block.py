@@ -40,7 +40,8 @@ def _run(pair: Pair, h: torch.Tensor, start_pos, tol_hidden):
     return got
 
 
-@pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 2), (512, 4, 4), (256, 4, 1), (1024, 8, 1), (1024, 8, 8)])
+@pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 2), (512, 4, 4), (256, 4, 1), (1024, 8, 1), (1024, 8, 8),
+                                       (2048, 16, 1), (4096, 32, 1)])
 def test_block_prefill_chunk_and_decode(dim, H, Hkv):
     w = _wl(dim, H, Hkv)
     pair = Pair(w)
@@ -124,5 +125,27 @@ def test_position_past_cache_raises_device_flag():
         assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
         with pytest.raises(B.LlamaError):
             B.llama_block_forward(pair.ctx, 0, torch.zeros((3, 1, 512), device="cuda"), 0)  # B > max_batch
+    finally:
+        pair.close()
+
+
+def test_long_context_prefill_rows_and_decode():
+    """A 16384-position cache (RoPE table of 32768 positions): a 4096-token chunk
+    appended at start_pos 12000 after a prefill, then a decode step at 16383."""
+    w = _wl(512, 4, 1, Bm=1, S=16384)
+    pair = Pair(w)
+    try:
+        h = synth.hidden(w, (1, 1000, 512), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        # jump: positions 1000..11999 stay zero on both sides (zero keys and values)
+        h = synth.hidden(w, (1, 4096, 512), call=1)
+        _run(pair, h, 12000, BF16_HIDDEN_ABS)
+        h = synth.hidden(w, (1, 1, 512), call=2)
+        _run(pair, h, 16383, BF16_HIDDEN_ABS)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[0, :1000] = True
+        written[0, 12000:16096] = True
+        written[0, 16383] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
     finally:
         pair.close()
