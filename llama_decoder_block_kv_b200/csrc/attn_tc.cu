@@ -37,8 +37,8 @@ struct AttnTcCfg {
   static constexpr int HALVES = D / 64;
   static constexpr uint32_t Q_BYTES = 128 * D * 2;   // two (or one) 128 x 64 boxes
   static constexpr uint32_t KV_BYTES = KT * D * 2;   // one K or one V tile
-  static constexpr uint32_t P_BYTES = 128 * KT * 2;  // 128 rows x 64 keys
-  static constexpr size_t SMEM = 1024 + Q_BYTES + RING * 2 * KV_BYTES + P_BYTES + 256;
+  static constexpr uint32_t P_BYTES = 128 * KT * 2;  // 128 rows x 64 keys (two buffers)
+  static constexpr size_t SMEM = 1024 + Q_BYTES + RING * 2 * KV_BYTES + 2 * P_BYTES + 256;
   static constexpr uint32_t TMEM_COLS = 256;  // S0, S1 (64 columns each), O (D columns)
 };
 
@@ -92,15 +92,15 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = base;
   uint8_t* sKV = sQ + Cfg::Q_BYTES;                 // RING x (K, V)
   uint8_t* sP = sKV + RING * 2 * Cfg::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + Cfg::P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * Cfg::P_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;          // [RING]
   uint64_t* kv_empty = kv_full + RING;   // [RING]
   uint64_t* s_full = kv_empty + RING;    // [2]
   uint64_t* s_free = s_full + 2;         // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drained = o_done + 1;
+  uint64_t* p_full = s_free + 2;         // [2] per P buffer
+  uint64_t* o_done = p_full + 2;         // [2] PV(j) completes o_done[j & 1]
+  uint64_t* drained = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -125,8 +125,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
     mbar_init(drained, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -200,17 +202,17 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (j >= 1) {
           const int jp = j - 1, stp = jp % RING;
-          if (!wait_or_abort(p_full, jp & 1, err, abort_flag)) break;
+          if (!wait_or_abort(&p_full[jp & 1], (jp >> 1) & 1, err, abort_flag)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(sKV + stp * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < KT / 16; ++kk) {
             // A = P (K-major: 128 rows x 64 keys); B = V N-major: 16 keys (2048 B) per step,
             // 64-wide d blocks 8 KB apart (leading byte offset), 8-key groups 1 KB apart
-            tc_mma_bf16(tmem + 2 * KT, make_sw128_desc(p_addr + kk * 32),
+            tc_mma_bf16(tmem + 2 * KT, make_sw128_desc(p_addr + (jp & 1) * Cfg::P_BYTES + kk * 32),
                         make_sw128_desc_lbo(v_addr + kk * 2048, 8192, 1024), idesc_pv, (jp | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(o_done);
+          tc_commit(&o_done[jp & 1]);
           tc_commit(&kv_empty[stp]);
         }
       }
@@ -249,9 +251,9 @@ __global__ void __launch_bounds__(192, 1)
         s[c] = v;
         mt = fmaxf(mt, v);
       }
-      // PV(j-1) must be complete before O is rescaled or the P buffer is rewritten
-      if (j >= 1) {
-        ok = wait_or_abort(o_done, (j - 1) & 1, err, abort_flag);
+      // P(j) goes to buffer j & 1, last read by PV(j-2)
+      if (j >= 2) {
+        ok = wait_or_abort(&o_done[j & 1], ((j - 2) >> 1) & 1, err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -261,6 +263,13 @@ __global__ void __launch_bounds__(192, 1)
       if (j == 0) {
         m_used = mt;
       } else if (__any_sync(0xffffffffu, mt > m_used + RESCALE_LOG2)) {
+        // O is rescaled in TMEM only once PV(j-1) has finished accumulating into it
+        ok = wait_or_abort(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const float m_new = fmaxf(m_used, mt);
         const float alpha = exp2f(m_used - m_new);
         l *= alpha;
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(192, 1)
         m_used = m_new;
       }
       // P row -> bf16 in the 128-byte-swizzled K-major layout the MMA reads
-      uint8_t* prow = sP + r * 128;
+      uint8_t* prow = sP + (j & 1) * Cfg::P_BYTES + r * 128;
 #pragma unroll
       for (int c8 = 0; c8 < KT / 8; ++c8) {
         float pv[8];
@@ -294,10 +303,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
     if (ok) {
-      ok = wait_or_abort(o_done, (n - 1) & 1, err, abort_flag);
+      ok = wait_or_abort(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {

@@ -41,7 +41,7 @@ def _run(pair: Pair, h: torch.Tensor, start_pos, tol_hidden):
 
 
 @pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 2), (512, 4, 4), (256, 4, 1), (1024, 8, 1), (1024, 8, 8),
-                                       (2048, 16, 1), (4096, 32, 1)])
+                                       (2048, 16, 1), (2048, 32, 1)])
 def test_block_prefill_chunk_and_decode(dim, H, Hkv):
     w = _wl(dim, H, Hkv)
     pair = Pair(w)
