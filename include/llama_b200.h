@@ -67,6 +67,11 @@ extern "C" {
 #define LLAMA_PATH_GEMV 2    /* weight-streaming split-K kernel for M <= 32 (bf16) */
 #define LLAMA_PATH_SIMT 3    /* fp32 CUDA-core tiled GEMM (fp32 or bf16) */
 
+/* Kernels of decode calls (T == 1), llama_set_decode_kernel */
+#define LLAMA_DECODE_AUTO 0       /* one persistent launch per block when the shapes allow, else LAYERED */
+#define LLAMA_DECODE_LAYERED 1    /* a kernel per step: RMSNorm, GEMV, attention, GEMV, RMSNorm, GEMV, GEMV */
+#define LLAMA_DECODE_PERSISTENT 2 /* always the persistent launch; an ineligible decode call fails */
+
 /*
  * ModelArgs of the notes' section 3 code plus rope_theta ("灵哥讲llama3(中)",
  * Transformer class) and the storage type.
@@ -226,8 +231,31 @@ int llama_generate(llama_ctx* ctx, int32_t* tokens_dev, const uint8_t* prompt_ma
 int llama_kv_read(llama_ctx* ctx, int layer, void* k_dev, void* v_dev, void* cuda_stream);
 int llama_kv_write(llama_ctx* ctx, int layer, const void* k_dev, const void* v_dev, void* cuda_stream);
 
-/* Zero every cache (synchronous). */
+/* Zero every cache and re-arm the workspace's arrival counters (synchronous). */
 int llama_reset(llama_ctx* ctx);
+
+/*
+ * Choose how decode calls (T == 1) of this context run one block
+ * (LLAMA_DECODE_*). Both compute TransformerBlock.forward of the notes; they
+ * differ only in the order of fp32 sums. The pages have no counterpart: this
+ * is a launch-structure switch of the library.
+ *  LLAMA_DECODE_LAYERED: seven kernels per block and step (RMSNorm, QKV GEMV
+ *   with RoPE and the cache append, split-K decode attention, wo GEMV plus
+ *   residual, RMSNorm, w1|w3 GEMV with SwiGLU, w2 GEMV plus residual).
+ *  LLAMA_DECODE_PERSISTENT: one launch per block and step with one CTA per SM
+ *   that streams all four weight matrices while its consumer warps walk the
+ *   steps in order, separated by grid-wide barriers; the RMSNorms are fused
+ *   into the loads of the linears' inputs. Eligible when dtype == LLAMA_BF16,
+ *   B <= 32, head_dim == 128, dim % 128 == 0 and ffn % 64 == 0; an ineligible
+ *   decode call returns LLAMA_ERR_INVALID_ARGS before any launch. The grid
+ *   barriers need all of the launch's CTAs resident at once: on a GPU whose
+ *   SMs are partly held by work on other streams or processes a barrier can
+ *   wait past its bound, which raises LLAMA_ERR_TIMEOUT on the device flag.
+ *  LLAMA_DECODE_AUTO (the default): PERSISTENT when eligible, else LAYERED.
+ * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it
+ * applies to calls made after it.
+ */
+int llama_set_decode_kernel(llama_ctx* ctx, int mode);
 
 /*
  * Synchronise the device, then return and clear the device flags: LLAMA_OK,

@@ -28,12 +28,13 @@ LLAMA_ERR_TOKEN_RANGE = -10
 LLAMA_ERR_POS_RANGE = -11
 LLAMA_ERR_TIMEOUT = -12
 LLAMA_PATH_AUTO, LLAMA_PATH_TCGEN05, LLAMA_PATH_GEMV, LLAMA_PATH_SIMT = 0, 1, 2, 3
+LLAMA_DECODE_AUTO, LLAMA_DECODE_LAYERED, LLAMA_DECODE_PERSISTENT = 0, 1, 2
 
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
-            "llama_linear_noalloc", "llama_sample", "llama_generate")
+            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -82,6 +83,7 @@ def lib() -> ctypes.CDLL:
         L.llama_linear_noalloc.argtypes = [vp, vp, vp, i, i, i, vp]
         L.llama_sample.argtypes = [vp, i, i, f, f, vp, vp, vp]
         L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
+        L.llama_set_decode_kernel.argtypes = [vp, i]
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -204,6 +206,10 @@ def llama_kv_write(ctx, layer: int, k: torch.Tensor, v: torch.Tensor, stream=Non
 
 def llama_reset(ctx) -> None:
     _check(lib().llama_reset(ctx), "llama_reset")
+
+
+def llama_set_decode_kernel(ctx, mode: int) -> None:
+    _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel")
 
 
 def llama_get_error(ctx):

@@ -84,4 +84,48 @@ template <typename T>
 cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, void* o, const int* sp, int sp_scalar,
                                int B, int T_, int H, int Hkv, int D, int S_max, cudaStream_t st);
 
+
+// decode_block.cu: one decode step of a whole block in one persistent launch
+constexpr int DB_RING_STAGES = 9;                 // 16 KB weight tiles in flight per SM
+constexpr uint32_t DB_AREA_BYTES = 64 * 1024;     // x slice of a linear / K,V tiles of the attention
+
+struct DbLinear {  // one linear [N][K] as stream-K stages of 128 rows x 64 k, k cut into S slices
+  int N = 0, K = 0, RB = 0, NK = 0, S = 1, total = 0;
+};
+
+struct DecodeBlockParams {
+  DbLinear lin[4];  // wqkv, wo, w1|w3, w2
+  int M, dim, H, Hkv, D, F, S_max;
+  float eps;
+  const bf16* attn_norm;
+  const bf16* ffn_norm;
+  float* h;          // [M][dim] fp32 residual stream, in/out
+  bf16* q;           // [M][H*D]
+  bf16* o;           // [M][H*D]
+  bf16* g;           // [M][F]
+  bf16* cache_k;     // this layer's cache [B_max][Hkv][S_max][D]
+  bf16* cache_v;
+  const float2* rope;
+  const int* start_pos;  // [M] device positions, or nullptr -> sp_scalar
+  int sp_scalar;
+  float* part;       // partial tiles (linears) and chunk partials (attention)
+  int* counters;     // self-resetting arrival counters
+  float* ssq;        // [dim/128][M] sums of squares of h per 128-column block
+  unsigned* gbar;    // grid barrier {arrived, generation}
+  int* err;
+  int hpc, CK, max_chunks;  // attention split
+  int ssq_ready;     // 1: ssq already holds the statistics of the incoming h
+};
+
+struct DecodeBlockPlan {
+  bool ok = false;
+  DbLinear lin[4];
+  int grid = 1, hpc = 1, CK = 128, max_chunks = 1, counters = 0;
+  size_t part_floats = 0;
+};
+DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, int S_max, int max_len,
+                                  int num_sms);
+cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st);
+size_t decode_block_smem(int M);
+
 }  // namespace llama

@@ -34,6 +34,7 @@ struct Layer {
   void* cache_k = nullptr;
   void* cache_v = nullptr;
   CUtensorMap map_k, map_v;
+  CUtensorMap map_w[4];  // wqkv, wo, w13, w2 as 128-row x 64-k TMA tiles (persistent decode kernel)
   bool set = false;
 };
 
@@ -66,6 +67,10 @@ struct llama_ctx {
   size_t part_floats = 0;
   int* counters = nullptr;
   int counters_n = 0;
+  // persistent decode kernel: grid-barrier words and per-128-column sums of squares of h
+  unsigned* gbar = nullptr;
+  float* ssq = nullptr;
+  int decode_mode = LLAMA_DECODE_AUTO;
   // generation: last-position logits and sampling scratch, [max_batch][vocab] each
   float* gen_logits = nullptr;
   float* gen_probs = nullptr;
@@ -171,11 +176,61 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
   return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+// One decode step of a block in one persistent launch (decode_block.cu), when
+// the call and the shapes allow it. Returns 1 when the call must take the
+// kernel-per-step path instead.
+int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp_dev, int sp_host,
+                         cudaStream_t st) {
+  const int max_len = sp_dev ? c->S : sp_host + 1;
+  DecodeBlockPlan pl = plan_decode_block(B, c->dim, c->H, c->Hkv, c->D, c->F, c->S, max_len, c->num_sms);
+  if (!pl.ok || pl.part_floats > c->part_floats || pl.counters > c->counters_n) return 1;
+  Layer& Ly = c->layers[layer];
+  DecodeBlockParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int i = 0; i < 4; ++i) p.lin[i] = pl.lin[i];
+  p.M = B;
+  p.dim = c->dim;
+  p.H = c->H;
+  p.Hkv = c->Hkv;
+  p.D = c->D;
+  p.F = c->F;
+  p.S_max = c->S;
+  p.eps = c->a.norm_eps;
+  p.attn_norm = reinterpret_cast<const bf16*>(Ly.attn_norm);
+  p.ffn_norm = reinterpret_cast<const bf16*>(Ly.ffn_norm);
+  p.h = h;
+  p.q = reinterpret_cast<bf16*>(c->q);
+  p.o = reinterpret_cast<bf16*>(c->o);
+  p.g = reinterpret_cast<bf16*>(c->g);
+  p.cache_k = reinterpret_cast<bf16*>(Ly.cache_k);
+  p.cache_v = reinterpret_cast<bf16*>(Ly.cache_v);
+  p.rope = c->rope;
+  p.start_pos = sp_dev;
+  p.sp_scalar = sp_host;
+  p.part = c->part;
+  p.counters = c->counters;
+  p.ssq = c->ssq;
+  p.gbar = c->gbar;
+  p.err = c->err;
+  p.hpc = pl.hpc;
+  p.CK = pl.CK;
+  p.max_chunks = pl.max_chunks;
+  p.ssq_ready = 0;
+  return launch_decode_block(Ly.map_w, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
   Layer& Ly = c->layers[layer];
   const int M = B * T;
   const int HD = c->H * c->D;
   int r;
+  if (c->bf16 && T == 1 && c->decode_mode != LLAMA_DECODE_LAYERED && c->gbar) {
+    r = run_block_persistent(c, layer, h, B, sp_dev, sp_host, st);
+    if (r != 1) return r;
+    if (c->decode_mode == LLAMA_DECODE_PERSISTENT) return LLAMA_ERR_INVALID_ARGS;
+  } else if (T == 1 && c->decode_mode == LLAMA_DECODE_PERSISTENT) {
+    return LLAMA_ERR_INVALID_ARGS;
+  }
   if (c->bf16)
     launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
   else
@@ -356,6 +411,11 @@ int llama_create(const llama_args* args, llama_ctx** out) {
       const uint64_t rows = (uint64_t)c->Bm * c->Hkv * c->S;
       if (!make_tmap_bf16(&Ly.map_k, Ly.cache_k, rows, D, 64) || !make_tmap_bf16(&Ly.map_v, Ly.cache_v, rows, D, 64))
         return fail(LLAMA_ERR_CUDA);
+      if (!make_tmap_bf16(&Ly.map_w[0], Ly.wqkv, c->n_qkv, c->dim, 128) ||
+          !make_tmap_bf16(&Ly.map_w[1], Ly.wo, c->dim, c->H * D, 128) ||
+          !make_tmap_bf16(&Ly.map_w[2], Ly.w13, 2 * F, c->dim, 128) ||
+          !make_tmap_bf16(&Ly.map_w[3], Ly.w2, c->dim, F, 128))
+        return fail(LLAMA_ERR_CUDA);
     }
   }
   if (c->V > 0) {
@@ -387,12 +447,23 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     }
     const size_t dec = (size_t)c->Bm * c->H * ((c->S + 127) / 128) * (128 + 2);
     if (dec > need) need = dec;
+    // the persistent decode kernel, for every batch it serves
+    for (int m = 1; m <= c->Bm && m <= 32; ++m) {
+      DecodeBlockPlan pl = plan_decode_block(m, c->dim, c->H, c->Hkv, D, F, c->S, c->S, c->num_sms);
+      if (!pl.ok) continue;
+      if (pl.part_floats > need) need = pl.part_floats;
+      if (pl.counters > rbs) rbs = pl.counters;
+    }
     c->part_floats = need;
     if ((r = alloc(reinterpret_cast<void**>(&c->part), need * sizeof(float)))) return fail(r);
     if (rbs < c->Bm * c->H) rbs = c->Bm * c->H;  // decode attention: one counter per (sequence, head group)
     c->counters_n = rbs;
     if ((r = alloc(reinterpret_cast<void**>(&c->counters), (size_t)rbs * sizeof(int)))) return fail(r);
     cudaMemset(c->counters, 0, (size_t)rbs * sizeof(int));
+    if ((r = alloc(reinterpret_cast<void**>(&c->gbar), 2 * sizeof(unsigned)))) return fail(r);
+    cudaMemset(c->gbar, 0, 2 * sizeof(unsigned));
+    const int bm = c->Bm < 32 ? c->Bm : 32;
+    if ((r = alloc(reinterpret_cast<void**>(&c->ssq), (size_t)(c->dim / 64) * bm * sizeof(float)))) return fail(r);
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLAMA_ERR_CUDA);
   *out = c;
@@ -420,6 +491,8 @@ void llama_destroy(llama_ctx* c) {
   release(c->g);
   release(reinterpret_cast<void*&>(c->part));
   release(reinterpret_cast<void*&>(c->counters));
+  release(reinterpret_cast<void*&>(c->gbar));
+  release(reinterpret_cast<void*&>(c->ssq));
   release(reinterpret_cast<void*&>(c->gen_logits));
   release(reinterpret_cast<void*&>(c->gen_probs));
   delete c;
@@ -569,7 +642,15 @@ int llama_reset(llama_ctx* c) {
     CK(cudaMemset(Ly.cache_k, 0, bytes));
     CK(cudaMemset(Ly.cache_v, 0, bytes));
   }
+  if (c->counters) CK(cudaMemset(c->counters, 0, (size_t)c->counters_n * sizeof(int)));
+  if (c->gbar) CK(cudaMemset(c->gbar, 0, 2 * sizeof(unsigned)));
   CK(cudaDeviceSynchronize());
+  return LLAMA_OK;
+}
+
+int llama_set_decode_kernel(llama_ctx* c, int mode) {
+  if (!c || mode < LLAMA_DECODE_AUTO || mode > LLAMA_DECODE_PERSISTENT) return LLAMA_ERR_INVALID_ARGS;
+  c->decode_mode = mode;
   return LLAMA_OK;
 }
 
@@ -582,7 +663,13 @@ int llama_get_error(llama_ctx* c, int* flags) {
   CK(cudaMemcpy(&f, c->err, sizeof(int), cudaMemcpyDeviceToHost));
   CK(cudaMemset(c->err, 0, sizeof(int)));
   if (flags) *flags = f;
-  if (f & LLAMA_DEV_TIMEOUT) return LLAMA_ERR_TIMEOUT;
+  if (f & LLAMA_DEV_TIMEOUT) {
+    // a wait that gave up can leave arrival counters mid-count: re-arm them
+    if (c->counters) cudaMemset(c->counters, 0, (size_t)c->counters_n * sizeof(int));
+    if (c->gbar) cudaMemset(c->gbar, 0, 2 * sizeof(unsigned));
+    cudaDeviceSynchronize();
+    return LLAMA_ERR_TIMEOUT;
+  }
   if (f & LLAMA_DEV_POS_RANGE) return LLAMA_ERR_POS_RANGE;
   if (f & LLAMA_DEV_TOKEN_RANGE) return LLAMA_ERR_TOKEN_RANGE;
   return LLAMA_OK;
