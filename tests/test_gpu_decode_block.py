@@ -152,7 +152,7 @@ def test_ineligible_shape_and_position_errors():
     try:
         B.llama_set_decode_kernel(pair.ctx, B.LLAMA_DECODE_PERSISTENT)
         sp = torch.tensor([5, 128], dtype=torch.int32, device="cuda")
-        B.llama_block_forward(pair.ctx, 0, torch.zeros((2, 1, 512), device="cuda"), sp)
+        B.llama_block_forward(pair.ctx, 0, synth.hidden(w, (2, 1, 512), call=0).to("cuda").contiguous(), sp)
         code, flags = B.llama_get_error(pair.ctx)
         assert code == B.LLAMA_ERR_POS_RANGE and flags & 2
         k, _ = pair.kv(0)
