@@ -68,7 +68,7 @@ extern "C" {
 #define LLAMA_PATH_SIMT 3    /* fp32 CUDA-core tiled GEMM (fp32 or bf16) */
 
 /* Kernels of decode calls (T == 1), llama_set_decode_kernel */
-#define LLAMA_DECODE_AUTO 0       /* one persistent launch per block when the shapes allow, else LAYERED */
+#define LLAMA_DECODE_AUTO 0       /* the library's choice: currently LAYERED (measured faster) */
 #define LLAMA_DECODE_LAYERED 1    /* a kernel per step: RMSNorm, GEMV, attention, GEMV, RMSNorm, GEMV, GEMV */
 #define LLAMA_DECODE_PERSISTENT 2 /* always the persistent launch; an ineligible decode call fails */
 
@@ -251,7 +251,8 @@ int llama_reset(llama_ctx* ctx);
  *   barriers need all of the launch's CTAs resident at once: on a GPU whose
  *   SMs are partly held by work on other streams or processes a barrier can
  *   wait past its bound, which raises LLAMA_ERR_TIMEOUT on the device flag.
- *  LLAMA_DECODE_AUTO (the default): PERSISTENT when eligible, else LAYERED.
+ *  LLAMA_DECODE_AUTO (the default): the path measured faster on B200 for
+ *   the decode workloads, currently LAYERED for every shape.
  * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it
  * applies to calls made after it.
  */

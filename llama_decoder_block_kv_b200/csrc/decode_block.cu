@@ -97,15 +97,15 @@ __device__ __forceinline__ float db_quad_sum(float v) {
   return v + __shfl_xor_sync(0xffffffffu, v, 2);
 }
 
-// Stream-K split of `total` stages over `grid` CTAs: CTA c owns [begin(c), begin(c+1)).
+// Stream-K split of `total` stages over `grid` CTAs: CTA c owns [begin(c),
+// begin(c+1)), begin(c) = floor(c * total / grid). All products stay below
+// 2^31 (the host checks total * grid). owner(x), the CTA whose range holds
+// stage x, is the largest c with begin(c) <= x: floor(((x + 1) grid - 1) / total).
 __host__ __device__ __forceinline__ int db_begin(int c, int total, int grid) {
-  return (int)(((long long)c * total) / grid);
+  return (int)((unsigned)c * (unsigned)total / (unsigned)grid);
 }
 __host__ __device__ __forceinline__ int db_owner(int x, int total, int grid) {
-  int c = (int)(((long long)x * grid) / total);
-  while (c + 1 < grid && db_begin(c + 1, total, grid) <= x) ++c;
-  while (c > 0 && db_begin(c, total, grid) > x) --c;
-  return c;
+  return (int)(((unsigned)(x + 1) * (unsigned)grid - 1u) / (unsigned)total);
 }
 
 // CTAs that take part in a linear: all of them, or one per stage when the
@@ -123,12 +123,14 @@ struct DbStage {
   int s, rb, start, len, reg_beg;  // slice, row block, first k stage and k stages of the slice, region start
 };
 __host__ __device__ __forceinline__ int db_slice_start(const DbLinear& L, int s) {
-  return (int)(((long long)s * L.NK) / L.S);
+  return (int)((unsigned)s * (unsigned)L.NK / (unsigned)L.S);
 }
 __host__ __device__ __forceinline__ DbStage db_locate(const DbLinear& L, int x) {
-  int s = (int)(((long long)x * L.S) / L.total);
-  while (s + 1 < L.S && L.RB * db_slice_start(L, s + 1) <= x) ++s;
+  // slice s holds stages [RB * start(s), RB * start(s+1)): the largest s with RB * floor(s NK / S) <= x
+  int s = (int)(((unsigned)(x / L.RB + 1) * (unsigned)L.S - 1u) / (unsigned)L.NK);
+  if (s >= L.S) s = L.S - 1;
   while (s > 0 && L.RB * db_slice_start(L, s) > x) --s;
+  while (s + 1 < L.S && L.RB * db_slice_start(L, s + 1) <= x) ++s;
   DbStage r;
   r.s = s;
   r.start = db_slice_start(L, s);
@@ -156,22 +158,39 @@ __host__ __device__ __forceinline__ int db_contributors(const DbLinear& L, int r
   return count;
 }
 
-// Grid-wide barrier of the consumer threads (generation counting; the last
-// arriver re-arms the counter, so nothing needs clearing between launches).
-__device__ __forceinline__ void db_grid_sync(unsigned* gbar, int grid, int* err, volatile int* abort_flag) {
+// Grid-wide barrier of the consumer threads. gbar[0] counts arrivals and only
+// ever grows: every barrier takes exactly `grid` arrivals, so the arrival that
+// returns v belongs to barrier number k = v / grid + 1, and the arrival that
+// makes the count k * grid (the last one) publishes k in gbar[16], a separate
+// 128-byte line that the other CTAs poll. Nothing is re-armed between barriers
+// or launches (a timed-out wait leaves the count misaligned; the host clears
+// both words when it reads the timeout flag).
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void db_grid_sync(unsigned long long* gbar, int grid, int* err, volatile int* abort_flag) {
   bar_consumers();
   if (threadIdx.x == 0 && !*abort_flag) {
-    unsigned* arrived = gbar;
-    unsigned* gen = gbar + 1;
-    const unsigned g0 = ld_acquire_gpu(gen);
-    __threadfence();
-    if (atomicAdd(arrived, 1u) == (unsigned)grid - 1u) {
-      atomicExch(arrived, 0u);
-      __threadfence();
-      st_release_gpu(gen, g0 + 1u);
+    const unsigned long long G = (unsigned long long)grid;
+    const unsigned long long v = atom_add_acq_rel_gpu(gbar, 1ull);
+    const unsigned long long k = v / G + 1ull;
+    if (v + 1ull == k * G) {
+      st_release_gpu_u64(gbar + 16, k);
     } else {
       const uint64_t t0 = global_timer_ns();
-      while (ld_acquire_gpu(gen) == g0) {
+      while (ld_acquire_gpu_u64(gbar + 16) < k) {
         if (global_timer_ns() - t0 > LLAMA_WAIT_LIMIT_NS) {
           atomicOr(err, LLAMA_DEV_TIMEOUT);
           *abort_flag = 1;
@@ -181,6 +200,80 @@ __device__ __forceinline__ void db_grid_sync(unsigned* gbar, int grid, int* err,
     }
   }
   bar_consumers();
+}
+
+// L2 prefetch of one weight tile (no shared-memory destination, no completion)
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// This CTA's stages of the four linears in launch order, walked with
+// increments (a division only when a linear starts): linear li, stage x,
+// and the tile it names, k stage start + kl of row block rb.
+struct DbCursor {
+  int li, x, end;
+  int rb, kl, len, start, s;
+};
+__device__ __forceinline__ void db_cursor_enter(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
+  for (; c.li < 4; ++c.li) {
+    db_range(p.lin[c.li], cta, grid, c.x, c.end);
+    if (c.x < c.end) {
+      const DbStage S = db_locate(p.lin[c.li], c.x);
+      c.s = S.s;
+      c.rb = S.rb;
+      c.start = S.start;
+      c.len = S.len;
+      c.kl = c.x - S.reg_beg;
+      return;
+    }
+  }
+}
+__device__ __forceinline__ void db_cursor_init(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
+  c.li = 0;
+  db_cursor_enter(c, p, cta, grid);
+}
+__device__ __forceinline__ void db_cursor_next(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
+  if (++c.x >= c.end) {
+    ++c.li;
+    db_cursor_enter(c, p, cta, grid);
+    return;
+  }
+  if (++c.kl == c.len) {
+    c.kl = 0;
+    if (++c.rb == p.lin[c.li].RB) {
+      c.rb = 0;
+      ++c.s;
+      c.start = db_slice_start(p.lin[c.li], c.s);
+      c.len = db_slice_start(p.lin[c.li], c.s + 1) - c.start;
+    }
+  }
+}
+
+// L2 prefetch of the cache rows this CTA's attention units will read (the
+// host enables it when the whole launch's rows fit comfortably in L2). The
+// row at this step's position is written later in the launch; L2 is the point
+// of coherence, so the write simply replaces the prefetched line.
+__device__ void db_prefetch_kv(const DecodeBlockParams& p, int cta, int grid) {
+  const int n_rep = p.H / p.Hkv, groups = n_rep / p.hpc;
+  const int units = p.M * p.Hkv * groups * p.max_chunks;
+  for (int u = cta; u < units; u += grid) {
+    const int z = u / p.max_chunks, chunk = u - z * p.max_chunks;
+    const int b = z / (p.Hkv * groups), kvh = (z / groups) % p.Hkv;
+    const int sp = p.start_pos ? p.start_pos[b] : p.sp_scalar;
+    const int L = min(sp + 1, p.S_max);
+    const int k_begin = chunk * p.CK;
+    if (k_begin >= L) continue;
+    const int k_end = min(L, k_begin + p.CK);
+    const size_t off = ((size_t)(b * p.Hkv + kvh) * p.S_max + k_begin) * AD;
+    const uint32_t bytes = (uint32_t)(k_end - k_begin) * AD * 2;
+    bulk_prefetch_l2(p.cache_k + off, bytes);
+    bulk_prefetch_l2(p.cache_v + off, bytes);
+  }
 }
 
 // ------------------------------------------------------------------ phases
@@ -209,7 +302,21 @@ __device__ int db_load_x(const DecodeBlockParams& p, int li, int k0, int klen, u
   const int ksp = klen + 8, per_row = klen / 8;
   bf16* xs = reinterpret_cast<bf16*>(area);
   if (li == 0 || li == 2) {
-    if (tid < M) {
+    if (p.norm_local) {
+      // the slice is the whole row: its sums of squares, one warp per row
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int m = warp; m < M; m += 4) {
+        const float* hr = p.h + (size_t)m * p.dim;
+        float ss = 0.f;
+        for (int i = lane * 4; i < p.dim; i += 128) {
+          const float4 a = __ldcg(reinterpret_cast<const float4*>(hr + i));
+          ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) s_r[m] = rsqrtf(ss / (float)p.dim + p.eps);
+      }
+    } else if (tid < M) {
       float ss = 0.f;
       for (int rb = 0; rb < p.dim / RPC; ++rb) ss += __ldcg(p.ssq + rb * M + tid);
       s_r[tid] = rsqrtf(ss / (float)p.dim + p.eps);
@@ -662,6 +769,7 @@ __global__ void __launch_bounds__(160, 1)
   float* os = reinterpret_cast<float*>(area + DB_AREA_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(os + 8 * MB * OS);
   uint64_t* empty = full + STAGES;
+  unsigned long long* gbar = reinterpret_cast<unsigned long long*>(p.gbar);
   __shared__ int s_abort;
   __shared__ int s_last;
   __shared__ float s_r[32];
@@ -685,33 +793,40 @@ __global__ void __launch_bounds__(160, 1)
       const CUtensorMap* maps[4] = {&map_qkv, &map_o, &map_13, &map_2};
 #pragma unroll
       for (int i = 0; i < 4; ++i) prefetch_tensormap(maps[i]);
+      // Two cursors over this CTA's stages of the four linears: `ld` fills the
+      // ring, `pf` runs DB_L2_AHEAD stages beyond the ring and pulls tiles into
+      // L2, so that the ring's loads see L2 latency and HBM always has
+      // (ring + look-ahead) tiles of this SM in flight.
+      DbCursor ld, pf;
+      db_cursor_init(ld, p, cta, grid);
+      db_cursor_init(pf, p, cta, grid);
+      if (DB_L2_AHEAD > 0)
+        for (int i = 0; i < STAGES; ++i) db_cursor_next(pf, p, cta, grid);
+      int pf_idx = STAGES;
       int j = 0;
-      bool ok = true, waited = false;
-      for (int li = 0; li < 4 && ok; ++li) {
-        const DbLinear& L = p.lin[li];
-        int sbeg, send;
-        db_range(L, cta, grid, sbeg, send);
-        for (int x = sbeg; x < send; ++x, ++j) {
-          if (!waited && j == STAGES) {
-            // the first ring of weights is in flight before the previous kernel ends
-            pdl_wait();
-            pdl_trigger();
-            waited = true;
-          }
-          const int st = j % STAGES;
-          if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const DbStage S = db_locate(L, x);
-          const int kg = S.start + (x - S.reg_beg);
-          mbar_arrive_expect_tx(&full[st], W_BYTES);
-          tma_load_2d(ring + st * W_BYTES, maps[li], &full[st], kg * KB, S.rb * RPC);
+      bool ok = true;
+      for (; ld.li < 4; db_cursor_next(ld, p, cta, grid), ++j) {
+        if (DB_L2_AHEAD > 0)
+          for (; pf.li < 4 && pf_idx < j + STAGES + DB_L2_AHEAD; db_cursor_next(pf, p, cta, grid), ++pf_idx)
+            tma_prefetch_l2_2d(maps[pf.li], (pf.start + pf.kl) * KB, pf.rb * RPC);
+        if (j == STAGES) {
+          // the first ring of weights is in flight before the previous kernel ends
+          pdl_wait();
+          pdl_trigger();
+          if (p.kv_prefetch) db_prefetch_kv(p, cta, grid);
         }
+        const int st = j % STAGES;
+        if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, p.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], W_BYTES);
+        tma_load_2d(ring + st * W_BYTES, maps[ld.li], &full[st], (ld.start + ld.kl) * KB, ld.rb * RPC);
       }
-      if (!waited) {
+      if (j <= STAGES) {
         pdl_wait();
         pdl_trigger();
+        if (ok && p.kv_prefetch) db_prefetch_kv(p, cta, grid);
       }
       // the CTA must not retire while a copy into its shared memory is in flight
       for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.err);
@@ -723,18 +838,18 @@ __global__ void __launch_bounds__(160, 1)
   pdl_wait();
   pdl_trigger();
   int j = 0;
-  if (!p.ssq_ready) {
+  if (!p.norm_local) {
     db_sumsq_phase(p, cta, grid);
-    db_grid_sync(p.gbar, grid, p.err, abort_flag);
+    db_grid_sync(gbar, grid, p.err, abort_flag);
   }
   db_linear_phase<MB>(p, 0, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
-  db_grid_sync(p.gbar, grid, p.err, abort_flag);
+  db_grid_sync(gbar, grid, p.err, abort_flag);
   db_attention_phase(p, cta, grid, area, &s_last);
-  db_grid_sync(p.gbar, grid, p.err, abort_flag);
+  db_grid_sync(gbar, grid, p.err, abort_flag);
   db_linear_phase<MB>(p, 1, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
-  db_grid_sync(p.gbar, grid, p.err, abort_flag);
+  db_grid_sync(gbar, grid, p.err, abort_flag);
   db_linear_phase<MB>(p, 2, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
-  db_grid_sync(p.gbar, grid, p.err, abort_flag);
+  db_grid_sync(gbar, grid, p.err, abort_flag);
   db_linear_phase<MB>(p, 3, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
 }
 
@@ -774,6 +889,7 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
   for (int i = 0; i < 4; ++i) {
     DbLinear& L = pl.lin[i];
     L = db_plan_linear(M, Ns[i], Ks[i], pl.grid);
+    if ((long long)L.total * (pl.grid + 1) >= (1LL << 31)) return pl;  // index math is 32-bit
     if ((size_t)M * ((size_t)((L.NK + L.S - 1) / L.S) * KB + 8) * 2 > DB_AREA_BYTES) return pl;
     int maxc = 1;
     for (int rb = 0; rb < L.RB; ++rb) {
@@ -793,11 +909,14 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
   ck = (ck + AKT - 1) / AKT * AKT;
   if (ck < 128) ck = 128;
   pl.CK = ck;
-  pl.max_chunks = (S_max + ck - 1) / ck;
+  pl.max_chunks = (max_len + ck - 1) / ck;
+  // cache rows read by the attention: prefetched into L2 early when they are few
+  pl.kv_prefetch = (size_t)M * Hkv * max_len * AD * 2 * 2 <= ((size_t)32 << 20);
   const size_t att = (size_t)M * H * pl.max_chunks * (AD + 2);
   if (att > part) part = att;
   if (Z > counters) counters = Z;
   pl.part_floats = part;
+  pl.norm_local = pl.lin[0].S == 1 && pl.lin[2].S == 1;
   pl.counters = counters;
   pl.ok = true;
   return pl;

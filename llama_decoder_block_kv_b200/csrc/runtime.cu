@@ -129,6 +129,9 @@ std::vector<float2> rope_table(int D, int end, double theta) {
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
+// grid barrier of the persistent decode kernel: arrival counter and release word, 128 B apart
+constexpr size_t kGbarBytes = 256;
+
 int reserve(llama_ctx* c, int tokens) {
   if (tokens <= c->ws_tokens) return LLAMA_OK;
   cudaDeviceSynchronize();
@@ -215,7 +218,8 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
   p.hpc = pl.hpc;
   p.CK = pl.CK;
   p.max_chunks = pl.max_chunks;
-  p.ssq_ready = 0;
+  p.norm_local = pl.norm_local ? 1 : 0;
+  p.kv_prefetch = pl.kv_prefetch ? 1 : 0;
   return launch_decode_block(Ly.map_w, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
@@ -224,12 +228,10 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   const int M = B * T;
   const int HD = c->H * c->D;
   int r;
-  if (c->bf16 && T == 1 && c->decode_mode != LLAMA_DECODE_LAYERED && c->gbar) {
+  if (T == 1 && c->decode_mode == LLAMA_DECODE_PERSISTENT) {
+    if (!c->bf16 || !c->gbar) return LLAMA_ERR_INVALID_ARGS;
     r = run_block_persistent(c, layer, h, B, sp_dev, sp_host, st);
-    if (r != 1) return r;
-    if (c->decode_mode == LLAMA_DECODE_PERSISTENT) return LLAMA_ERR_INVALID_ARGS;
-  } else if (T == 1 && c->decode_mode == LLAMA_DECODE_PERSISTENT) {
-    return LLAMA_ERR_INVALID_ARGS;
+    return r == 1 ? LLAMA_ERR_INVALID_ARGS : r;
   }
   if (c->bf16)
     launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
@@ -460,8 +462,8 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     c->counters_n = rbs;
     if ((r = alloc(reinterpret_cast<void**>(&c->counters), (size_t)rbs * sizeof(int)))) return fail(r);
     cudaMemset(c->counters, 0, (size_t)rbs * sizeof(int));
-    if ((r = alloc(reinterpret_cast<void**>(&c->gbar), 2 * sizeof(unsigned)))) return fail(r);
-    cudaMemset(c->gbar, 0, 2 * sizeof(unsigned));
+    if ((r = alloc(reinterpret_cast<void**>(&c->gbar), kGbarBytes))) return fail(r);
+    cudaMemset(c->gbar, 0, kGbarBytes);
     const int bm = c->Bm < 32 ? c->Bm : 32;
     if ((r = alloc(reinterpret_cast<void**>(&c->ssq), (size_t)(c->dim / 64) * bm * sizeof(float)))) return fail(r);
   }
@@ -643,7 +645,7 @@ int llama_reset(llama_ctx* c) {
     CK(cudaMemset(Ly.cache_v, 0, bytes));
   }
   if (c->counters) CK(cudaMemset(c->counters, 0, (size_t)c->counters_n * sizeof(int)));
-  if (c->gbar) CK(cudaMemset(c->gbar, 0, 2 * sizeof(unsigned)));
+  if (c->gbar) CK(cudaMemset(c->gbar, 0, kGbarBytes));
   CK(cudaDeviceSynchronize());
   return LLAMA_OK;
 }
@@ -666,7 +668,7 @@ int llama_get_error(llama_ctx* c, int* flags) {
   if (f & LLAMA_DEV_TIMEOUT) {
     // a wait that gave up can leave arrival counters mid-count: re-arm them
     if (c->counters) cudaMemset(c->counters, 0, (size_t)c->counters_n * sizeof(int));
-    if (c->gbar) cudaMemset(c->gbar, 0, 2 * sizeof(unsigned));
+    if (c->gbar) cudaMemset(c->gbar, 0, kGbarBytes);
     cudaDeviceSynchronize();
     return LLAMA_ERR_TIMEOUT;
   }

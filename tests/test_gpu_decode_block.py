@@ -92,7 +92,7 @@ def test_repeated_launches_rearm_counters():
         h = synth.hidden(w, (2, 8, 512), call=0)
         _step(pair, h, 0)
         for i in range(30):
-            B.llama_set_decode_kernel(pair.ctx, B.LLAMA_DECODE_LAYERED if i % 7 == 3 else B.LLAMA_DECODE_AUTO)
+            B.llama_set_decode_kernel(pair.ctx, B.LLAMA_DECODE_LAYERED if i % 7 == 3 else B.LLAMA_DECODE_PERSISTENT)
             h = synth.hidden(w, (2, 1, 512), call=1 + i)
             _step(pair, h, 8 + i)
     finally:
@@ -139,7 +139,7 @@ def test_ineligible_shape_and_position_errors():
         with pytest.raises(B.LlamaError) as e:
             B.llama_block_forward(pair.ctx, 0, torch.zeros((2, 1, 256), device="cuda"), 3)
         assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
-        B.llama_set_decode_kernel(pair.ctx, B.LLAMA_DECODE_AUTO)   # AUTO falls back to the per-step kernels
+        B.llama_set_decode_kernel(pair.ctx, B.LLAMA_DECODE_AUTO)   # AUTO runs the per-step kernels here
         B.llama_block_forward(pair.ctx, 0, torch.zeros((2, 1, 256), device="cuda"), 3)
         assert B.llama_get_error(pair.ctx)[0] == B.LLAMA_OK
         with pytest.raises(B.LlamaError):
