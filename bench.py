@@ -143,6 +143,7 @@ class LayerBench:
         self.w = w
         self.args = B.ModelArgs.from_workload(w)
         self.model = B.Llama(self.args)
+        B.llama_set_decode_kernel(self.model.ctx, DECODE_KERNELS[DECODE_KERNEL])
         self.lw = synth.layer_weights(w, 0, device="cuda")
         B.llama_set_layer(self.model.ctx, 0, self.lw)
         dim = w.dim
@@ -368,7 +369,8 @@ def run_ours(args, world, rank, local):
            "data": "synthetic: seeded N(0,1) hidden states, N(0,0.02) weights, RMSNorm weights 1",
            "config": {"workload": w.name, "batch": lb.Bsz, "prefill_tokens": lb.P, "decode_steps": lb.ND,
                       "decode_start_pos": lb.dec_pos0, "l2": "inputs larger than L2: %.0f MB of weights per pass"
-                      % (wbytes / 1e6), "parallelism": "replicas" if world > 1 else "single GPU"},
+                      % (wbytes / 1e6), "parallelism": "replicas" if world > 1 else "single GPU",
+                      "decode_kernel": DECODE_KERNEL},
            "phases": phases, "roofline": roof, "e2e": e2e,
            "gpu_launches": lb.kernels_per_step() * args.steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -416,6 +418,7 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
     """Whole-model workloads (LLaMA-3-8B shape): ragged decode or long prefill."""
     m = B.Llama(B.ModelArgs.from_workload(w))
     ctx = m.ctx
+    B.llama_set_decode_kernel(ctx, DECODE_KERNELS[DECODE_KERNEL])
     for i in range(w.n_layers):
         B.llama_set_layer(ctx, i, synth.layer_weights(w, i, device="cuda"))
     enh = synth.embed_norm_head(w, device="cuda")
@@ -460,7 +463,7 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": w.name}, "clocks": clocks, "device_error": code}
+           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL}, "clocks": clocks, "device_error": code}
     m.close()
     return out
 
@@ -488,6 +491,11 @@ def run_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+DECODE_KERNELS = {"auto": B.LLAMA_DECODE_AUTO, "layered": B.LLAMA_DECODE_LAYERED,
+                  "persistent": B.LLAMA_DECODE_PERSISTENT}
+DECODE_KERNEL = "auto"
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,7 +504,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b-layer", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-kernel", default="auto", choices=sorted(DECODE_KERNELS),
+                    help="decode-step launch structure (llama_set_decode_kernel)")
     args = ap.parse_args()
+    global DECODE_KERNEL
+    DECODE_KERNEL = args.decode_kernel
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -46,7 +46,6 @@ constexpr int OS = RPC + 4;                 // row stride of the fp32 output sta
 constexpr int STAGES = DB_RING_STAGES;
 constexpr int AKT = 64;                     // keys per attention tile
 constexpr int AD = 128;                     // head dim of this kernel
-constexpr uint32_t ATB = AKT * AD * 2;      // one K or V tile, 16 KB
 constexpr float LOG2E_DB = 1.4426950408889634f;
 }  // namespace
 
@@ -67,16 +66,6 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 }
 __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// 16-byte asynchronous copy global -> shared through L2; src_bytes 0 fills zeros
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // swizzled byte address of (row, col) in a tile of 128-byte rows written by TMA
@@ -165,6 +154,14 @@ __host__ __device__ __forceinline__ int db_contributors(const DbLinear& L, int r
 // 128-byte line that the other CTAs poll. Nothing is re-armed between barriers
 // or launches (a timed-out wait leaves the count misaligned; the host clears
 // both words when it reads the timeout flag).
+// arrival on a counter: releases this CTA's earlier writes (all threads'
+// writes ordered before it by a bar.sync) and acquires the writes released by
+// the arrivals before it
+__device__ __forceinline__ int atom_add_acq_rel_gpu_s32(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long long* p, unsigned long long v) {
   unsigned long long old;
   asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
@@ -202,79 +199,41 @@ __device__ __forceinline__ void db_grid_sync(unsigned long long* gbar, int grid,
   bar_consumers();
 }
 
-// L2 prefetch of one weight tile (no shared-memory destination, no completion)
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// This CTA's stages of the four linears in launch order, walked with
-// increments (a division only when a linear starts): linear li, stage x,
-// and the tile it names, k stage start + kl of row block rb.
-struct DbCursor {
-  int li, x, end;
-  int rb, kl, len, start, s;
+// One attention work unit (sequence, kv head, group of query heads, chunk of
+// keys), as both roles of the CTA enumerate them.
+struct DbUnit {
+  int z, chunk, b, kvh, grp, sp, L, k_begin, k_end, nc, n_tiles;
+  size_t row0;  // first key row of the chunk in the cache [B_max][Hkv][S_max]
 };
-__device__ __forceinline__ void db_cursor_enter(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
-  for (; c.li < 4; ++c.li) {
-    db_range(p.lin[c.li], cta, grid, c.x, c.end);
-    if (c.x < c.end) {
-      const DbStage S = db_locate(p.lin[c.li], c.x);
-      c.s = S.s;
-      c.rb = S.rb;
-      c.start = S.start;
-      c.len = S.len;
-      c.kl = c.x - S.reg_beg;
-      return;
-    }
-  }
-}
-__device__ __forceinline__ void db_cursor_init(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
-  c.li = 0;
-  db_cursor_enter(c, p, cta, grid);
-}
-__device__ __forceinline__ void db_cursor_next(DbCursor& c, const DecodeBlockParams& p, int cta, int grid) {
-  if (++c.x >= c.end) {
-    ++c.li;
-    db_cursor_enter(c, p, cta, grid);
-    return;
-  }
-  if (++c.kl == c.len) {
-    c.kl = 0;
-    if (++c.rb == p.lin[c.li].RB) {
-      c.rb = 0;
-      ++c.s;
-      c.start = db_slice_start(p.lin[c.li], c.s);
-      c.len = db_slice_start(p.lin[c.li], c.s + 1) - c.start;
-    }
-  }
+__device__ __forceinline__ bool db_unit(const DecodeBlockParams& p, int u, DbUnit& w) {
+  const int groups = (p.H / p.Hkv) / p.hpc;
+  w.z = u / p.max_chunks;
+  w.chunk = u - w.z * p.max_chunks;
+  w.b = w.z / (p.Hkv * groups);
+  w.kvh = (w.z / groups) % p.Hkv;
+  w.grp = w.z % groups;
+  // positions are inputs of the call, never written by a kernel of the forward pass
+  w.sp = p.start_pos ? p.start_pos[w.b] : p.sp_scalar;
+  w.L = min(w.sp + 1, p.S_max);
+  w.k_begin = w.chunk * p.CK;
+  if (w.k_begin >= w.L) return false;  // a shorter sequence of a ragged batch
+  w.k_end = min(w.L, w.k_begin + p.CK);
+  w.nc = (w.L + p.CK - 1) / p.CK;
+  w.n_tiles = (w.k_end - w.k_begin + AKT - 1) / AKT;
+  w.row0 = (size_t)(w.b * p.Hkv + w.kvh) * p.S_max + w.k_begin;
+  return true;
 }
 
-// L2 prefetch of the cache rows this CTA's attention units will read (the
-// host enables it when the whole launch's rows fit comfortably in L2). The
-// row at this step's position is written later in the launch; L2 is the point
-// of coherence, so the write simply replaces the prefetched line.
-__device__ void db_prefetch_kv(const DecodeBlockParams& p, int cta, int grid) {
-  const int n_rep = p.H / p.Hkv, groups = n_rep / p.hpc;
-  const int units = p.M * p.Hkv * groups * p.max_chunks;
-  for (int u = cta; u < units; u += grid) {
-    const int z = u / p.max_chunks, chunk = u - z * p.max_chunks;
-    const int b = z / (p.Hkv * groups), kvh = (z / groups) % p.Hkv;
-    const int sp = p.start_pos ? p.start_pos[b] : p.sp_scalar;
-    const int L = min(sp + 1, p.S_max);
-    const int k_begin = chunk * p.CK;
-    if (k_begin >= L) continue;
-    const int k_end = min(L, k_begin + p.CK);
-    const size_t off = ((size_t)(b * p.Hkv + kvh) * p.S_max + k_begin) * AD;
-    const uint32_t bytes = (uint32_t)(k_end - k_begin) * AD * 2;
-    bulk_prefetch_l2(p.cache_k + off, bytes);
-    bulk_prefetch_l2(p.cache_v + off, bytes);
-  }
+__device__ __forceinline__ void st_release_cta_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
+__device__ __forceinline__ int ld_acquire_cta_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// orders this thread's earlier (acquired) view of global memory before its later async-proxy (TMA) reads
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // ------------------------------------------------------------------ phases
 
@@ -369,11 +328,14 @@ __device__ __forceinline__ void db_rowblock_epilogue(const DecodeBlockParams& p,
     float sq = 0.f;
     if (act) {
       float v[8];
+      float* hp = p.h + (size_t)m * p.dim + n;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+      if (residual) {
+        a = __ldcg(reinterpret_cast<const float4*>(hp));
+        b = __ldcg(reinterpret_cast<const float4*>(hp + 4));
+      }
       get(m, jc, v);
       if (residual) {
-        float* hp = p.h + (size_t)m * p.dim + n;
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(hp));
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(hp + 4));
         v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
         v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
         __stcg(reinterpret_cast<float4*>(hp), make_float4(v[0], v[1], v[2], v[3]));
@@ -513,16 +475,15 @@ __device__ void db_linear_phase(const DecodeBlockParams& p, int li, int cta, int
                                    os[m * OS + jc * 4 + 3]);
       __stcg(reinterpret_cast<float4*>(p.part + ((size_t)slot * M + m) * L.N + nbase + jc * 4), v);
     }
-    __threadfence();
     bar_consumers();
-    if (tid == 0) *s_last = (atomicAdd(&p.counters[rb], 1) == count - 1);
+    if (tid == 0) *s_last = (atom_add_acq_rel_gpu_s32(&p.counters[rb], 1) == count - 1);
     bar_consumers();
     if (!*s_last) continue;
-    __threadfence();
     db_rowblock_epilogue(p, li, rb, ep, [&](int m, int jc, float* v) {
       const int n = nbase + jc * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = 0.f;
+#pragma unroll 4
       for (int sl = 0; sl < count; ++sl) {
         const float4* src = reinterpret_cast<const float4*>(p.part + ((size_t)sl * M + m) * L.N + n);
         const float4 a = __ldcg(src), b = __ldcg(src + 1);
@@ -541,46 +502,22 @@ __device__ void db_linear_phase(const DecodeBlockParams& p, int li, int cta, int
 // warps take 16 keys of each tile, their states merge in shared memory, and
 // the unit that finishes last for a (sequence, head group) merges the chunks'
 // partials with the log-sum-exp rule in chunk order.
-__device__ void db_attention_phase(const DecodeBlockParams& p, int cta, int grid, uint8_t* area, int* s_last) {
+__device__ void db_attention_phase(const DecodeBlockParams& p, int cta, int grid, int& j, uint8_t* ring, uint8_t* area,
+                                   uint64_t* full, uint64_t* empty, volatile int* abort_flag, int* s_last) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, qd = lane & 3;
-  const int n_rep = p.H / p.Hkv, hpc = p.hpc, groups = n_rep / hpc;
-  const int Z = p.M * p.Hkv * groups;
-  const int units = Z * p.max_chunks;
+  const int n_rep = p.H / p.Hkv, hpc = p.hpc;
+  const int units = p.M * p.Hkv * (n_rep / hpc) * p.max_chunks;
   const float sl2 = rsqrtf((float)AD) * LOG2E_DB;
   float* part_o = p.part;
   float* part_ml = p.part + (size_t)p.M * p.H * p.max_chunks * AD;
-  const uint32_t abase = smem_u32(area);
 
   for (int u = cta; u < units; u += grid) {
-    const int z = u / p.max_chunks, chunk = u - z * p.max_chunks;
-    const int b = z / (p.Hkv * groups);
-    const int kvh = (z / groups) % p.Hkv;
-    const int grp = z % groups;
-    const int sp = p.start_pos ? p.start_pos[b] : p.sp_scalar;
-    const int L = min(sp + 1, p.S_max);
-    const int k_begin = chunk * p.CK;
-    if (k_begin >= L) continue;  // a shorter sequence of a ragged batch (CTA-uniform)
-    const int k_end = min(L, k_begin + p.CK);
-    const int nc = (L + p.CK - 1) / p.CK;
-    const int n_tiles = (k_end - k_begin + AKT - 1) / AKT;
-    const size_t row0 = (size_t)(b * p.Hkv + kvh) * p.S_max + k_begin;
-    const int h0 = kvh * n_rep + grp * hpc;
-
-    auto load_tile = [&](int jt, int stage) {
-      const uint32_t kd = abase + stage * 2 * ATB, vd = kd + ATB;
-      for (int c = tid; c < AKT * (AD / 8); c += 128) {
-        const int r = c >> 4, dc = c & 15;
-        const bool valid = k_begin + jt * AKT + r < k_end;
-        const size_t goff = valid ? ((row0 + jt * AKT + r) * AD + dc * 8) : 0;
-        const uint32_t soff = (dc >> 3) * 8192 + r * 128 + (((dc & 7) ^ (r & 7)) << 4);
-        cp_async16(kd + soff, p.cache_k + goff, valid ? 16u : 0u);
-        cp_async16(vd + soff, p.cache_v + goff, valid ? 16u : 0u);
-      }
-      cp_async_commit();
-    };
-    load_tile(0, 0);
-    if (n_tiles > 1) load_tile(1, 1);
+    DbUnit w;
+    if (!db_unit(p, u, w)) continue;  // CTA-uniform
+    const int b = w.b, chunk = w.chunk, z = w.z, k_begin = w.k_begin, k_end = w.k_end, nc = w.nc;
+    const int n_tiles = w.n_tiles;
+    const int h0 = w.kvh * n_rep + w.grp * hpc;
 
     // query rows g and g + 8: heads h0 + g, h0 + g + 8 when inside the group
     uint32_t qa[AD / 16][4];
@@ -601,16 +538,15 @@ __device__ void db_attention_phase(const DecodeBlockParams& p, int cta, int grid
     for (int i = 0; i < AD / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    for (int jt = 0; jt < n_tiles; ++jt) {
-      if (jt + 1 < n_tiles)
-        cp_async_wait<1>();
-      else
-        cp_async_wait<0>();
-      bar_consumers();
+    for (int jt = 0; jt < n_tiles; ++jt, j += 2) {
+      // the K tile then the V tile of keys k_begin + 64 jt .., two ring stages
+      const int stk = j % STAGES, stv = (j + 1) % STAGES;
+      const bool okk = wait_or_abort(&full[stk], (j / STAGES) & 1, p.err, abort_flag);
+      const bool okv = wait_or_abort(&full[stv], ((j + 1) / STAGES) & 1, p.err, abort_flag);
       const int key0 = k_begin + jt * AKT + 16 * warp;  // first key of this warp's 16
-      if (key0 < k_end) {
-        const uint32_t kb = abase + (jt & 1) * 2 * ATB;
-        const uint32_t vb = kb + ATB;
+      if (__all_sync(0xffffffffu, okk && okv) && key0 < k_end) {
+        const uint32_t kb = smem_u32(ring + stk * W_BYTES);
+        const uint32_t vb = smem_u32(ring + stv * W_BYTES);
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < AD / 16; ++kk) {
@@ -680,11 +616,15 @@ __device__ void db_attention_phase(const DecodeBlockParams& p, int cta, int grid
           mma_bf16_16816(oacc[jd + 1], pl, b1);
         }
       }
-      bar_consumers();  // the stage is free again
-      if (jt + 2 < n_tiles) load_tile(jt + 2, jt & 1);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[stk]);
+        mbar_arrive(&empty[stv]);
+      }
     }
 
-    // merge the 4 warps' states through shared memory (the tiles are done)
+    // merge the 4 warps' states through shared memory
+    bar_consumers();  // the previous unit's merge has finished reading the area
     l0 = db_quad_sum(l0);
     l1 = db_quad_sum(l1);
     float* sm_o = reinterpret_cast<float*>(area);  // [4][16][AD]
@@ -729,12 +669,10 @@ __device__ void db_attention_phase(const DecodeBlockParams& p, int cta, int grid
       }
     }
     if (nc > 1) {
-      __threadfence();
       bar_consumers();
-      if (tid == 0) *s_last = (atomicAdd(&p.counters[z], 1) == nc - 1);
+      if (tid == 0) *s_last = (atom_add_acq_rel_gpu_s32(&p.counters[z], 1) == nc - 1);
       bar_consumers();
       if (*s_last) {
-        __threadfence();
         for (int e = tid; e < hpc * AD; e += 128) {
           const int r = e / AD, d = e - r * AD;
           const size_t row = ((size_t)b * p.H + h0 + r) * p.max_chunks;
@@ -761,6 +699,7 @@ template <int MB>
 __global__ void __launch_bounds__(160, 1)
     decode_block_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_o,
                         const __grid_constant__ CUtensorMap map_13, const __grid_constant__ CUtensorMap map_2,
+                        const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                         const __grid_constant__ DecodeBlockParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -772,6 +711,8 @@ __global__ void __launch_bounds__(160, 1)
   unsigned long long* gbar = reinterpret_cast<unsigned long long*>(p.gbar);
   __shared__ int s_abort;
   __shared__ int s_last;
+  __shared__ int s_qkv_done_word;
+  int* s_qkv_done = &s_qkv_done_word;
   __shared__ float s_r[32];
   volatile int* abort_flag = &s_abort;
 
@@ -783,50 +724,109 @@ __global__ void __launch_bounds__(160, 1)
       mbar_init(&empty[i], 4);
     }
     s_abort = 0;
+    s_qkv_done_word = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
+    // One stream of 16 KB ring stages in the consumers' order: this CTA's
+    // wqkv tiles, the K and V tiles of its attention units, then its wo, w1|w3
+    // and w2 tiles. Weights never wait for the activations. A cache tile
+    // that ends before the step's position holds rows written by earlier calls
+    // and is loaded at once (during the wqkv phase); the tile holding the
+    // position waits until the consumers have passed the barrier after wqkv,
+    // whose epilogue writes that row.
     if (lane == 0) {
       const CUtensorMap* maps[4] = {&map_qkv, &map_o, &map_13, &map_2};
 #pragma unroll
       for (int i = 0; i < 4; ++i) prefetch_tensormap(maps[i]);
-      // Two cursors over this CTA's stages of the four linears: `ld` fills the
-      // ring, `pf` runs DB_L2_AHEAD stages beyond the ring and pulls tiles into
-      // L2, so that the ring's loads see L2 latency and HBM always has
-      // (ring + look-ahead) tiles of this SM in flight.
-      DbCursor ld, pf;
-      db_cursor_init(ld, p, cta, grid);
-      db_cursor_init(pf, p, cta, grid);
-      if (DB_L2_AHEAD > 0)
-        for (int i = 0; i < STAGES; ++i) db_cursor_next(pf, p, cta, grid);
-      int pf_idx = STAGES;
+      prefetch_tensormap(&map_k);
+      prefetch_tensormap(&map_v);
       int j = 0;
-      bool ok = true;
-      for (; ld.li < 4; db_cursor_next(ld, p, cta, grid), ++j) {
-        if (DB_L2_AHEAD > 0)
-          for (; pf.li < 4 && pf_idx < j + STAGES + DB_L2_AHEAD; db_cursor_next(pf, p, cta, grid), ++pf_idx)
-            tma_prefetch_l2_2d(maps[pf.li], (pf.start + pf.kl) * KB, pf.rb * RPC);
-        if (j == STAGES) {
-          // the first ring of weights is in flight before the previous kernel ends
+      bool ok = true, waited = false;
+      // a free ring stage, armed for `bytes`; the previous kernel is waited for
+      // once the first ring of weights is in flight
+      auto next_stage = [&](uint32_t bytes) -> int {
+        if (!waited && j == STAGES) {
           pdl_wait();
           pdl_trigger();
-          if (p.kv_prefetch) db_prefetch_kv(p, cta, grid);
+          waited = true;
         }
         const int st = j % STAGES;
-        if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, p.err, abort_flag)) {
-          ok = false;
-          break;
+        if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, p.err, abort_flag)) return -1;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        return st;
+      };
+      auto produce_linear = [&](int li) {
+        const DbLinear& L = p.lin[li];
+        int x, end;
+        db_range(L, cta, grid, x, end);
+        if (x >= end) return;
+        const DbStage S = db_locate(L, x);
+        int rb = S.rb, kl = x - S.reg_beg, sl = S.s, start = S.start, len = S.len;
+        for (; x < end; ++x, ++j) {
+          const int st = next_stage(W_BYTES);
+          if (st < 0) {
+            ok = false;
+            return;
+          }
+          tma_load_2d(ring + st * W_BYTES, maps[li], &full[st], (start + kl) * KB, rb * RPC);
+          if (++kl == len) {
+            kl = 0;
+            if (++rb == L.RB) {
+              rb = 0;
+              ++sl;
+              start = db_slice_start(L, sl);
+              len = db_slice_start(L, sl + 1) - start;
+            }
+          }
         }
-        mbar_arrive_expect_tx(&full[st], W_BYTES);
-        tma_load_2d(ring + st * W_BYTES, maps[ld.li], &full[st], (ld.start + ld.kl) * KB, ld.rb * RPC);
-      }
-      if (j <= STAGES) {
+      };
+      produce_linear(0);
+      if (ok && !waited) {
         pdl_wait();
         pdl_trigger();
-        if (ok && p.kv_prefetch) db_prefetch_kv(p, cta, grid);
+        waited = true;
+      }
+      const int units = p.M * p.Hkv * ((p.H / p.Hkv) / p.hpc) * p.max_chunks;
+      bool fresh = false;  // the row at the position is visible to this thread's TMA reads
+      for (int u = cta; ok && u < units; u += grid) {
+        DbUnit w;
+        if (!db_unit(p, u, w)) continue;
+        for (int jt = 0; ok && jt < w.n_tiles; ++jt) {
+          const int key0 = w.k_begin + jt * AKT;
+          if (!fresh && key0 + AKT > w.sp) {
+            const uint64_t t0 = global_timer_ns();
+            while (!ld_acquire_cta_shared(s_qkv_done)) {
+              if (*abort_flag || global_timer_ns() - t0 > LLAMA_WAIT_LIMIT_NS) {
+                if (!*abort_flag) atomicOr(p.err, LLAMA_DEV_TIMEOUT);
+                *abort_flag = 1;
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+            fence_proxy_async_global();
+            fresh = true;
+          }
+          for (int kv = 0; kv < 2; ++kv, ++j) {
+            const int st = next_stage(W_BYTES);
+            if (st < 0) {
+              ok = false;
+              break;
+            }
+            const CUtensorMap* m = kv ? &map_v : &map_k;
+            tma_load_2d(ring + st * W_BYTES, m, &full[st], 0, (int)(w.row0 + jt * AKT));
+            tma_load_2d(ring + st * W_BYTES + 8192, m, &full[st], 64, (int)(w.row0 + jt * AKT));
+          }
+        }
+      }
+      for (int li = 1; li < 4 && ok; ++li) produce_linear(li);
+      if (!waited) {
+        pdl_wait();
+        pdl_trigger();
       }
       // the CTA must not retire while a copy into its shared memory is in flight
       for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.err);
@@ -844,7 +844,8 @@ __global__ void __launch_bounds__(160, 1)
   }
   db_linear_phase<MB>(p, 0, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
   db_grid_sync(gbar, grid, p.err, abort_flag);
-  db_attention_phase(p, cta, grid, area, &s_last);
+  if (tid == 0) st_release_cta_shared(s_qkv_done, 1);
+  db_attention_phase(p, cta, grid, j, ring, area, full, empty, abort_flag, &s_last);
   db_grid_sync(gbar, grid, p.err, abort_flag);
   db_linear_phase<MB>(p, 1, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
   db_grid_sync(gbar, grid, p.err, abort_flag);
@@ -903,15 +904,13 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
   // attention: about one work unit per CTA, chunks of at least 128 keys
   pl.hpc = hpc;
   const int Z = M * Hkv * (n_rep / hpc);
-  int want = (pl.grid + Z - 1) / Z;
+  int want = pl.grid / Z;  // chunks per (sequence, head group): at most one unit per CTA
   if (want < 1) want = 1;
   int ck = (max_len + want - 1) / want;
   ck = (ck + AKT - 1) / AKT * AKT;
   if (ck < 128) ck = 128;
   pl.CK = ck;
   pl.max_chunks = (max_len + ck - 1) / ck;
-  // cache rows read by the attention: prefetched into L2 early when they are few
-  pl.kv_prefetch = (size_t)M * Hkv * max_len * AD * 2 * 2 <= ((size_t)32 << 20);
   const size_t att = (size_t)M * H * pl.max_chunks * (AD + 2);
   if (att > part) part = att;
   if (Z > counters) counters = Z;
@@ -932,7 +931,8 @@ static cudaError_t db_launch(const CUtensorMap* maps, const DecodeBlockParams& p
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(decode_block_kernel<MB>, dim3(grid), dim3(160), smem, st, maps[0], maps[1], maps[2], maps[3], p);
+  return launch_pdl(decode_block_kernel<MB>, dim3(grid), dim3(160), smem, st, maps[0], maps[1], maps[2], maps[3],
+                    maps[4], maps[5], p);
 }
 
 cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st) {

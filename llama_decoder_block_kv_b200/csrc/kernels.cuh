@@ -88,7 +88,6 @@ cudaError_t launch_attn_simple(const void* q, const void* ck, const void* cv, vo
 // decode_block.cu: one decode step of a whole block in one persistent launch
 constexpr int DB_RING_STAGES = 9;                 // 16 KB weight tiles in flight per SM
 constexpr uint32_t DB_AREA_BYTES = 64 * 1024;     // x slice of a linear / K,V tiles of the attention
-constexpr int DB_L2_AHEAD = 0;                    // weight tiles prefetched into L2 beyond the ring, per SM (0: off)
 
 struct DbLinear {  // one linear [N][K] as stream-K stages of 128 rows x 64 k, k cut into S slices
   int N = 0, K = 0, RB = 0, NK = 0, S = 1, total = 0;
@@ -116,18 +115,18 @@ struct DecodeBlockParams {
   int* err;
   int hpc, CK, max_chunks;  // attention split
   int norm_local;    // 1: a linear's x slice is the whole row; RMSNorm statistics are computed where it is loaded
-  int kv_prefetch;   // 1: prefetch the attention's cache rows into L2 at the start
 };
 
 struct DecodeBlockPlan {
   bool ok = false;
   DbLinear lin[4];
   int grid = 1, hpc = 1, CK = 128, max_chunks = 1, counters = 0;
-  bool norm_local = false, kv_prefetch = false;
+  bool norm_local = false;
   size_t part_floats = 0;
 };
 DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, int S_max, int max_len,
                                   int num_sms);
+// maps: wqkv, wo, w1|w3, w2 (128-row x 64-k boxes), then the layer's K and V caches (64-row x 64 boxes)
 cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st);
 size_t decode_block_smem(int M);
 

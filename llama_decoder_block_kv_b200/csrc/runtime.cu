@@ -219,8 +219,8 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
   p.CK = pl.CK;
   p.max_chunks = pl.max_chunks;
   p.norm_local = pl.norm_local ? 1 : 0;
-  p.kv_prefetch = pl.kv_prefetch ? 1 : 0;
-  return launch_decode_block(Ly.map_w, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  const CUtensorMap maps[6] = {Ly.map_w[0], Ly.map_w[1], Ly.map_w[2], Ly.map_w[3], Ly.map_k, Ly.map_v};
+  return launch_decode_block(maps, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
