@@ -486,13 +486,11 @@ __global__ void __launch_bounds__(160)
   // The CTA that finishes last for this (sequence, head group) merges every
   // chunk's partial with the log-sum-exp rule, in chunk order (deterministic),
   // and re-arms the counter for the next launch.
-  __threadfence();
   asm volatile("bar.sync 1, 128;" ::: "memory");
   __shared__ int s_last;
-  if (threadIdx.x == 0) s_last = (atomicAdd(&counters[z], 1) == nc - 1);
+  if (threadIdx.x == 0) s_last = (atomic_add_acq_rel(&counters[z], 1) == nc - 1);
   asm volatile("bar.sync 1, 128;" ::: "memory");
   if (!s_last) return;
-  __threadfence();
   for (int e = threadIdx.x; e < hpc * D; e += 128) {
     const int r = e / D, d = e - r * D;
     const size_t row = ((size_t)b * H + h0 + r) * max_chunks;

@@ -257,6 +257,16 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   }
 }
 
+// Arrival on a global counter with acquire-release semantics at GPU scope:
+// releases this thread's earlier writes and the writes of its CTA ordered
+// before it by a bar.sync, and acquires the writes released by the arrivals
+// before it (one L2 round trip where a fence plus an atomic takes two).
+__device__ __forceinline__ int atomic_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // 2-D tiled TMA load (no multicast) into this CTA's shared memory, completing
 // on an mbarrier with a transaction-byte count.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {

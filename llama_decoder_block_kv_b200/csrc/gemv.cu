@@ -218,24 +218,36 @@ __global__ void __launch_bounds__(160, 1)
         __stcg(reinterpret_cast<float4*>(part + ((size_t)slot * M + m) * N + n), v);
       }
     }
-    __threadfence();
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (tid == 0) s_last = (atomicAdd(&counters[rb], 1) == count - 1);
+    if (tid == 0) s_last = (atomic_add_acq_rel(&counters[rb], 1) == count - 1);
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (!s_last) continue;
-    __threadfence();
     for (int c = tid; c < M * (RPC / 8); c += 128) {
       const int m = c / (RPC / 8), jc = c - m * (RPC / 8);
       const int n = nbase + jc * 8;
       if (n >= N) continue;
+      // the residual row is fetched before the partial sums, not after them
+      const bool res = ep.kind == EPI_RESIDUAL;
+      float4* hp = res ? reinterpret_cast<float4*>(ep.out + (size_t)m * ep.ld_out + n) : nullptr;
+      float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0;
+      if (res) {
+        h0 = hp[0];
+        h1 = hp[1];
+      }
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
       for (int sl = 0; sl < count; ++sl) {
         const float4* src = reinterpret_cast<const float4*>(part + ((size_t)sl * M + m) * N + n);
         const float4 a = __ldcg(src), b = __ldcg(src + 1);
         v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
         v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
       }
-      epilogue8<bf16>(ep, m, n, v);
+      if (res) {
+        hp[0] = make_float4(h0.x + v[0], h0.y + v[1], h0.z + v[2], h0.w + v[3]);
+        hp[1] = make_float4(h1.x + v[4], h1.y + v[5], h1.z + v[6], h1.w + v[7]);
+      } else {
+        epilogue8<bf16>(ep, m, n, v);
+      }
     }
     if (tid == 0) counters[rb] = 0;
   }
