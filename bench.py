@@ -189,10 +189,9 @@ class LayerBench:
         return g
 
     def kernels_per_step(self):
-        pre = 7 if self.P else 0            # rmsnorm, gemm x4, attention, rmsnorm
-        dec = 8                             # rmsnorm, gemv, attn, combine, gemv, rmsnorm, gemv, gemv
-        if self.Bsz * 1 > 32:
-            dec = 7
+        pre = 7 if self.P else 0  # rmsnorm, gemm x2, attention, rmsnorm, gemm x2 (the QKV and wo GEMMs: 4 in all)
+        # decode: rmsnorm, gemv, attention (chunk merge fused), gemv, rmsnorm, gemv, gemv; or one persistent launch
+        dec = 1 if DECODE_KERNEL == "persistent" else 7
         return pre + self.ND * dec
 
     def decode_gemms(self):
@@ -441,6 +440,9 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
             for s in range(w.decode_steps):
                 B.llama_forward_ragged(ctx, toks[s], pos[s], logits)
         tokens_per_step = w.batch * w.decode_steps
+        # per forward: embedding, the blocks, final RMSNorm, LM head
+        per_block = 1 if DECODE_KERNEL == "persistent" else 7
+        launches_per_step = w.decode_steps * (1 + w.n_layers * per_block + 2)
     else:
         toks = synth.tokens(w, (w.batch, w.prefill_len), 0, "cuda")
         logits = torch.empty((w.batch, w.vocab_size), device="cuda")
@@ -449,6 +451,7 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
         def enqueue():
             B.llama_forward(ctx, toks, 0, logits, False)
         tokens_per_step = w.batch * w.prefill_len
+        launches_per_step = 1 + w.n_layers * 7 + 2
     enqueue()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -463,7 +466,8 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL}, "clocks": clocks, "device_error": code}
+           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL}, "clocks": clocks, "device_error": code,
+           "gpu_launches": launches_per_step * args.steps}
     m.close()
     return out
 
