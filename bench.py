@@ -49,6 +49,84 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+class NvmlClockSampler:
+    """Read-only NVML sampling of the SM clock and the clock-event reasons every
+    ~5 ms from a thread while the timed region runs (short regions still get
+    samples; a final sample is taken at stop). Falls back to nvidia-smi."""
+    REASONS = (("hw_slowdown", "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksThrottleReasonSwPowerCap", 0x4))
+
+    def __init__(self, index: int):
+        self.index = index
+        self.fallback = None
+        self.samples = []
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_sm = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.bits = {n: getattr(pynvml, c, b) for n, c, b in self.REASONS}
+        except Exception:
+            self.nv = None
+            self.fallback = ClockSampler(index)
+
+    def _sample(self):
+        nv = self.nv
+        sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((time.time(), sm, int(r)))
+
+    def _run(self):
+        while not self.done.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            self.done.wait(0.005)
+
+    def start(self):
+        if self.fallback is not None:
+            return self.fallback.start()
+        import threading
+        self.done = threading.Event()
+        self._sample()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.fallback is not None:
+            return self.fallback.stop()
+        self.done.set()
+        self.thread.join(timeout=5)
+        try:
+            self._sample()
+        except Exception:
+            pass
+        reasons = set()
+        for _, _, r in self.samples:
+            for n, b in self.bits.items():
+                if r & b:
+                    reasons.add(n)
+        sm = [x[1] for x in self.samples]
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as f:
+                f.write("time,clocks.sm,clocks.max.sm,reasons_bits\n")
+                for t, c, r in self.samples:
+                    f.write(f"{t:.4f},{c:.0f},{self.max_sm:.0f},{r:#x}\n")
+        except Exception:
+            pass
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_sm, "samples": len(sm),
+                "reasons": sorted(reasons), "source": "nvml"}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -228,7 +306,7 @@ def time_graph(g, steps, warmup, world):
 # capture profiles/gemv_bf16_m1_n22016_k4096.md (dram read + write of one
 # launch / weights + activations + outputs). Valid for the kernel version that
 # capture names; set to None when the kernel changes until it is re-measured.
-GEMV_TRAFFIC_RATIO = (181.597184e6 + 5.217792e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
+GEMV_TRAFFIC_RATIO = (181.60e6 + 3.34e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
 
 
 def gemv_roofline(lb: LayerBench, peaks, reps=10):
@@ -323,7 +401,7 @@ def run_ours(args, world, rank, local):
         return run_model_bench(args, world, rank, local, w, peaks, peak_kind)
     lb = LayerBench(w)
     g = lb.capture("all")
-    sampler = ClockSampler(local)
+    sampler = NvmlClockSampler(local)
     barrier(world)
     sampler.start()
     ms = time_graph(g, args.steps, args.warmup, world)
@@ -457,7 +535,7 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         enqueue()
-    sampler = ClockSampler(local)
+    sampler = NvmlClockSampler(local)
     sampler.start()
     ms = max_over_ranks(time_graph(g, args.steps, args.warmup, world), world)
     clocks = sampler.stop()
