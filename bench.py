@@ -62,7 +62,7 @@ class NvmlClockSampler:
         self.index = index
         self.fallback = None
         self.samples = []
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(CLOCK_LOG_DIR, f"clocks_rank{index}.csv")
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -136,7 +136,7 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(CLOCK_LOG_DIR, f"clocks_rank{index}.csv")
 
     def start(self):
         try:
@@ -303,7 +303,7 @@ def time_graph(g, steps, warmup, world):
 
 
 # DRAM traffic per algorithmic byte of the decode GEMV, from the committed ncu
-# capture profiles/gemv_bf16_m1_n22016_k4096.md (dram read + write of one
+# capture of one w1|w3 launch, M=1, N=22016, K=4096 (dram read + write of one
 # launch / weights + activations + outputs). Valid for the kernel version that
 # capture names; set to None when the kernel changes until it is re-measured.
 GEMV_TRAFFIC_RATIO = (181.60e6 + 3.34e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
@@ -342,7 +342,7 @@ def gemv_roofline(lb: LayerBench, peaks, reps=10):
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
             "traffic_source": "ncu dram read+write of the w1|w3 launch scaled by algorithmic bytes "
-                              "(profiles/gemv_bf16_m1_n22016_k4096.md)",
+                              "(M=1, N=22016, K=4096)",
             "bytes_per_launch": int(per_launch), "avg_launch_us": round(t_ms * 1e3, 2),
             "launches_timed": launches}
 
@@ -576,6 +576,7 @@ def run_reference(args, world, rank):
 DECODE_KERNELS = {"auto": B.LLAMA_DECODE_AUTO, "layered": B.LLAMA_DECODE_LAYERED,
                   "persistent": B.LLAMA_DECODE_PERSISTENT}
 DECODE_KERNEL = "auto"
+CLOCK_LOG_DIR = os.environ.get("TMPDIR", "/tmp")
 
 
 def main():
@@ -586,11 +587,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b-layer", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None, help="directory for the per-rank clock sample CSV")
     ap.add_argument("--decode-kernel", default="auto", choices=sorted(DECODE_KERNELS),
                     help="decode-step launch structure (llama_set_decode_kernel)")
     args = ap.parse_args()
-    global DECODE_KERNEL
+    global DECODE_KERNEL, CLOCK_LOG_DIR
     DECODE_KERNEL = args.decode_kernel
+    if args.clock_log:
+        CLOCK_LOG_DIR = args.clock_log
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -27,8 +27,8 @@ Sources, cited by page title and section throughout:
 [P5] "灵哥讲llama3(中)" (blog.csdn.net/RussellTheRush/article/details/139664760):
      Transformer class (rope_theta, the cached causal-mask comment).
 
-Readings where the pages are silent or disagree are listed in the design doc and
-restated at the function that applies them.
+Readings where the pages are silent or disagree are stated at the function
+that applies them.
 """
 from __future__ import annotations
 
