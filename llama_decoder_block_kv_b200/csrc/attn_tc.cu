@@ -62,6 +62,13 @@ __device__ __forceinline__ uint64_t make_sw128_desc_lbo(uint32_t smem_addr, uint
   return d;
 }
 
+// 2^x on the special-function unit (inputs below -126 give 0; -inf gives 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tmem_st_32cols(uint32_t taddr, const float* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -243,14 +250,22 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld_32cols(lane_base + (j & 1) * KT + 32, s + 32);
       tc_fence_before();
       mbar_arrive(&s_free[j & 1]);
-      float mt = -INFINITY;
+      // row maximum of the raw scores (masked keys -inf), four independent chains
       const int key0 = j * KT;
+      if (__any_sync(0xffffffffu, key0 + KT - 1 > p_row)) {
 #pragma unroll
-      for (int c = 0; c < KT; ++c) {
-        const float v = (key0 + c <= p_row) ? s[c] * sl2 : -INFINITY;
-        s[c] = v;
-        mt = fmaxf(mt, v);
+        for (int c = 0; c < KT; ++c)
+          if (key0 + c > p_row) s[c] = -INFINITY;
       }
+      float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int c = 4; c < KT; c += 4) {
+        mx[0] = fmaxf(mx[0], s[c]);
+        mx[1] = fmaxf(mx[1], s[c + 1]);
+        mx[2] = fmaxf(mx[2], s[c + 2]);
+        mx[3] = fmaxf(mx[3], s[c + 3]);
+      }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;  // log2 units
       // P(j) goes to buffer j & 1, last read by PV(j-2)
       if (j >= 2) {
         ok = wait_or_abort(&o_done[j & 1], ((j - 2) >> 1) & 1, err, abort_flag);
@@ -284,15 +299,17 @@ __global__ void __launch_bounds__(192, 1)
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         m_used = m_new;
       }
-      // P row -> bf16 in the 128-byte-swizzled K-major layout the MMA reads
+      // P row -> bf16 in the 128-byte-swizzled K-major layout the MMA reads;
+      // p = 2^(s * log2(e)/sqrt(D) - m) is one FMA and one ex2
       uint8_t* prow = sP + (j & 1) * Cfg::P_BYTES + r * 128;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c8 = 0; c8 < KT / 8; ++c8) {
         float pv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          pv[e] = exp2f(s[c8 * 8 + e] - m_used);
-          l += pv[e];
+          pv[e] = ex2_approx(fmaf(s[c8 * 8 + e], sl2, -m_used));
+          ls[e & 3] += pv[e];
         }
         uint4 u;
         u.x = pack_bf16x2(pv[0], pv[1]);
@@ -301,6 +318,7 @@ __global__ void __launch_bounds__(192, 1)
         u.w = pack_bf16x2(pv[6], pv[7]);
         *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = u;
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[j & 1]);
