@@ -317,14 +317,17 @@ def gemv_roofline(lb: LayerBench, peaks, reps=10):
     pairs = lb.decode_gemms()
     ys = [torch.empty((x.shape[0], w.shape[0]), device="cuda") for x, w in pairs]
     byts = sum(w.numel() * 2 + x.numel() * 2 + x.shape[0] * w.shape[0] * 4 for x, w in pairs)
-    for (x, w), y in zip(pairs, ys):
-        B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+    # the weights in the tile layout the library keeps for its own linears
+    tiles = [(x, B.llama_tile_weights(w), w.shape[0]) for x, w in pairs]
+    path = B.LLAMA_PATH_GEMV | B.LLAMA_WEIGHTS_TILED
+    for (x, wt, n), y in zip(tiles, ys):
+        B.llama_linear(x, wt, y, path, n=n)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for _ in range(reps):
-            for (x, w), y in zip(pairs, ys):
-                B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+            for (x, wt, n), y in zip(tiles, ys):
+                B.llama_linear(x, wt, y, path, n=n)
     g.replay()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()

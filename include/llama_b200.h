@@ -66,6 +66,7 @@ extern "C" {
 #define LLAMA_PATH_TCGEN05 1 /* TMA + tcgen05/TMEM tensor-core GEMM (bf16) */
 #define LLAMA_PATH_GEMV 2    /* weight-streaming split-K kernel for M <= 32 (bf16) */
 #define LLAMA_PATH_SIMT 3    /* fp32 CUDA-core tiled GEMM (fp32 or bf16) */
+#define LLAMA_WEIGHTS_TILED 16 /* OR-ed into a path: w holds llama_tile_weights tiles (bf16, GEMV or TCGEN05) */
 
 /* Kernels of decode calls (T == 1), llama_set_decode_kernel */
 #define LLAMA_DECODE_AUTO 0       /* the library's choice: currently LAYERED (measured faster) */
@@ -271,12 +272,26 @@ int llama_get_error(llama_ctx* ctx, int* flags);
 const char* llama_strerror(int code);
 
 /*
+ * The weight layout the library keeps for its bf16 linears (the pages have no
+ * counterpart; it is a storage choice): w_dev [N][K] bf16 row-major is cut into
+ * tiles of 128 rows x 64 columns, tile (n / 128, k / 64) stored contiguously
+ * (16 KB) at tile index (n / 128) * (K / 64) + k / 64, rows past N zero-filled.
+ * out_dev must hold ceil(N / 128) * 128 * K bf16 values. Rules: K % 64 == 0,
+ * both pointers 16-byte aligned, the two regions disjoint. Stream-ordered.
+ * Every decode and prefill GEMM then reads each 128 x 64 operand stage as one
+ * contiguous 16 KB block.
+ */
+int llama_tile_weights(const void* w_dev, void* out_dev, int N, int K, void* cuda_stream);
+
+/*
  * Diagnostics: y_dev[M][N] (fp32) = x_dev[M][K] * w_dev[N][K]^T with fp32
  * accumulation, x and w both of storage type dtype, through the chosen GEMM
- * path (LLAMA_PATH_*). Rules: M, N, K > 0, N % 8 == 0, K % 8 == 0;
+ * path (LLAMA_PATH_*), optionally OR-ed with LLAMA_WEIGHTS_TILED when w_dev
+ * holds llama_tile_weights tiles. Rules: M, N, K > 0, N % 8 == 0, K % 8 == 0;
  * LLAMA_PATH_GEMV needs M <= 32 and K % 64 == 0; LLAMA_PATH_TCGEN05 needs
- * dtype == LLAMA_BF16. Uses a private, lazily allocated workspace; not
- * thread-safe.
+ * dtype == LLAMA_BF16; tiled weights need dtype == LLAMA_BF16, K % 64 == 0
+ * and the GEMV or TCGEN05 path. Uses a private, lazily allocated workspace;
+ * not thread-safe.
  */
 int llama_linear(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, int dtype, int path,
                  void* cuda_stream);

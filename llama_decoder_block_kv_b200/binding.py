@@ -28,13 +28,14 @@ LLAMA_ERR_TOKEN_RANGE = -10
 LLAMA_ERR_POS_RANGE = -11
 LLAMA_ERR_TIMEOUT = -12
 LLAMA_PATH_AUTO, LLAMA_PATH_TCGEN05, LLAMA_PATH_GEMV, LLAMA_PATH_SIMT = 0, 1, 2, 3
+LLAMA_WEIGHTS_TILED = 16
 LLAMA_DECODE_AUTO, LLAMA_DECODE_LAYERED, LLAMA_DECODE_PERSISTENT = 0, 1, 2
 
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
-            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel")
+            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel", "llama_tile_weights")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -84,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.llama_sample.argtypes = [vp, i, i, f, f, vp, vp, vp]
         L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
         L.llama_set_decode_kernel.argtypes = [vp, i]
+        L.llama_tile_weights.argtypes = [vp, vp, i, i, vp]
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -209,7 +211,7 @@ def llama_reset(ctx) -> None:
 
 
 def llama_set_decode_kernel(ctx, mode: int) -> None:
-    _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel")
+    _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel", "llama_tile_weights")
 
 
 def llama_get_error(ctx):
@@ -219,9 +221,19 @@ def llama_get_error(ctx):
     return code, flags.value
 
 
-def llama_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, path: int = LLAMA_PATH_AUTO, stream=None) -> None:
+def llama_tile_weights(w: torch.Tensor, stream=None) -> torch.Tensor:
+    """The library's tile layout of a bf16 [N][K] weight matrix (returned as a new tensor)."""
+    N, K = w.shape
+    out = torch.empty(((N + 127) // 128 * 128 * K,), dtype=torch.bfloat16, device=w.device)
+    _check(lib().llama_tile_weights(_ptr(w), _ptr(out), N, K, _stream(stream)), "llama_tile_weights")
+    return out
+
+
+def llama_linear(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, path: int = LLAMA_PATH_AUTO, stream=None,
+                 n: Optional[int] = None) -> None:
+    """y = x w^T; w is [N][K], or with path | LLAMA_WEIGHTS_TILED the tiles of llama_tile_weights (pass n = N)."""
     M, K = x.shape
-    N = w.shape[0]
+    N = w.shape[0] if n is None else n
     dt = LLAMA_BF16 if x.dtype == torch.bfloat16 else LLAMA_FP32
     _check(lib().llama_linear(_ptr(x), _ptr(w), _ptr(y), M, N, K, dt, int(path), _stream(stream)), "llama_linear")
 

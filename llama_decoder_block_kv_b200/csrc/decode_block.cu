@@ -772,7 +772,8 @@ __global__ void __launch_bounds__(160, 1)
             ok = false;
             return;
           }
-          tma_load_2d(ring + st * W_BYTES, maps[li], &full[st], (start + kl) * KB, rb * RPC);
+          // the library's weight tiles: tile (rb, k stage) at rows (rb * NK + k stage) * 128 of the map
+          tma_load_2d(ring + st * W_BYTES, maps[li], &full[st], 0, (rb * L.NK + start + kl) * RPC);
           if (++kl == len) {
             kl = 0;
             if (++rb == L.RB) {

@@ -105,6 +105,33 @@ __global__ void pack_w13_kernel(const T* __restrict__ w1, const T* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
+// Weight tiles: the bf16 weights of a block are stored as contiguous 16 KB
+// tiles of 128 rows x 64 k, tile (rb, kb) at index rb * (K/64) + kb, so each
+// 128 x 64 operand stage of the GEMV and the tensor-core GEMM is one
+// contiguous 16 KB read instead of 128 row pieces of 128 bytes. Element
+// (n, k) goes to tile (n / 128, k / 64), row n % 128, column k % 64; rows past
+// N are zero.
+__global__ void tile_weights_kernel(const bf16* __restrict__ src, bf16* __restrict__ dst, int N, int K) {
+  const int nk = K / 64;
+  const size_t chunks = tiled_weight_elems(N, K) / 8;  // 16-byte pieces of the destination
+  for (size_t c = blockIdx.x * (size_t)blockDim.x + threadIdx.x; c < chunks; c += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = c * 8;
+    const size_t tile = e / (128 * 64);
+    const int in_tile = (int)(e - tile * (128 * 64));
+    const int r = in_tile / 64, col = in_tile % 64;
+    const int rb = (int)(tile / nk), kb = (int)(tile - (size_t)rb * nk);
+    const int n = rb * 128 + r, k = kb * 64 + col;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (n < N) v = *reinterpret_cast<const uint4*>(src + (size_t)n * K + k);
+    *reinterpret_cast<uint4*>(dst + e) = v;
+  }
+}
+
+void launch_tile_weights(const void* src, void* dst, int N, int K, cudaStream_t st) {
+  tile_weights_kernel<<<1184, 256, 0, st>>>(reinterpret_cast<const bf16*>(src), reinterpret_cast<bf16*>(dst), N, K);
+}
+
+// ---------------------------------------------------------------------------
 // Half-split RoPE weights (pairs (i, i + D/2) of each head) into the
 // interleaved order the kernels rotate (pairs (2i, 2i+1)): row 2i of a head
 // takes row i, row 2i+1 takes row i + D/2. q.k products are unchanged.

@@ -46,7 +46,7 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, int num_m, int num_n) 
 template <typename T, int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M, int N,
-                   int K, EpiParams ep) {
+                   int K, int b_tiled, EpiParams ep) {
   using Cfg = TcCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -110,7 +110,15 @@ __global__ void __launch_bounds__(192, 1)
           }
           mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_BYTES);
           tma_load_2d(sA + stage * Cfg::A_BYTES, &map_a, &full[stage], kb * BK, tc.mb * BM);
-          tma_load_2d(sB + stage * Cfg::B_BYTES, &map_b, &full[stage], kb * BK, tc.nb * BN);
+          if (b_tiled) {
+            // B in 128-row x 64-k tiles, tile (rb, kb) at rows (rb * num_k + kb) * 128 of the map
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              tma_load_2d(sB + stage * Cfg::B_BYTES + h * 16384, &map_b, &full[stage], 0,
+                          ((tc.nb * (BN / 128) + h) * num_k + kb) * 128);
+          } else {
+            tma_load_2d(sB + stage * Cfg::B_BYTES, &map_b, &full[stage], kb * BK, tc.nb * BN);
+          }
         }
       }
       if (!ok) {
@@ -241,6 +249,15 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of a weight matrix [N][K]: row-major (box 64 columns x box_rows
+// rows), or, when tiled, the library's tile layout [ceil(N/128)][K/64][128][64]
+// seen as rows of 64 elements (box 64 x box_rows rows, one tile per 128 rows).
+bool make_tmap_weights(CUtensorMap* map, const void* ptr, int tiled, uint64_t N, uint64_t K, uint32_t box_rows) {
+  if (!tiled) return make_tmap_bf16(map, ptr, N, K, box_rows);
+  const uint64_t rows = (N + 127) / 128 * 128 * (K / 64);
+  return make_tmap_bf16(map, ptr, rows, 64, box_rows);
+}
+
 // 3-D bf16 tensor map over a row-major [d2][d1][d0] array with a box of
 // b0 x b1 x b2 elements (b0 * 2 bytes = 128) and 128-byte swizzling.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
@@ -258,10 +275,11 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t 
 }
 
 template <int BN>
-static cudaError_t launch_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
-                             cudaStream_t st) {
+static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
+                             int num_sms, cudaStream_t st) {
   CUtensorMap ma, mb;
-  if (!make_tmap_bf16(&ma, A, M, K, BM) || !make_tmap_bf16(&mb, B, N, K, BN)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&ma, A, M, K, BM) || !make_tmap_weights(&mb, B, b_tiled, N, K, b_tiled ? 128 : BN))
+    return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<bf16, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -271,12 +289,13 @@ static cudaError_t launch_tc(const void* A, const void* B, int M, int N, int K, 
   }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(gemm_tc_kernel<bf16, BN>, dim3(grid), dim3(192), TcCfg<BN>::SMEM, st, ma, mb, M, N, K, ep);
+  return launch_pdl(gemm_tc_kernel<bf16, BN>, dim3(grid), dim3(192), TcCfg<BN>::SMEM, st, ma, mb, M, N, K, b_tiled,
+                    ep);
 }
 
 // BN = 256 unless that leaves the last wave badly filled.
-cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
-                           cudaStream_t st) {
+cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
+                           int num_sms, cudaStream_t st) {
   const int num_m = (M + BM - 1) / BM;
   const int t256 = num_m * ((N + 255) / 256);
   const int t128 = num_m * ((N + 127) / 128);
@@ -285,7 +304,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, co
     return (double)waves * cost;  // time ~ waves x per-tile cost
   };
   const bool use256 = (N % 256 == 0) && eff(t256, 2.0) <= eff(t128, 1.0) * 1.05;
-  return use256 ? launch_tc<256>(A, B, M, N, K, ep, num_sms, st) : launch_tc<128>(A, B, M, N, K, ep, num_sms, st);
+  return use256 ? launch_tc<256>(A, B, b_tiled, M, N, K, ep, num_sms, st)
+                : launch_tc<128>(A, B, b_tiled, M, N, K, ep, num_sms, st);
 }
 
 }  // namespace llama

@@ -62,7 +62,8 @@ __host__ __device__ __forceinline__ int sk_owner(int x, int total, int grid) {
 template <int MB>
 __global__ void __launch_bounds__(160, 1)
     gemv_bf16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
-                     int N, int nk, int total, float* __restrict__ part, int* __restrict__ counters, EpiParams ep) {
+                     int N, int nk, int total, int tiled, float* __restrict__ part, int* __restrict__ counters,
+                     EpiParams ep) {
   constexpr int STAGES = stages(MB);
   constexpr uint32_t SB = stage_bytes(MB);
   extern __shared__ uint8_t smem_raw[];
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(160, 1)
       for (int i = 0; i < pre; ++i) {
         const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
         mbar_arrive_expect_tx(&full[i], SB);
-        tma_load_2d(base + i * SB, &map_w, &full[i], ks * KB, rb * RPC);
+        tma_load_2d(base + i * SB, &map_w, &full[i], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
       }
       pdl_wait();
       pdl_trigger();
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(160, 1)
         const int rb = x / nk, ks = x - rb * nk;
         uint8_t* dst = base + st * SB;
         mbar_arrive_expect_tx(&full[st], SB);
-        tma_load_2d(dst, &map_w, &full[st], ks * KB, rb * RPC);
+        tma_load_2d(dst, &map_w, &full[st], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
         tma_load_2d(dst + W_BYTES, &map_x, &full[st], ks * KB, 0);
       }
       // the CTA must not retire while a copy into its shared memory is in flight
@@ -274,7 +275,7 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
 
 template <int MB>
 static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
-                             float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
+                             int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
   constexpr size_t smem = gemv_smem(MB);
   static bool attr = false;
   if (!attr) {
@@ -283,21 +284,22 @@ static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, part,
+  return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
                     counters, ep);
 }
 
-cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
-                             int* counters, const EpiParams& ep, int num_sms, cudaStream_t st) {
+cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
+                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st) {
   (void)num_sms;
   const int MB = (M + 7) / 8;
   CUtensorMap mw, mx;
-  if (!make_tmap_bf16(&mw, W, N, K, RPC) || !make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
+  if (!make_tmap_weights(&mw, W, tiled, N, K, RPC) || !make_tmap_bf16(&mx, X, M, K, 8 * MB))
+    return cudaErrorInvalidValue;
   switch (MB) {
-    case 1: return launch_mb<1>(mw, mx, M, N, p, part, counters, ep, st);
-    case 2: return launch_mb<2>(mw, mx, M, N, p, part, counters, ep, st);
-    case 3: return launch_mb<3>(mw, mx, M, N, p, part, counters, ep, st);
-    default: return launch_mb<4>(mw, mx, M, N, p, part, counters, ep, st);
+    case 1: return launch_mb<1>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    case 2: return launch_mb<2>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    case 3: return launch_mb<3>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    default: return launch_mb<4>(mw, mx, M, N, p, tiled, part, counters, ep, st);
   }
 }
 

@@ -38,6 +38,9 @@ void launch_kv_convert(const void* src, void* dst, int Bm, int S, int Hkv, int D
                        cudaStream_t st);
 template <typename T>
 void launch_rope_rows_to_interleaved(const void* src, void* dst, int heads, int D, int dim, cudaStream_t st);
+// [N][K] row-major bf16 -> [ceil(N/128)][K/64][128][64] tiles (rows past N zero); K % 64 == 0
+void launch_tile_weights(const void* src, void* dst, int N, int K, cudaStream_t st);
+__host__ __device__ constexpr size_t tiled_weight_elems(size_t N, size_t K) { return (N + 127) / 128 * 128 * K; }
 
 // gemm_simt.cu
 template <typename T>
@@ -49,15 +52,17 @@ struct GemvPlan {
   size_t part_floats = 0;
 };
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
-cudaError_t launch_gemv_bf16(const void* X, const void* W, int M, int N, int K, const GemvPlan& p, float* part,
-                             int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
+// W: [N][K] row-major (tiled = 0) or the library's weight tiles (tiled = 1, tile_weights)
+cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
+                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                        uint32_t b1, uint32_t b2);
-cudaError_t launch_gemm_tc(const void* A, const void* B, int M, int N, int K, const EpiParams& ep, int num_sms,
-                           cudaStream_t st);
+bool make_tmap_weights(CUtensorMap* map, const void* ptr, int tiled, uint64_t N, uint64_t K, uint32_t box_rows);
+cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
+                           int num_sms, cudaStream_t st);
 
 // attention.cu
 struct DecodePlan {

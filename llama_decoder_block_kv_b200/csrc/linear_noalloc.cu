@@ -84,6 +84,6 @@ extern "C" int llama_linear_noalloc(const void* x, const void* w, float* y, int 
   e.out = y;
   e.ld_out = N;
   e.err = err;
-  if (launch_gemv_bf16(x, w, M, N, K, p, part, counters, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+  if (launch_gemv_bf16(x, w, 0, M, N, K, p, part, counters, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
   return LLAMA_OK;
 }

@@ -13,6 +13,7 @@
 //   h += g * W2^T                                                        (residual epilogue)
 // Whole-model calls add the embedding gather before and the final RMSNorm
 // plus the LM head after ("... notes", Transformer.forward).
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -165,6 +166,8 @@ EpiParams epi_base(llama_ctx* c, int kind, int M, int N) {
 }
 
 // C[M][N] = A[M][K] * W[N][K]^T through the path that suits the shape.
+// W is one of the library's weight matrices: row-major fp32 in fp32 mode,
+// 128 x 64 bf16 tiles (tile_weights) in bf16 mode.
 int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st) {
   if (!c->bf16) {
     launch_gemm_simt<float>(A, W, M, N, K, ep, st);
@@ -173,11 +176,15 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
   if (M <= 32 && K % 64 == 0) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_bf16(A, W, M, N, K, p, c->part, c->counters, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK
-                                                                                          : LLAMA_ERR_CUDA;
+    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st) == cudaSuccess
+               ? LLAMA_OK
+               : LLAMA_ERR_CUDA;
   }
-  return launch_gemm_tc(A, W, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
+
+// elements of one stored weight matrix [N][K]: tiles in bf16 mode, row-major in fp32 mode
+size_t weight_elems(const llama_ctx* c, size_t N, size_t K) { return c->bf16 ? tiled_weight_elems(N, K) : N * K; }
 
 // One decode step of a block in one persistent launch (decode_block.cu), when
 // the call and the shapes allow it. Returns 1 when the call must take the
@@ -386,8 +393,8 @@ int llama_create(const llama_args* args, llama_ctx** out) {
   };
   int r;
   const size_t es = c->esz;
-  const size_t wsz = ((size_t)c->n_qkv * c->dim + (size_t)c->dim * c->H * D + 2 * (size_t)F * c->dim +
-                      (size_t)c->dim * F) * es;
+  const size_t wsz = (weight_elems(c, c->n_qkv, c->dim) + weight_elems(c, c->dim, (size_t)c->H * D) +
+                      weight_elems(c, 2 * (size_t)F, c->dim) + weight_elems(c, c->dim, F)) * es;
   const size_t cache_elems = (size_t)c->Bm * c->Hkv * c->S * D;
   for (int l = 0; l < c->L; ++l) {
     Layer& Ly = c->layers[l];
@@ -395,13 +402,13 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     if ((r = alloc(&blob, wsz + 2 * round256((size_t)c->dim * es)))) return fail(r);
     uint8_t* p = reinterpret_cast<uint8_t*>(blob);
     Ly.wqkv = p;
-    p += (size_t)c->n_qkv * c->dim * es;
+    p += weight_elems(c, c->n_qkv, c->dim) * es;
     Ly.wo = p;
-    p += (size_t)c->dim * c->H * D * es;
+    p += weight_elems(c, c->dim, (size_t)c->H * D) * es;
     Ly.w13 = p;
-    p += 2 * (size_t)F * c->dim * es;
+    p += weight_elems(c, 2 * (size_t)F, c->dim) * es;
     Ly.w2 = p;
-    p += (size_t)c->dim * F * es;
+    p += weight_elems(c, c->dim, F) * es;
     Ly.attn_norm = p;
     p += round256((size_t)c->dim * es);
     Ly.ffn_norm = p;
@@ -413,17 +420,17 @@ int llama_create(const llama_args* args, llama_ctx** out) {
       const uint64_t rows = (uint64_t)c->Bm * c->Hkv * c->S;
       if (!make_tmap_bf16(&Ly.map_k, Ly.cache_k, rows, D, 64) || !make_tmap_bf16(&Ly.map_v, Ly.cache_v, rows, D, 64))
         return fail(LLAMA_ERR_CUDA);
-      if (!make_tmap_bf16(&Ly.map_w[0], Ly.wqkv, c->n_qkv, c->dim, 128) ||
-          !make_tmap_bf16(&Ly.map_w[1], Ly.wo, c->dim, c->H * D, 128) ||
-          !make_tmap_bf16(&Ly.map_w[2], Ly.w13, 2 * F, c->dim, 128) ||
-          !make_tmap_bf16(&Ly.map_w[3], Ly.w2, c->dim, F, 128))
+      if (!make_tmap_weights(&Ly.map_w[0], Ly.wqkv, 1, c->n_qkv, c->dim, 128) ||
+          !make_tmap_weights(&Ly.map_w[1], Ly.wo, 1, c->dim, c->H * D, 128) ||
+          !make_tmap_weights(&Ly.map_w[2], Ly.w13, 1, 2 * F, c->dim, 128) ||
+          !make_tmap_weights(&Ly.map_w[3], Ly.w2, 1, c->dim, F, 128))
         return fail(LLAMA_ERR_CUDA);
     }
   }
   if (c->V > 0) {
     if ((r = alloc(&c->tok_emb, (size_t)c->V * c->dim * es))) return fail(r);
     if ((r = alloc(&c->final_norm, round256((size_t)c->dim * es)))) return fail(r);
-    if ((r = alloc(&c->output, (size_t)c->V * c->dim * es))) return fail(r);
+    if ((r = alloc(&c->output, weight_elems(c, c->V, c->dim) * es))) return fail(r);
   }
   std::vector<float2> rt = rope_table(D, 2 * c->S, (double)a.rope_theta);
   if ((r = alloc(reinterpret_cast<void**>(&c->rope), rt.size() * sizeof(float2)))) return fail(r);
@@ -504,11 +511,32 @@ int llama_set_layer(llama_ctx* c, int layer, const void* wq, const void* wk, con
                     const void* w1, const void* w2, const void* w3, const void* attn_norm, const void* ffn_norm) {
   if (!c || layer < 0 || layer >= c->L) return LLAMA_ERR_INVALID_ARGS;
   if (!wq || !wk || !wv || !wo || !w1 || !w2 || !w3 || !attn_norm || !ffn_norm) return LLAMA_ERR_INVALID_ARGS;
+  for (const void* q : {wq, wk, wv, wo, w1, w2, w3})
+    if (reinterpret_cast<uintptr_t>(q) % 16) return LLAMA_ERR_INVALID_ARGS;
   CK(cudaSetDevice(c->device));
   Layer& Ly = c->layers[layer];
   const size_t es = c->esz;
   const size_t qb = (size_t)c->H * c->D * c->dim * es, kb = (size_t)c->Hkv * c->D * c->dim * es;
-  uint8_t* p = reinterpret_cast<uint8_t*>(Ly.wqkv);
+  // Row-major packing happens in place in fp32 mode; in bf16 mode it goes to a
+  // temporary buffer from which the tiles are cut (tile_weights).
+  void* tmp = nullptr;
+  if (c->bf16) {
+    const size_t n = std::max((size_t)c->n_qkv, 2 * (size_t)c->F) * c->dim * es;
+    int r;
+    if ((r = alloc(&tmp, n))) return r;
+  }
+  auto done = [&](int code) {
+    if (tmp) {
+      cudaDeviceSynchronize();
+      cudaFree(tmp);
+    }
+    return code;
+  };
+#define CKT(call)                                             \
+  do {                                                        \
+    if ((call) != cudaSuccess) return done(LLAMA_ERR_CUDA);   \
+  } while (0)
+  uint8_t* p = reinterpret_cast<uint8_t*>(c->bf16 ? tmp : Ly.wqkv);
   if (c->half_split) {  // rotate interleaved pairs on rows permuted from the half-split order
     if (c->bf16) {
       launch_rope_rows_to_interleaved<bf16>(wq, p, c->H, c->D, c->dim, 0);
@@ -517,32 +545,44 @@ int llama_set_layer(llama_ctx* c, int layer, const void* wq, const void* wk, con
       launch_rope_rows_to_interleaved<float>(wq, p, c->H, c->D, c->dim, 0);
       launch_rope_rows_to_interleaved<float>(wk, p + qb, c->Hkv, c->D, c->dim, 0);
     }
-    CK(cudaGetLastError());
+    CKT(cudaGetLastError());
   } else {
-    CK(cudaMemcpy(p, wq, qb, cudaMemcpyDeviceToDevice));
-    CK(cudaMemcpy(p + qb, wk, kb, cudaMemcpyDeviceToDevice));
+    CKT(cudaMemcpy(p, wq, qb, cudaMemcpyDeviceToDevice));
+    CKT(cudaMemcpy(p + qb, wk, kb, cudaMemcpyDeviceToDevice));
   }
-  CK(cudaMemcpy(p + qb + kb, wv, kb, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(Ly.wo, wo, (size_t)c->dim * c->H * c->D * es, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(Ly.w2, w2, (size_t)c->dim * c->F * es, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(Ly.attn_norm, attn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(Ly.ffn_norm, ffn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
-  if (c->bf16)
-    launch_pack_w13<bf16>(w1, w3, Ly.w13, c->F, c->dim, 0);
-  else
+  CKT(cudaMemcpy(p + qb + kb, wv, kb, cudaMemcpyDeviceToDevice));
+  CKT(cudaMemcpy(Ly.attn_norm, attn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
+  CKT(cudaMemcpy(Ly.ffn_norm, ffn_norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
+  if (c->bf16) {
+    launch_tile_weights(tmp, Ly.wqkv, c->n_qkv, c->dim, 0);
+    launch_tile_weights(wo, Ly.wo, c->dim, c->H * c->D, 0);
+    launch_tile_weights(w2, Ly.w2, c->dim, c->F, 0);
+    launch_pack_w13<bf16>(w1, w3, tmp, c->F, c->dim, 0);  // after the wqkv tiles have been cut (same stream)
+    launch_tile_weights(tmp, Ly.w13, 2 * c->F, c->dim, 0);
+  } else {
+    CKT(cudaMemcpy(Ly.wo, wo, (size_t)c->dim * c->H * c->D * es, cudaMemcpyDeviceToDevice));
+    CKT(cudaMemcpy(Ly.w2, w2, (size_t)c->dim * c->F * es, cudaMemcpyDeviceToDevice));
     launch_pack_w13<float>(w1, w3, Ly.w13, c->F, c->dim, 0);
-  CK(cudaDeviceSynchronize());
+  }
+  CKT(cudaGetLastError());
+  CKT(cudaDeviceSynchronize());
+#undef CKT
   Ly.set = true;
-  return LLAMA_OK;
+  return done(LLAMA_OK);
 }
 
 int llama_set_embed_norm_head(llama_ctx* c, const void* tok, const void* norm, const void* output) {
   if (!c || c->V <= 0 || !tok || !norm || !output) return LLAMA_ERR_INVALID_ARGS;
+  if (reinterpret_cast<uintptr_t>(output) % 16) return LLAMA_ERR_INVALID_ARGS;
   CK(cudaSetDevice(c->device));
   const size_t es = c->esz;
   CK(cudaMemcpy(c->tok_emb, tok, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
   CK(cudaMemcpy(c->final_norm, norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
-  CK(cudaMemcpy(c->output, output, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
+  if (c->bf16)
+    launch_tile_weights(output, c->output, c->V, c->dim, 0);
+  else
+    CK(cudaMemcpy(c->output, output, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
+  CK(cudaGetLastError());
   CK(cudaDeviceSynchronize());
   c->head_set = true;
   return LLAMA_OK;
@@ -712,9 +752,19 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
              : LLAMA_ERR_CUDA;
 }
 
+int llama_tile_weights(const void* w, void* out, int N, int K, void* stream) {
+  if (!w || !out || N <= 0 || K <= 0 || K % 64) return LLAMA_ERR_INVALID_ARGS;
+  if (reinterpret_cast<uintptr_t>(w) % 16 || reinterpret_cast<uintptr_t>(out) % 16) return LLAMA_ERR_INVALID_ARGS;
+  launch_tile_weights(w, out, N, K, S_(stream));
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
 int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, int dtype, int path, void* stream) {
   if (!x || !w || !y || M <= 0 || N <= 0 || K <= 0 || N % 8 || K % 8) return LLAMA_ERR_INVALID_ARGS;
   if (dtype != LLAMA_FP32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
+  const int tiled = (path & LLAMA_WEIGHTS_TILED) ? 1 : 0;
+  path &= ~LLAMA_WEIGHTS_TILED;
+  if (tiled && (dtype != LLAMA_BF16 || K % 64 || path == LLAMA_PATH_SIMT)) return LLAMA_ERR_INVALID_ARGS;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -758,13 +808,13 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
         cudaMemset(g_lin_counters, 0, (size_t)p.row_blocks * sizeof(int));
         g_lin_counters_n = p.row_blocks;
       }
-      if (launch_gemv_bf16(x, w, M, N, K, p, g_lin_part, g_lin_counters, e, sms, st) != cudaSuccess)
+      if (launch_gemv_bf16(x, w, tiled, M, N, K, p, g_lin_part, g_lin_counters, e, sms, st) != cudaSuccess)
         return LLAMA_ERR_CUDA;
       break;
     }
     case LLAMA_PATH_TCGEN05:
       if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
-      if (launch_gemm_tc(x, w, M, N, K, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+      if (launch_gemm_tc(x, w, tiled, M, N, K, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
       break;
     default:
       return LLAMA_ERR_INVALID_ARGS;

@@ -25,6 +25,8 @@ def main():
     ap.add_argument("sizes", type=int, nargs="+")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--graph", action="store_true", help="time the launches inside one CUDA graph")
+    ap.add_argument("--row-major", action="store_true",
+                    help="gemv / tc: pass the weights row-major instead of in the library's tile layout")
     a = ap.parse_args()
     torch.cuda.set_device(0)
     st = torch.cuda.current_stream()
@@ -37,15 +39,18 @@ def main():
         ws = [synth.normal((N, K), 0.02, 2 + i, torch.bfloat16, "cuda") for i in range(n_w)]
         y = torch.empty((M, N), device="cuda")
         path = {"gemv": B.LLAMA_PATH_GEMV, "tc": B.LLAMA_PATH_TCGEN05, "simt": B.LLAMA_PATH_SIMT}[a.kind]
+        if a.kind != "simt" and not a.row_major:
+            ws = [B.llama_tile_weights(w) for w in ws]
+            path |= B.LLAMA_WEIGHTS_TILED
         for w in ws:
-            B.llama_linear(x, w, y, path)
+            B.llama_linear(x, w, y, path, n=N)
         torch.cuda.synchronize()
         if a.graph:
             # a graph of `reps` back-to-back launches: no host overhead between them
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 for i in range(a.reps):
-                    B.llama_linear(x, ws[i % n_w], y, path)
+                    B.llama_linear(x, ws[i % n_w], y, path, n=N)
             g.replay()
             torch.cuda.synchronize()
             e0.record(st)
@@ -54,7 +59,7 @@ def main():
         else:
             e0.record(st)
             for i in range(a.reps):
-                B.llama_linear(x, ws[i % n_w], y, path)
+                B.llama_linear(x, ws[i % n_w], y, path, n=N)
             e1.record(st)
         e1.synchronize()
         ms = e0.elapsed_time(e1) / a.reps

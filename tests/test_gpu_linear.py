@@ -53,3 +53,29 @@ def test_simt_gemm(M, N, K, dt):
     B.llama_linear(x, w, y, B.LLAMA_PATH_SIMT)
     torch.cuda.synchronize()
     _check(x, w, y, rel=1e-5)
+
+
+@pytest.mark.parametrize("path,M,N,K", [(B.LLAMA_PATH_GEMV, 1, 12288, 4096), (B.LLAMA_PATH_GEMV, 9, 136, 192),
+                                        (B.LLAMA_PATH_GEMV, 32, 4096, 11008), (B.LLAMA_PATH_TCGEN05, 300, 1024, 1024),
+                                        (B.LLAMA_PATH_TCGEN05, 512, 12288, 4096), (B.LLAMA_PATH_TCGEN05, 77, 384, 448)])
+def test_tiled_weights_give_identical_results(path, M, N, K):
+    """The tile layout only changes where a 128 x 64 stage is read from: the
+    shared-memory image, hence every MMA and every sum, is the same as with
+    row-major weights, so the outputs are bit-identical."""
+    x, w = _inputs(M, N, K, torch.bfloat16, 41)
+    wt = B.llama_tile_weights(w)
+    assert wt.numel() == (N + 127) // 128 * 128 * K
+    # the layout itself: tile (n // 128, k // 64), row n % 128, column k % 64; rows past N zero
+    nk = K // 64
+    tiles = wt.view(-1, 128, 64)
+    for n, k in [(0, 0), (N - 1, K - 1), (min(130, N - 1), 70 % K), (N // 2, K // 2)]:
+        assert tiles[(n // 128) * nk + k // 64, n % 128, k % 64] == w[n, k]
+    if N % 128:
+        assert torch.all(tiles[(N // 128) * nk:, N % 128:, :] == 0)
+    y0 = torch.full((M, N), float("nan"), device="cuda")
+    y1 = torch.full((M, N), float("nan"), device="cuda")
+    B.llama_linear(x, w, y0, path)
+    B.llama_linear(x, wt, y1, path | B.LLAMA_WEIGHTS_TILED, n=N)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    _check(x, w, y1)
