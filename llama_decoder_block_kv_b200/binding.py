@@ -211,7 +211,7 @@ def llama_reset(ctx) -> None:
 
 
 def llama_set_decode_kernel(ctx, mode: int) -> None:
-    _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel", "llama_tile_weights")
+    _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel")
 
 
 def llama_get_error(ctx):

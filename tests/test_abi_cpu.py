@@ -90,3 +90,14 @@ def test_null_and_bad_calls_are_rejected_without_a_device():
         == B.LLAMA_ERR_INVALID_ARGS
     assert B.strerror(B.LLAMA_ERR_POS_RANGE).startswith("position")
     L.llama_destroy(None)
+
+
+def test_wrappers_reach_the_library_without_a_device():
+    """Wrappers whose C call rejects a NULL context before touching the device:
+    the argument error comes back as LlamaError (checks the marshalling)."""
+    with pytest.raises(B.LlamaError) as e:
+        B.llama_set_decode_kernel(None, B.LLAMA_DECODE_LAYERED)
+    assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
+    with pytest.raises(B.LlamaError) as e:
+        B.llama_reset(None)
+    assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
