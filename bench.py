@@ -306,7 +306,7 @@ def time_graph(g, steps, warmup, world):
 # capture of one w1|w3 launch, M=1, N=22016, K=4096 (dram read + write of one
 # launch / weights + activations + outputs). Valid for the kernel version that
 # capture names; set to None when the kernel changes until it is re-measured.
-GEMV_TRAFFIC_RATIO = (181.60e6 + 3.34e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
+GEMV_TRAFFIC_RATIO = (180.45e6 + 3.53e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
 
 
 def gemv_roofline(lb: LayerBench, peaks, reps=10):
