@@ -605,7 +605,7 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
   int want = (2 * num_sms + units - 1) / units;
   int ck = (max_len + want - 1) / want;
   ck = (ck + KT - 1) / KT * KT;
-  if (ck < 512) ck = 512;  // below ~512 keys the merge costs more than the parallelism gains
+  if (ck < 128) ck = 128;  // at least two tiles per CTA (measured: 128 beats 256 and 512 on short histories)
   if (ck > 1024) ck = 1024;
   p.CK = ck;
   p.max_chunks = (S_max + ck - 1) / ck;

@@ -186,8 +186,8 @@ void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int
 template <typename T>
 void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
                     int in_row_offset, cudaStream_t st) {
-  if (dim >= 4096)
-    launch_pdl(rmsnorm_kernel<T, 256>, dim3(rows), dim3(256), 0, st, h, reinterpret_cast<const T*>(w),
+  if (dim >= 4096)  // one float4 per thread and pass at dim 4096 (a row is read in one round trip)
+    launch_pdl(rmsnorm_kernel<T, 1024>, dim3(rows), dim3(1024), 0, st, h, reinterpret_cast<const T*>(w),
                reinterpret_cast<T*>(out), dim, eps, in_row_stride_T, in_row_offset);
   else
     launch_pdl(rmsnorm_kernel<T, 64>, dim3(rows), dim3(64), 0, st, h, reinterpret_cast<const T*>(w),
