@@ -7,23 +7,19 @@
 // j = 0 .. p of kv head h / n_rep (repeat_kv maps kv head j to query heads
 // j*n_rep .. j*n_rep + n_rep - 1) with scores q.k / sqrt(D) and a softmax.
 // The additive mask of the pages is never built: the predicate j <= p is
-// applied inside the kernels, and key tiles that are fully masked for a warp
-// are skipped (the pages' xformers remark: masked scores are not computed).
+// applied inside the kernels and key tiles past the last position are never
+// read (the pages' xformers remark: masked scores are not computed).
 //
-// Kernels:
-//  - attn_prefill_kernel (T > 1): flash-style online softmax. A CTA owns one
-//    (sequence, kv head) and 128 query rows made of up to 8 query heads of
-//    that kv group times 128/heads positions, so each K/V tile is loaded once
-//    for the whole group. K/V tiles (64 keys) arrive by TMA (128-byte swizzle,
-//    no multicast) into a 3-stage ring fed by a producer warp; 8 compute warps
-//    run S = QK^T and O += PV on the warp-level bf16 tensor-core MMA.
+// Kernels (the prefill attention, T > 1, is the tcgen05 kernel of attn_tc.cu):
 //  - attn_decode_kernel (T == 1): split-K flash decode. A CTA owns one
-//    (sequence, kv head, chunk of keys); the chunk streams through the same
-//    TMA ring, the 4 compute warps each take 16 keys of every 64-key tile,
-//    their (max, sum, O) states merge in shared memory and the CTA writes one
-//    partial; the CTA that finishes last for a (sequence, head group) merges
-//    the partials of all chunks with the log-sum-exp rule m = max m_c,
-//    l = sum l_c e^(m_c - m), o = sum o_c e^(m_c - m) / l.
+//    (sequence, kv head group, chunk of keys); the chunk streams through a
+//    3-stage TMA ring (64-key K and V tiles, 128-byte swizzle, no multicast)
+//    fed by a producer warp, the 4 compute warps each take 16 keys of every
+//    64-key tile on the warp-level bf16 tensor-core MMA, their (max, sum, O)
+//    states merge in shared memory and the CTA writes one partial; the CTA
+//    that finishes last for a (sequence, head group) merges the partials of
+//    all chunks with the log-sum-exp rule m = max m_c, l = sum l_c e^(m_c - m),
+//    o = sum o_c e^(m_c - m) / l.
 //  - attn_simple_kernel: fp32 mode (tiny models), one CTA per (token, head),
 //    scores in shared memory, plain two-pass softmax.
 #include "kernels.cuh"
@@ -65,193 +61,6 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* mk, const CUtens
   for (int h = 0; h < AttnSmem<D>::HALVES; ++h) {
     tma_load_2d(sk + h * 8192, mk, bar, h * 64, row);
     tma_load_2d(sv + h * 8192, mv, bar, h * 64, row);
-  }
-}
-
-// ============================================================================ prefill
-
-template <int D>
-__global__ void __launch_bounds__(288, 1)
-    attn_prefill_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                        const bf16* __restrict__ q, bf16* __restrict__ o, const int* __restrict__ start_pos,
-                        int sp_scalar, int T, int H, int Hkv, int S_max, int hpc, int* err) {
-  constexpr int STAGES = 3;
-  constexpr uint32_t TB = AttnSmem<D>::TILE_BYTES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * 2 * TB);
-  uint64_t* empty = full + STAGES;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, qd = lane & 3;
-  const int n_rep = H / Hkv, groups = n_rep / hpc;
-  const int BQ = 128 / hpc;
-  const int qblk = gridDim.x - 1 - blockIdx.x;  // longest (latest) query blocks first
-  const int z = blockIdx.y;
-  const int b = z / (Hkv * groups);
-  const int kvh = (z / groups) % Hkv;
-  const int grp = z % groups;
-  const int q0 = qblk * BQ;
-  const int sp = start_pos ? start_pos[b] : sp_scalar;
-  const int q_last = min(q0 + BQ, T) - 1;
-  const int kv_len = min(sp + q_last + 1, S_max);
-  const int n_tiles = (kv_len + KT - 1) / KT;
-  const int row0 = (b * Hkv + kvh) * S_max;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 8);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == 8) {
-    if (lane == 0) {
-      prefetch_tensormap(&map_k);
-      prefetch_tensormap(&map_v);
-      int j = 0;
-      for (; j < n_tiles; ++j) {
-        const int st = j % STAGES;
-        if (!mbar_wait(&empty[st], ((j / STAGES) & 1) ^ 1, err)) break;
-        load_kv_tile<D>(&map_k, &map_v, base + st * 2 * TB, base + st * 2 * TB + TB, &full[st], row0 + j * KT);
-      }
-      // the CTA must not retire while a copy into its shared memory is in flight
-      for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, err);
-    }
-    return;
-  }
-
-  // ---------------------------------------------------------------- compute warps
-  const int hl = (warp * 16) / BQ;           // query head inside this CTA
-  const int pl0 = (warp * 16) % BQ;          // first position (inside the block) of this warp
-  const int h = kvh * n_rep + grp * hpc + hl;
-  const int t0 = q0 + pl0 + g, t1 = t0 + 8;  // call-relative positions of this thread's two rows
-  const int c0 = min(t0, T - 1), c1 = min(t1, T - 1);
-  const int p0 = sp + c0, p1 = sp + c1;
-  const int warp_pmax = sp + min(q0 + pl0 + 15, T - 1);
-
-  uint32_t qa[D / 16][4];
-  {
-    const bf16* r0 = q + ((size_t)(b * T + c0) * H + h) * D;
-    const bf16* r1 = q + ((size_t)(b * T + c1) * H + h) * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      qa[kk][0] = *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd);
-      qa[kk][1] = *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd);
-      qa[kk][2] = *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd);
-      qa[kk][3] = *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd);
-    }
-  }
-  float oacc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const float sl2 = rsqrtf((float)D) * LOG2E;
-
-  for (int j = 0; j < n_tiles; ++j) {
-    const int st = j % STAGES;
-    const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    if (j * KT <= warp_pmax) {
-      const uint32_t kb = smem_u32(base + st * 2 * TB);
-      const uint32_t vb = kb + TB;
-      float s[8][4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-        for (int jn = 0; jn < 8; jn += 2) {
-          const int mi = lane >> 3;
-          const int key = 8 * (jn + (mi >> 1)) + (lane & 7);
-          const int d = 16 * kk + 8 * (mi & 1);
-          uint32_t bf[4];
-          ldmatrix_x4(bf, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
-          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-          mma_bf16_16816(s[jn], qa[kk], b0);
-          mma_bf16_16816(s[jn + 1], qa[kk], b1);
-        }
-      }
-      const bool need_mask = (j * KT + KT - 1) > (sp + min(q0 + pl0, T - 1));
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int jn = 0; jn < 8; ++jn) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = s[jn][e] * sl2;
-          if (need_mask) {
-            const int key = j * KT + 8 * jn + 2 * qd + (e & 1);
-            if (key > (e < 2 ? p0 : p1)) v = -INFINITY;
-          }
-          s[jn][e] = v;
-        }
-        mx0 = fmaxf(mx0, fmaxf(s[jn][0], s[jn][1]));
-        mx1 = fmaxf(mx1, fmaxf(s[jn][2], s[jn][3]));
-      }
-      mx0 = quad_max(mx0);
-      mx1 = quad_max(mx1);
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      l0 *= sc0;
-      l1 *= sc1;
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        oacc[i][0] *= sc0;
-        oacc[i][1] *= sc0;
-        oacc[i][2] *= sc1;
-        oacc[i][3] *= sc1;
-      }
-#pragma unroll
-      for (int jn = 0; jn < 8; ++jn) {
-        s[jn][0] = exp2f(s[jn][0] - mn0);
-        s[jn][1] = exp2f(s[jn][1] - mn0);
-        s[jn][2] = exp2f(s[jn][2] - mn1);
-        s[jn][3] = exp2f(s[jn][3] - mn1);
-        l0 += s[jn][0] + s[jn][1];
-        l1 += s[jn][2] + s[jn][3];
-      }
-#pragma unroll
-      for (int kb2 = 0; kb2 < 4; ++kb2) {
-        const uint32_t pa[4] = {pack_bf16x2(s[2 * kb2][0], s[2 * kb2][1]), pack_bf16x2(s[2 * kb2][2], s[2 * kb2][3]),
-                                pack_bf16x2(s[2 * kb2 + 1][0], s[2 * kb2 + 1][1]),
-                                pack_bf16x2(s[2 * kb2 + 1][2], s[2 * kb2 + 1][3])};
-#pragma unroll
-        for (int jd = 0; jd < D / 8; jd += 2) {
-          const int mi = lane >> 3;
-          const int key = 16 * kb2 + 8 * (mi & 1) + (lane & 7);
-          const int d = 8 * (jd + (mi >> 1));
-          uint32_t bf[4];
-          ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
-          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-          mma_bf16_16816(oacc[jd], pa, b0);
-          mma_bf16_16816(oacc[jd + 1], pa, b1);
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-  }
-
-  l0 = quad_sum(l0);
-  l1 = quad_sum(l1);
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
-  if (t0 < T) {
-    bf16* dst = o + ((size_t)(b * T + t0) * H + h) * D;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i)
-      *reinterpret_cast<uint32_t*>(dst + 8 * i + 2 * qd) = pack_bf16x2(oacc[i][0] * i0, oacc[i][1] * i0);
-  }
-  if (t1 < T) {
-    bf16* dst = o + ((size_t)(b * T + t1) * H + h) * D;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i)
-      *reinterpret_cast<uint32_t*>(dst + 8 * i + 2 * qd) = pack_bf16x2(oacc[i][2] * i1, oacc[i][3] * i1);
   }
 }
 
@@ -570,31 +379,6 @@ __global__ void attn_simple_kernel(const T* __restrict__ q, const T* __restrict_
 }
 
 // ============================================================================ host launchers
-
-template <int D>
-static cudaError_t prefill_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
-                             int sp_scalar, int B, int T, int H, int Hkv, int S_max, int* err, cudaStream_t st) {
-  const int n_rep = H / Hkv;
-  const int hpc = n_rep < 8 ? n_rep : 8;
-  const int BQ = 128 / hpc;
-  const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid((T + BQ - 1) / BQ, B * Hkv * (n_rep / hpc));
-  return launch_pdl(attn_prefill_kernel<D>, grid, dim3(288), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
-                    reinterpret_cast<bf16*>(o), sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
-}
-
-cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
-                                int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max, int* err,
-                                cudaStream_t st) {
-  if (D == 128) return prefill_d<128>(mk, mv, q, o, sp, sp_scalar, B, T, H, Hkv, S_max, err, st);
-  return prefill_d<64>(mk, mv, q, o, sp, sp_scalar, B, T, H, Hkv, S_max, err, st);
-}
 
 DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sms) {
   DecodePlan p;

@@ -1,7 +1,7 @@
 // Causal grouped-query prefill attention on the 5th-generation tensor cores.
 //
-// What is computed is the same as attn_prefill_kernel (attention.cu): for the
-// query of sequence b at position p = start_pos[b] + s and query head h,
+// What is computed: for the query of sequence b at position
+// p = start_pos[b] + s and query head h,
 // softmax_j(q.k_j / sqrt(D)) over the cached keys j <= p of kv head h / n_rep,
 // times V ("LLaMA: Open and Efficient Foundation Language Models" notes,
 // Attention.forward and repeat_kv; "灵哥讲llama3(中)", the cached-mask comment).

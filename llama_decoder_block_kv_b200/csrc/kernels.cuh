@@ -70,9 +70,6 @@ struct DecodePlan {
   size_t part_floats = 0;
 };
 DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sms);
-cudaError_t launch_attn_prefill(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
-                                int sp_scalar, int B, int T, int H, int Hkv, int D, int S_max, int* err,
-                                cudaStream_t st);
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
