@@ -201,7 +201,9 @@ int llama_block_forward(llama_ctx* ctx, int layer, float* h_dev, int B, int T, c
  * order), whose cumulative renormalised probability exceeds uniforms_dev[b]
  * (caller-supplied uniforms in [0, 1), one per sequence: the draw is
  * reproducible). out_dev int32 [B]. Uses a private, lazily allocated
- * scratch of B*V floats; not thread-safe. Stream-ordered.
+ * scratch of B*V floats on the device of the first top-p call (a top-p call
+ * on another device returns LLAMA_ERR_INVALID_ARGS); not thread-safe.
+ * Stream-ordered.
  */
 int llama_sample(const float* logits_dev, int B, int V, float temperature, float top_p, const float* uniforms_dev,
                  int32_t* out_dev, void* cuda_stream);
@@ -290,8 +292,9 @@ int llama_tile_weights(const void* w_dev, void* out_dev, int N, int K, void* cud
  * holds llama_tile_weights tiles. Rules: M, N, K > 0, N % 8 == 0, K % 8 == 0;
  * LLAMA_PATH_GEMV needs M <= 32 and K % 64 == 0; LLAMA_PATH_TCGEN05 needs
  * dtype == LLAMA_BF16; tiled weights need dtype == LLAMA_BF16, K % 64 == 0
- * and the GEMV or TCGEN05 path. Uses a private, lazily allocated workspace;
- * not thread-safe.
+ * and the GEMV or TCGEN05 path. Uses a private, lazily allocated workspace
+ * on the device of the first call (a call with another current device
+ * returns LLAMA_ERR_INVALID_ARGS); not thread-safe.
  */
 int llama_linear(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, int dtype, int path,
                  void* cuda_stream);

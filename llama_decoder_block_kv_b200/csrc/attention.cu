@@ -402,12 +402,9 @@ static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
                             int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max,
                             const DecodePlan& p, int* err, cudaStream_t st) {
   const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(attn_decode_kernel<D>, smem, attr);
+  if (e != cudaSuccess) return e;
   const int n_rep = H / Hkv;
   float* part_o = part;
   float* part_ml = part + (size_t)B * H * p.max_chunks * D;

@@ -371,13 +371,9 @@ static cudaError_t prefill_tc_d(const CUtensorMap& mk, const CUtensorMap& mv, co
   const int BQ = 128 / hpc;
   CUtensorMap mq;
   if (!make_q_map(&mq, q, B * T, H, D, hpc)) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)AttnTcCfg<D>::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(attn_prefill_tc_kernel<D>, AttnTcCfg<D>::SMEM, attr);
+  if (e != cudaSuccess) return e;
   dim3 grid((T + BQ - 1) / BQ, B * Hkv * (n_rep / hpc));
   return launch_pdl(attn_prefill_tc_kernel<D>, grid, dim3(192), AttnTcCfg<D>::SMEM, st, mq, mk, mv,
                     reinterpret_cast<bf16*>(o), sp, sp_scalar, T, H, Hkv, S_max, hpc, err);

@@ -925,13 +925,9 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
 template <int MB>
 static cudaError_t db_launch(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st) {
   const size_t smem = db_smem(MB);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_block_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(decode_block_kernel<MB>, smem, attr);
+  if (e != cudaSuccess) return e;
   return launch_pdl(decode_block_kernel<MB>, dim3(grid), dim3(160), smem, st, maps[0], maps[1], maps[2], maps[3],
                     maps[4], maps[5], p);
 }

@@ -280,13 +280,9 @@ static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, i
   CUtensorMap ma, mb;
   if (!make_tmap_bf16(&ma, A, M, K, BM) || !make_tmap_weights(&mb, B, b_tiled, N, K, b_tiled ? 128 : BN))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<bf16, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)TcCfg<BN>::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(gemm_tc_kernel<bf16, BN>, TcCfg<BN>::SMEM, attr);
+  if (e != cudaSuccess) return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
   return launch_pdl(gemm_tc_kernel<bf16, BN>, dim3(grid), dim3(192), TcCfg<BN>::SMEM, st, ma, mb, M, N, K, b_tiled,

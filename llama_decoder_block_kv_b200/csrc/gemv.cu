@@ -277,13 +277,9 @@ template <int MB>
 static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
                              int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
   constexpr size_t smem = gemv_smem(MB);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemv_bf16_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(gemv_bf16_kernel<MB>, smem, attr);
+  if (e != cudaSuccess) return e;
   return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
                     counters, ep);
 }

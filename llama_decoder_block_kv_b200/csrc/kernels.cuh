@@ -1,6 +1,7 @@
 // Launchers of the library's kernels (host-side declarations).
 #pragma once
 
+#include <atomic>
 #include <utility>
 
 #include "common.cuh"
@@ -22,6 +23,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Opt a kernel in to `bytes` of dynamic shared memory on the current device,
+// once per device (the attribute is per device; `done` is one bit per device
+// ordinal, kept by the caller in a static).
+template <typename... KArgs>
+cudaError_t ensure_smem(void (*kernel)(KArgs...), size_t bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 // elementwise.cu

@@ -337,6 +337,7 @@ size_t g_lin_part_floats = 0;
 int* g_lin_counters = nullptr;
 int g_lin_counters_n = 0;
 int* g_lin_err = nullptr;
+int g_lin_dev = -1;  // device of the private workspace (the first call's)
 
 }  // namespace
 
@@ -739,7 +740,12 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
   if (!greedy && (!uniforms || !(top_p > 0.f) || !(top_p <= 1.f))) return LLAMA_ERR_INVALID_ARGS;
   static float* scratch = nullptr;
   static size_t scratch_n = 0;
+  static int scratch_dev = -1;  // the scratch lives on the device of the first top-p call
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LLAMA_ERR_CUDA;
+  if (!greedy && scratch_dev >= 0 && dev != scratch_dev) return LLAMA_ERR_INVALID_ARGS;
   if (!greedy && scratch_n < (size_t)B * V) {
+    scratch_dev = dev;
     cudaDeviceSynchronize();
     release(reinterpret_cast<void*&>(scratch));
     scratch_n = 0;
@@ -768,6 +774,8 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (g_lin_dev >= 0 && dev != g_lin_dev) return LLAMA_ERR_INVALID_ARGS;  // the workspace is on another device
+  g_lin_dev = dev;
   if (path == LLAMA_PATH_AUTO)
     path = dtype == LLAMA_FP32 ? LLAMA_PATH_SIMT : (M <= 32 && K % 64 == 0 ? LLAMA_PATH_GEMV : LLAMA_PATH_TCGEN05);
   if (!g_lin_err) {
