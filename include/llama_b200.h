@@ -270,6 +270,21 @@ int llama_set_decode_kernel(llama_ctx* ctx, int mode);
  */
 int llama_get_error(llama_ctx* ctx, int* flags);
 
+/*
+ * Failure-detection self-test of the library's bounded device waits (the
+ * pages have no counterpart). which = 0: one thread waits on an mbarrier phase
+ * that nothing completes (the wait every kernel's pipeline uses); which = 1:
+ * the persistent decode kernel's grid barrier, with one of its two CTAs never
+ * arriving. The wait must give up after about one second, record the timeout
+ * bit and return; nothing faults or traps. Synchronous (synchronises the
+ * device); allocates and frees 512 bytes of device memory. *flags receives the
+ * device flag bits the wait recorded (4 = timeout), *seconds the time the
+ * waiting thread spent before giving up. Returns LLAMA_OK when the test ran
+ * (the result is in *flags), LLAMA_ERR_INVALID_ARGS for another `which`,
+ * LLAMA_ERR_CUDA or LLAMA_ERR_OOM when it could not run.
+ */
+int llama_selftest_bounded_wait(int which, int* flags, double* seconds);
+
 /* A static description of an error code. */
 const char* llama_strerror(int code);
 

@@ -35,7 +35,8 @@ LLAMA_DECODE_AUTO, LLAMA_DECODE_LAYERED, LLAMA_DECODE_PERSISTENT = 0, 1, 2
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
-            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel", "llama_tile_weights")
+            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel", "llama_tile_weights",
+            "llama_selftest_bounded_wait")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
         L.llama_set_decode_kernel.argtypes = [vp, i]
         L.llama_tile_weights.argtypes = [vp, vp, i, i, vp]
+        L.llama_selftest_bounded_wait.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_double)]
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -219,6 +221,14 @@ def llama_get_error(ctx):
     flags = ctypes.c_int(0)
     code = lib().llama_get_error(ctx, ctypes.byref(flags))
     return code, flags.value
+
+
+def llama_selftest_bounded_wait(which: int):
+    """Returns (flags, seconds) of a device wait that nothing completes (0: mbarrier, 1: grid barrier)."""
+    flags, secs = ctypes.c_int(0), ctypes.c_double(0.0)
+    _check(lib().llama_selftest_bounded_wait(int(which), ctypes.byref(flags), ctypes.byref(secs)),
+           "llama_selftest_bounded_wait")
+    return flags.value, secs.value
 
 
 def llama_tile_weights(w: torch.Tensor, stream=None) -> torch.Tensor:

@@ -855,6 +855,25 @@ __global__ void __launch_bounds__(160, 1)
   db_linear_phase<MB>(p, 3, cta, grid, j, ring, area, os, full, empty, abort_flag, &s_last, s_r);
 }
 
+// Self-test of the grid barrier's bound: two CTAs of 128 threads, CTA 1 never
+// arrives, so CTA 0's wait runs out after the limit, records the timeout and
+// returns; elapsed[0] receives the time CTA 0 spent in the barrier.
+__global__ void __launch_bounds__(128) grid_barrier_selftest_kernel(unsigned long long* gbar, int* err,
+                                                                    unsigned long long* elapsed) {
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) s_abort = 0;
+  __syncthreads();
+  if (blockIdx.x == 1) return;
+  const uint64_t t0 = global_timer_ns();
+  db_grid_sync(gbar, 2, err, &s_abort);
+  if (threadIdx.x == 0) elapsed[0] = global_timer_ns() - t0;
+}
+
+cudaError_t launch_grid_barrier_selftest(void* gbar, int* err, unsigned long long* elapsed, cudaStream_t st) {
+  grid_barrier_selftest_kernel<<<2, 128, 0, st>>>(reinterpret_cast<unsigned long long*>(gbar), err, elapsed);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ host side
 
 static size_t db_smem(int mb) {

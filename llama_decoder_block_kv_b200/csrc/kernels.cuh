@@ -147,5 +147,8 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
 // maps: wqkv, wo, w1|w3, w2 (128-row x 64-k boxes), then the layer's K and V caches (64-row x 64 boxes)
 cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st);
 size_t decode_block_smem(int M);
+// failure-detection self-tests (selftest.cu, decode_block.cu): a bounded wait that nothing completes
+cudaError_t launch_grid_barrier_selftest(void* gbar, int* err, unsigned long long* elapsed, cudaStream_t st);
+cudaError_t launch_mbarrier_selftest(int* err, unsigned long long* elapsed, cudaStream_t st);
 
 }  // namespace llama

@@ -758,6 +758,35 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
              : LLAMA_ERR_CUDA;
 }
 
+int llama_selftest_bounded_wait(int which, int* flags, double* seconds) {
+  if (flags) *flags = 0;
+  if (seconds) *seconds = 0.0;
+  if (which != 0 && which != 1) return LLAMA_ERR_INVALID_ARGS;
+  void* buf = nullptr;  // error word, elapsed time, 256-byte grid-barrier block
+  int r;
+  if ((r = alloc(&buf, 512))) return r;
+  uint8_t* b = reinterpret_cast<uint8_t*>(buf);
+  int* err = reinterpret_cast<int*>(b);
+  unsigned long long* elapsed = reinterpret_cast<unsigned long long*>(b + 8);
+  void* gbar = b + 256;
+  int code = LLAMA_OK;
+  if (cudaMemset(buf, 0, 512) != cudaSuccess) code = LLAMA_ERR_CUDA;
+  if (code == LLAMA_OK) {
+    const cudaError_t e = which == 0 ? launch_mbarrier_selftest(err, elapsed, 0)
+                                     : launch_grid_barrier_selftest(gbar, err, elapsed, 0);
+    if (e != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) code = LLAMA_ERR_CUDA;
+  }
+  int f = 0;
+  unsigned long long ns = 0;
+  if (code == LLAMA_OK && (cudaMemcpy(&f, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+                           cudaMemcpy(&ns, elapsed, sizeof(ns), cudaMemcpyDeviceToHost) != cudaSuccess))
+    code = LLAMA_ERR_CUDA;
+  cudaFree(buf);
+  if (flags) *flags = f;
+  if (seconds) *seconds = (double)ns * 1e-9;
+  return code;
+}
+
 int llama_tile_weights(const void* w, void* out, int N, int K, void* stream) {
   if (!w || !out || N <= 0 || K <= 0 || K % 64) return LLAMA_ERR_INVALID_ARGS;
   if (reinterpret_cast<uintptr_t>(w) % 16 || reinterpret_cast<uintptr_t>(out) % 16) return LLAMA_ERR_INVALID_ARGS;
