@@ -9,7 +9,10 @@
 // blocks (128 rows x 64 k each) are dealt out as equal contiguous ranges. A
 // producer warp streams its range's weight tiles together with the matching
 // X tiles (8*MB tokens x 64 bf16) through a deep shared-memory ring with TMA
-// (128-byte swizzle, no multicast), never pausing at row-block edges. Four
+// (128-byte swizzle, no multicast), never pausing at row-block edges. The
+// weights are either row-major or the library's tile layout (each stage one
+// contiguous 16 KB block, see tile_weights_kernel); the shared-memory image
+// of a stage is the same for both. Four
 // consumer warps (32 weight rows each) read the tiles with ldmatrix into the
 // warp-level bf16 tensor-core MMA, weights as the 16-row operand ("swap AB"):
 // one MMA covers 16 weight rows x 8 tokens x 16 k.
