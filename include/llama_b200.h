@@ -219,7 +219,12 @@ int llama_sample(const float* logits_dev, int B, int V, float temperature, float
  * [total_len][B], row cur used at step cur; may be NULL when temperature <= 0)
  * and writes it to tokens[:, cur] except where the prompt mask is set; then
  * prev = cur. Cache positions 0..total_len-2 of sequences 0..B-1 are
- * overwritten. Rules: 1 <= B <= max_batch_size, 1 <= min_prompt_len <=
+ * overwritten. The first step (the prompt prefix) and the first decode step
+ * are launched directly; the remaining decode steps replay a CUDA graph
+ * captured from one step, whose column lives in device memory (plain
+ * launches when there are fewer than three decode steps, or when cuda_stream
+ * is itself being captured). The graph is kept until the next call or
+ * llama_destroy. Rules: 1 <= B <= max_batch_size, 1 <= min_prompt_len <=
  * total_len <= max_seq_len, vocab_size > 0. Stream-ordered; tokens_dev holds
  * the result when the stream reaches the end of the call.
  */

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(160)
   const int b = z / (Hkv * groups);
   const int kvh = (z / groups) % Hkv;
   const int grp = z % groups;
-  // positions are inputs of the call, never written by a kernel of the forward pass
+  // positions are read before pdl_wait: inputs of the call, or written by a kernel that has completed (pdl_wait)
   const int sp = start_pos ? start_pos[b] : sp_scalar;
   const int L = min(sp + 1, S_max);  // keys 0 .. sp
   const int k_begin = chunk * CK;

@@ -176,10 +176,11 @@ __device__ __forceinline__ void epilogue8(const EpiParams& p, int m, int n0, flo
 // the previous kernel has completed and its writes are visible; pdl_trigger
 // (always called after pdl_wait) then lets the next kernel begin launching.
 // Hence when a kernel starts, every kernel before its immediate predecessor
-// has completed. Before pdl_wait a kernel may only read data no kernel of the
-// forward pass writes (weights, tensor maps, positions) or, for the decode
-// attention, cache slots written by calls before the predecessor; it never
-// writes global memory there.
+// has completed. Before pdl_wait a kernel may only read weights, tensor maps,
+// positions (inputs of the call, or written by the embedding kernel of a
+// captured generation step, which is at least three launches before any kernel
+// that reads them early) and, for the decode attention, cache slots written by
+// calls before the predecessor; it never writes global memory there.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

@@ -212,7 +212,7 @@ __device__ __forceinline__ bool db_unit(const DecodeBlockParams& p, int u, DbUni
   w.b = w.z / (p.Hkv * groups);
   w.kvh = (w.z / groups) % p.Hkv;
   w.grp = w.z % groups;
-  // positions are inputs of the call, never written by a kernel of the forward pass
+  // positions: inputs of the call, or written by a kernel that has completed (read after pdl_wait)
   w.sp = p.start_pos ? p.start_pos[w.b] : p.sp_scalar;
   w.L = min(w.sp + 1, p.S_max);
   w.k_begin = w.chunk * p.CK;

@@ -9,13 +9,19 @@ namespace llama {
 // notes, Transformer.forward: h = tok_embeddings(tokens)). One CTA per token;
 // the table row (act type) is widened to the fp32 residual stream. An id
 // outside [0, vocab) raises the token-range flag and yields a zero row.
+// With col (a captured decode step, T_ = 1) the token of sequence b is
+// tokens[b * tok_stride + *col] and CTA b also records its position, *col, in
+// pos[b] for the blocks that follow.
 template <typename T>
 __global__ void embed_gather_kernel(const int* __restrict__ tokens, const T* __restrict__ table,
-                                    float* __restrict__ h, int dim, int vocab, int T_, int tok_stride, int* err) {
+                                    float* __restrict__ h, int dim, int vocab, int T_, int tok_stride, int* err,
+                                    const int* col, int* pos) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;  // token b * T_ + s, read from tokens[b * tok_stride + s]
-  const int id = tokens[(t / T_) * tok_stride + t % T_];
+  const int c0 = col ? *col : 0;
+  if (col && pos && threadIdx.x == 0) pos[t] = c0;
+  const int id = tokens[(t / T_) * tok_stride + t % T_ + c0];
   float* dst = h + (size_t)t * dim;
   if (id < 0 || id >= vocab) {
     if (threadIdx.x == 0) atomicOr(err, LLAMA_DEV_TOKEN_RANGE);
@@ -178,9 +184,22 @@ __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ 
 
 template <typename T>
 void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
-                  int tok_stride, int* err, cudaStream_t st) {
+                  int tok_stride, int* err, cudaStream_t st, const int* col, int* pos) {
   launch_pdl(embed_gather_kernel<T>, dim3(n_tok), dim3(128), 0, st, tokens, reinterpret_cast<const T*>(table), h, dim,
-             vocab, T_, tok_stride, err);
+             vocab, T_, tok_stride, err, col, pos);
+}
+
+// ---------------------------------------------------------------------------
+// Step counter of a captured decode step: *col = value, or *col += 1 after the
+// step's last kernel (one thread; ordered by the launch dependencies).
+__global__ void step_counter_kernel(int* col, int value, int add) {
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) *col = add ? *col + 1 : value;
+}
+
+cudaError_t launch_step_counter(int* col, int value, int add, cudaStream_t st) {
+  return launch_pdl(step_counter_kernel, dim3(1), dim3(32), 0, st, col, value, add);
 }
 
 template <typename T>
@@ -215,7 +234,8 @@ void launch_rope_rows_to_interleaved(const void* src, void* dst, int heads, int 
 }
 
 #define INST(T)                                                                                              \
-  template void launch_embed<T>(const int*, const void*, float*, int, int, int, int, int, int*, cudaStream_t); \
+  template void launch_embed<T>(const int*, const void*, float*, int, int, int, int, int, int*, cudaStream_t, \
+                                const int*, int*);                                                          \
   template void launch_rmsnorm<T>(const float*, const void*, void*, int, int, float, int, int, cudaStream_t); \
   template void launch_pack_w13<T>(const void*, const void*, void*, int, int, cudaStream_t);                 \
   template void launch_kv_convert<T>(const void*, void*, int, int, int, int, int, int, cudaStream_t);   \

@@ -43,7 +43,8 @@ cudaError_t ensure_smem(void (*kernel)(KArgs...), size_t bytes, std::atomic<unsi
 // elementwise.cu
 template <typename T>
 void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
-                  int tok_stride, int* err, cudaStream_t st);
+                  int tok_stride, int* err, cudaStream_t st, const int* col = nullptr, int* pos = nullptr);
+cudaError_t launch_step_counter(int* col, int value, int add, cudaStream_t st);
 template <typename T>
 void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
                     int in_row_offset, cudaStream_t st);
@@ -90,9 +91,10 @@ cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, con
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
 // sample.cu
+// col (optional, device): out, keep and the uniforms row are offset by column *col
 cudaError_t launch_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
                           float* scratch, int32_t* out, int out_stride, const uint8_t* keep, int keep_stride,
-                          cudaStream_t st);
+                          cudaStream_t st, const int* col = nullptr);
 
 // attn_tc.cu
 cudaError_t launch_attn_prefill_tc(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o,

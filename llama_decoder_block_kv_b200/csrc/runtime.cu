@@ -72,9 +72,13 @@ struct llama_ctx {
   unsigned* gbar = nullptr;
   float* ssq = nullptr;
   int decode_mode = LLAMA_DECODE_AUTO;
-  // generation: last-position logits and sampling scratch, [max_batch][vocab] each
+  // generation: last-position logits and sampling scratch, [max_batch][vocab] each;
+  // the captured decode step's column counter and positions; its executable graph
   float* gen_logits = nullptr;
   float* gen_probs = nullptr;
+  int* gen_state = nullptr;  // [0] column being generated, [1 .. max_batch] positions
+  cudaGraphExec_t gen_exec = nullptr;
+  cudaStream_t gen_exec_stream = nullptr;
 };
 
 namespace {
@@ -297,18 +301,21 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
 }
 
 // embedding -> blocks -> final norm -> LM head
+// col (device, optional; then T = 1): the tokens are column *col of `tokens`
+// and sit at position *col; the embedding writes those positions to sp_dev.
 int run_model(llama_ctx* c, const int32_t* tokens, int tok_stride, int B, int T, const int* sp_dev, int sp_host,
-              float* logits, int all_positions, cudaStream_t st) {
+              float* logits, int all_positions, cudaStream_t st, const int* col = nullptr) {
   if (!c->head_set) return LLAMA_ERR_NOT_READY;
   for (int l = 0; l < c->L; ++l)
     if (!c->layers[l].set) return LLAMA_ERR_NOT_READY;
   const int M = B * T;
   int r;
   if ((r = reserve(c, M))) return r;
+  int* pos_out = col ? const_cast<int*>(sp_dev) : nullptr;
   if (c->bf16)
-    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st);
+    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col, pos_out);
   else
-    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st);
+    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col, pos_out);
   for (int l = 0; l < c->L; ++l)
     if ((r = run_block(c, l, c->h, B, T, sp_dev, sp_host, st))) return r;
   const int rows = all_positions ? M : B;
@@ -505,6 +512,8 @@ void llama_destroy(llama_ctx* c) {
   release(reinterpret_cast<void*&>(c->ssq));
   release(reinterpret_cast<void*&>(c->gen_logits));
   release(reinterpret_cast<void*&>(c->gen_probs));
+  release(reinterpret_cast<void*&>(c->gen_state));
+  if (c->gen_exec) cudaGraphExecDestroy(c->gen_exec);
   delete c;
 }
 
@@ -634,18 +643,75 @@ int llama_generate(llama_ctx* c, int32_t* tokens, const uint8_t* prompt_mask, in
     const size_t n = (size_t)c->Bm * c->V * sizeof(float);
     if ((r = alloc(reinterpret_cast<void**>(&c->gen_logits), n))) return r;
     if ((r = alloc(reinterpret_cast<void**>(&c->gen_probs), n))) return r;
+    if ((r = alloc(reinterpret_cast<void**>(&c->gen_state), (size_t)(1 + c->Bm) * sizeof(int)))) return r;
+  }
+  if ((r = reserve(c, B * min_prompt_len))) return r;
+  if (c->gen_exec) {  // the previous call's graph: let its launches finish, then release it
+    cudaStreamSynchronize(c->gen_exec_stream);
+    cudaGraphExecDestroy(c->gen_exec);
+    c->gen_exec = nullptr;
   }
   cudaStream_t st = S_(stream);
-  int prev = 0;
-  for (int cur = min_prompt_len; cur < total_len; ++cur) {
-    // Transformer.forward(tokens[:, prev:cur], prev), last position only
-    if ((r = run_model(c, tokens + prev, total_len, B, cur - prev, nullptr, prev, c->gen_logits, 0, st))) return r;
-    // next token unless the sequence's prompt still covers position cur
-    if (launch_sample(c->gen_logits, B, c->V, temperature, top_p, greedy ? nullptr : uniforms + (size_t)cur * B,
-                      c->gen_probs, tokens + cur, total_len, prompt_mask + cur, total_len, st) != cudaSuccess)
+  const float* uni = greedy ? nullptr : uniforms;
+  // Transformer.forward(tokens[:, prev:cur], prev) with last-position logits,
+  // then the next token unless the sequence's prompt still covers position cur
+  auto host_step = [&](int prev, int cur) -> int {
+    int rr;
+    if ((rr = run_model(c, tokens + prev, total_len, B, cur - prev, nullptr, prev, c->gen_logits, 0, st))) return rr;
+    return launch_sample(c->gen_logits, B, c->V, temperature, top_p, uni ? uni + (size_t)cur * B : nullptr,
+                         c->gen_probs, tokens + cur, total_len, prompt_mask + cur, total_len, st) == cudaSuccess
+               ? LLAMA_OK
+               : LLAMA_ERR_CUDA;
+  };
+  // One decode step whose column lives on the device (gen_state[0] = prev,
+  // the column and position of the token fed in; the token chosen goes to
+  // column prev + 1): the same kernels, so a CUDA graph of it replays unchanged.
+  int* col = c->gen_state;
+  int* pos = c->gen_state + 1;
+  auto device_step = [&](cudaStream_t s) -> int {
+    int rr;
+    if ((rr = run_model(c, tokens, total_len, B, 1, pos, 0, c->gen_logits, 0, s, col))) return rr;
+    if (launch_sample(c->gen_logits, B, c->V, temperature, top_p, uni ? uni + B : nullptr, c->gen_probs, tokens + 1,
+                      total_len, prompt_mask + 1, total_len, s, col) != cudaSuccess)
       return LLAMA_ERR_CUDA;
-    prev = cur;
+    return launch_step_counter(col, 0, 1, s) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  };
+  if (min_prompt_len >= total_len) return LLAMA_OK;
+  // the prompt prefix, then one decode step per remaining position
+  if ((r = host_step(0, min_prompt_len))) return r;
+  const int first = min_prompt_len + 1, n_dec = total_len - first;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return LLAMA_ERR_CUDA;
+  if (n_dec < 3 || cap != cudaStreamCaptureStatusNone) {
+    // few steps, or the caller is capturing this stream itself: plain launches
+    for (int cur = first; cur < total_len; ++cur)
+      if ((r = host_step(cur - 1, cur))) return r;
+    return LLAMA_OK;
   }
+  // the first decode step runs directly (it also sets up every kernel it uses
+  // on this device); the rest replay a graph captured from one step
+  if (launch_step_counter(col, first - 1, 0, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+  if ((r = device_step(st))) return r;
+  cudaStream_t cs;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return LLAMA_ERR_CUDA;
+  cudaGraph_t graph = nullptr;
+  r = LLAMA_OK;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    r = LLAMA_ERR_CUDA;
+  } else {
+    const int rs = device_step(cs);
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess || rs != LLAMA_OK) r = rs != LLAMA_OK ? rs : LLAMA_ERR_CUDA;
+  }
+  cudaStreamDestroy(cs);
+  if (r == LLAMA_OK && cudaGraphInstantiate(&c->gen_exec, graph, 0) != cudaSuccess) r = LLAMA_ERR_CUDA;
+  if (graph) cudaGraphDestroy(graph);
+  if (r != LLAMA_OK) {
+    c->gen_exec = nullptr;
+    return r;
+  }
+  c->gen_exec_stream = st;
+  for (int i = 1; i < n_dec; ++i)
+    if (cudaGraphLaunch(c->gen_exec, st) != cudaSuccess) return LLAMA_ERR_CUDA;
   return LLAMA_OK;
 }
 

@@ -68,14 +68,22 @@ __device__ float bisect_threshold(const float* p, int V, float target, float flo
 }
 
 // one CTA per sequence; logits [B][V] (row stride V); writes out[b * out_stride]
-// unless keep[b * keep_stride] is set (then the token already there stays)
+// unless keep[b * keep_stride] is set (then the token already there stays).
+// With col (a captured decode step) out and keep move by *col columns and the
+// uniforms by *col rows of B.
 __global__ void __launch_bounds__(ST) sample_kernel(const float* __restrict__ logits, int V, float temperature,
                                                     float top_p, const float* __restrict__ uniforms,
                                                     float* __restrict__ scratch, int32_t* __restrict__ out,
                                                     int out_stride, const uint8_t* __restrict__ keep,
-                                                    int keep_stride) {
+                                                    int keep_stride, const int* col) {
   pdl_wait();
   pdl_trigger();
+  if (col) {
+    const int c0 = *col;
+    out += c0;
+    if (keep) keep += c0;
+    if (uniforms) uniforms += (size_t)c0 * gridDim.x;
+  }
   __shared__ float red[ST / 32];
   __shared__ int red_i[ST / 32];
   const int b = blockIdx.x;
@@ -183,9 +191,9 @@ __global__ void __launch_bounds__(ST) sample_kernel(const float* __restrict__ lo
 
 cudaError_t launch_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
                           float* scratch, int32_t* out, int out_stride, const uint8_t* keep, int keep_stride,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int* col) {
   return launch_pdl(sample_kernel, dim3(B), dim3(ST), 0, st, logits, V, temperature, top_p, uniforms, scratch, out,
-                    out_stride, keep, keep_stride);
+                    out_stride, keep, keep_stride, col);
 }
 
 }  // namespace llama
