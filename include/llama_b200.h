@@ -290,6 +290,19 @@ int llama_get_error(llama_ctx* ctx, int* flags);
  */
 int llama_selftest_bounded_wait(int which, int* flags, double* seconds);
 
+/*
+ * Failure injection for out-of-memory handling (the pages have no
+ * counterpart): cap the device memory the library may hold, summed over all
+ * its allocations in this process (contexts, workspaces, scratch); 0 removes
+ * the cap (the default). An allocation that would pass the cap fails as if the
+ * device were full: the call returns LLAMA_ERR_OOM and frees what it had
+ * allocated so far. llama_allocated_bytes returns the bytes the library holds
+ * now (every allocation is tracked, so a failed call can be checked for
+ * leaks). Thread-safe. llama_set_alloc_limit always returns LLAMA_OK.
+ */
+int llama_set_alloc_limit(uint64_t bytes);
+uint64_t llama_allocated_bytes(void);
+
 /* A static description of an error code. */
 const char* llama_strerror(int code);
 

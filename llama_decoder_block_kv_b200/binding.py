@@ -36,7 +36,7 @@ EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_laye
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
             "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel", "llama_tile_weights",
-            "llama_selftest_bounded_wait")
+            "llama_selftest_bounded_wait", "llama_set_alloc_limit", "llama_allocated_bytes")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -88,9 +88,12 @@ def lib() -> ctypes.CDLL:
         L.llama_set_decode_kernel.argtypes = [vp, i]
         L.llama_tile_weights.argtypes = [vp, vp, i, i, vp]
         L.llama_selftest_bounded_wait.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_double)]
+        L.llama_set_alloc_limit.argtypes = [ctypes.c_uint64]
+        L.llama_allocated_bytes.argtypes = []
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
+        L.llama_allocated_bytes.restype = ctypes.c_uint64
         _lib = L
     return _lib
 
@@ -221,6 +224,15 @@ def llama_get_error(ctx):
     flags = ctypes.c_int(0)
     code = lib().llama_get_error(ctx, ctypes.byref(flags))
     return code, flags.value
+
+
+def llama_set_alloc_limit(nbytes: int) -> None:
+    """Cap the device memory the library may hold (0: no cap); see the header."""
+    _check(lib().llama_set_alloc_limit(int(nbytes)), "llama_set_alloc_limit")
+
+
+def llama_allocated_bytes() -> int:
+    return int(lib().llama_allocated_bytes())
 
 
 def llama_selftest_bounded_wait(which: int):

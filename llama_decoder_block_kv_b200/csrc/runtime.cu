@@ -17,6 +17,8 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "kernels.cuh"
@@ -89,19 +91,42 @@ namespace {
     if (e_ != cudaSuccess) return LLAMA_ERR_CUDA; \
   } while (0)
 
+// Every device allocation of the library goes through alloc / release, which
+// keep the live total and honour the optional cap of llama_set_alloc_limit.
+std::mutex g_alloc_mu;
+std::unordered_map<void*, size_t> g_alloc_sizes;
+uint64_t g_alloc_total = 0, g_alloc_limit = 0;
+
 int alloc(void** p, size_t bytes) {
   *p = nullptr;
   if (bytes == 0) return LLAMA_OK;
+  std::lock_guard<std::mutex> lock(g_alloc_mu);
+  if (g_alloc_limit && g_alloc_total + bytes > g_alloc_limit) return LLAMA_ERR_OOM;
   cudaError_t e = cudaMalloc(p, bytes);
   if (e == cudaErrorMemoryAllocation) {
     cudaGetLastError();
+    *p = nullptr;
     return LLAMA_ERR_OOM;
   }
-  return e == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    return LLAMA_ERR_CUDA;
+  }
+  g_alloc_sizes[*p] = bytes;
+  g_alloc_total += bytes;
+  return LLAMA_OK;
 }
 
 void release(void*& p) {
-  if (p) cudaFree(p);
+  if (p) {
+    cudaFree(p);
+    std::lock_guard<std::mutex> lock(g_alloc_mu);
+    auto it = g_alloc_sizes.find(p);
+    if (it != g_alloc_sizes.end()) {
+      g_alloc_total -= it->second;
+      g_alloc_sizes.erase(it);
+    }
+  }
   p = nullptr;
 }
 
@@ -538,7 +563,7 @@ int llama_set_layer(llama_ctx* c, int layer, const void* wq, const void* wk, con
   auto done = [&](int code) {
     if (tmp) {
       cudaDeviceSynchronize();
-      cudaFree(tmp);
+      release(tmp);
     }
     return code;
   };
@@ -824,6 +849,17 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
              : LLAMA_ERR_CUDA;
 }
 
+int llama_set_alloc_limit(uint64_t bytes) {
+  std::lock_guard<std::mutex> lock(g_alloc_mu);
+  g_alloc_limit = bytes;
+  return LLAMA_OK;
+}
+
+uint64_t llama_allocated_bytes(void) {
+  std::lock_guard<std::mutex> lock(g_alloc_mu);
+  return g_alloc_total;
+}
+
 int llama_selftest_bounded_wait(int which, int* flags, double* seconds) {
   if (flags) *flags = 0;
   if (seconds) *seconds = 0.0;
@@ -847,7 +883,7 @@ int llama_selftest_bounded_wait(int which, int* flags, double* seconds) {
   if (code == LLAMA_OK && (cudaMemcpy(&f, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
                            cudaMemcpy(&ns, elapsed, sizeof(ns), cudaMemcpyDeviceToHost) != cudaSuccess))
     code = LLAMA_ERR_CUDA;
-  cudaFree(buf);
+  release(buf);
   if (flags) *flags = f;
   if (seconds) *seconds = (double)ns * 1e-9;
   return code;

@@ -101,3 +101,22 @@ def test_wrappers_reach_the_library_without_a_device():
     with pytest.raises(B.LlamaError) as e:
         B.llama_reset(None)
     assert e.value.code == B.LLAMA_ERR_INVALID_ARGS
+
+
+def test_allocation_cap_fails_create_cleanly_on_the_host():
+    """Injected allocation failure: with a one-byte cap the first device
+    allocation of llama_create fails before cudaMalloc is reached, the call
+    returns LLAMA_ERR_OOM and the library holds nothing afterwards."""
+    args = B.ModelArgs(dim=256, n_layers=2, n_heads=4, n_kv_heads=2, vocab_size=1000, multiple_of=256,
+                       ffn_dim_multiplier=None, norm_eps=1e-5, rope_theta=10000.0, max_batch_size=1,
+                       max_seq_len=64, dtype="bf16").c()
+    before = B.llama_allocated_bytes()
+    B.llama_set_alloc_limit(1)
+    try:
+        ctx = ctypes.c_void_p()
+        code = B.lib().llama_create(ctypes.byref(args), ctypes.byref(ctx))
+        assert code == B.LLAMA_ERR_OOM
+        assert not ctx.value
+        assert B.llama_allocated_bytes() == before
+    finally:
+        B.llama_set_alloc_limit(0)
