@@ -57,6 +57,7 @@ extern "C" {
 #define LLAMA_ERR_CUDA -3         /* a CUDA runtime/driver call failed */
 #define LLAMA_ERR_NOT_READY -4    /* weights for a needed layer/head not set */
 #define LLAMA_ERR_TOO_LARGE -5    /* a size needs more than llama_linear_noalloc's fixed scratch */
+#define LLAMA_ERR_INTERNAL -6     /* an internal consistency check failed (llama_selfcheck_plans) */
 #define LLAMA_ERR_TOKEN_RANGE -10 /* device flag: a token id outside [0, vocab_size) */
 #define LLAMA_ERR_POS_RANGE -11   /* device flag: start_pos[b] + s outside [0, max_seq_len) */
 #define LLAMA_ERR_TIMEOUT -12     /* device flag: a bounded in-kernel wait gave up */
@@ -289,6 +290,19 @@ int llama_get_error(llama_ctx* ctx, int* flags);
  * LLAMA_ERR_CUDA or LLAMA_ERR_OOM when it could not run.
  */
 int llama_selftest_bounded_wait(int which, int* flags, double* seconds);
+
+/*
+ * Host-only consistency check of the work partitions the decode kernels use
+ * (the pages have no counterpart; it stands in for a sanitizer run): for M
+ * tokens and a model of these sizes it walks, on the host and with the
+ * kernels' own index functions, every CTA's share of the stream-K split of
+ * each decode linear and of the persistent decode kernel, and checks that
+ * every weight tile is covered exactly once and in bounds, that each split
+ * row block's partial slots are distinct and fit the workspace, and that the
+ * attention partials fit. Returns LLAMA_OK, LLAMA_ERR_INTERNAL when a check
+ * fails, or LLAMA_ERR_INVALID_ARGS for sizes the library rejects. Needs no GPU.
+ */
+int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, int max_seq_len, int num_sms);
 
 /*
  * Failure injection for out-of-memory handling (the pages have no

@@ -24,6 +24,7 @@ LLAMA_ERR_OOM = -2
 LLAMA_ERR_CUDA = -3
 LLAMA_ERR_NOT_READY = -4
 LLAMA_ERR_TOO_LARGE = -5
+LLAMA_ERR_INTERNAL = -6
 LLAMA_ERR_TOKEN_RANGE = -10
 LLAMA_ERR_POS_RANGE = -11
 LLAMA_ERR_TIMEOUT = -12
@@ -36,7 +37,8 @@ EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_laye
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
             "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel", "llama_tile_weights",
-            "llama_selftest_bounded_wait", "llama_set_alloc_limit", "llama_allocated_bytes")
+            "llama_selftest_bounded_wait", "llama_set_alloc_limit", "llama_allocated_bytes",
+            "llama_selfcheck_plans")
 
 
 class LlamaArgs(ctypes.Structure):
@@ -90,6 +92,7 @@ def lib() -> ctypes.CDLL:
         L.llama_selftest_bounded_wait.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_double)]
         L.llama_set_alloc_limit.argtypes = [ctypes.c_uint64]
         L.llama_allocated_bytes.argtypes = []
+        L.llama_selfcheck_plans.argtypes = [i] * 7
         for name in EXPORTED:
             if name not in ("llama_destroy", "llama_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -229,6 +232,12 @@ def llama_get_error(ctx):
 def llama_set_alloc_limit(nbytes: int) -> None:
     """Cap the device memory the library may hold (0: no cap); see the header."""
     _check(lib().llama_set_alloc_limit(int(nbytes)), "llama_set_alloc_limit")
+
+
+def llama_selfcheck_plans(M: int, dim: int, n_heads: int, n_kv_heads: int, ffn: int, max_seq_len: int,
+                          num_sms: int = 148) -> int:
+    """Host-only walk of the decode kernels' work partitions; returns the C code (0 = consistent)."""
+    return lib().llama_selfcheck_plans(M, dim, n_heads, n_kv_heads, ffn, max_seq_len, num_sms)
 
 
 def llama_allocated_bytes() -> int:

@@ -36,6 +36,9 @@
 // records LLAMA_DEV_TIMEOUT and the CTA unwinds.
 #include "kernels.cuh"
 
+#include <algorithm>
+#include <vector>
+
 namespace llama {
 
 namespace {
@@ -939,6 +942,73 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
   pl.counters = counters;
   pl.ok = true;
   return pl;
+}
+
+// Host-side walk of a plan with the kernel's own index functions (the
+// producer's cursor and the consumers' segments): every stage of every linear
+// belongs to one CTA; the cursor's tile equals db_locate's at every stage;
+// tiles lie inside the weight matrix; a CTA's x slice fits the shared area;
+// each row block's partial slots are 0 .. count-1 and fit the workspace; the
+// attention's partials and counters fit too.
+bool check_decode_block_plan(const DecodeBlockPlan& pl, int M, int H, size_t part_floats, int counters_n) {
+  if (!pl.ok) return false;
+  const int grid = pl.grid;
+  for (int li = 0; li < 4; ++li) {
+    const DbLinear& L = pl.lin[li];
+    std::vector<int> seen(L.total, 0);
+    std::vector<std::vector<int>> slots(L.RB);
+    std::vector<int> counts(L.RB, -1);
+    for (int cta = 0; cta < grid; ++cta) {
+      int x, end;
+      db_range(L, cta, grid, x, end);
+      if (x >= end) continue;
+      DbStage S = db_locate(L, x);
+      int rb = S.rb, kl = x - S.reg_beg, sl = S.s, start = S.start, len = S.len;  // the producer's cursor
+      int seg_first = x;
+      for (; x < end; ++x) {
+        const DbStage T = db_locate(L, x);
+        if (T.rb != rb || T.start + (x - T.reg_beg) != start + kl) return false;
+        if (rb >= L.RB || start + kl >= L.NK) return false;
+        if ((size_t)M * ((size_t)T.len * 64 + 8) * 2 > DB_AREA_BYTES) return false;
+        ++seen[x];
+        const bool seg_ends = x + 1 == end || x + 1 == T.reg_beg + T.len;
+        if (seg_ends) {
+          const bool whole = L.S == 1 && seg_first == T.reg_beg && x + 1 == T.reg_beg + T.len;
+          if (!whole) {
+            int slot = 0;
+            const int count = db_contributors(L, T.rb, grid, T.s, cta, &slot);
+            if (slot < 0 || slot >= count || (size_t)count * M * L.N > part_floats) return false;
+            if (counts[T.rb] >= 0 && counts[T.rb] != count) return false;
+            counts[T.rb] = count;
+            slots[T.rb].push_back(slot);
+          }
+          seg_first = x + 1;
+        }
+        if (++kl == len) {
+          kl = 0;
+          if (++rb == L.RB) {
+            rb = 0;
+            ++sl;
+            start = db_slice_start(L, sl);
+            len = db_slice_start(L, sl + 1) - start;
+          }
+        }
+      }
+    }
+    for (int v : seen)
+      if (v != 1) return false;
+    for (int r = 0; r < L.RB; ++r) {
+      if (counts[r] < 0) continue;
+      std::vector<int> v = slots[r];
+      std::sort(v.begin(), v.end());
+      if ((int)v.size() != counts[r]) return false;
+      for (int i = 0; i < counts[r]; ++i)
+        if (v[i] != i) return false;
+    }
+    if (L.RB > counters_n) return false;
+  }
+  if ((size_t)M * H * pl.max_chunks * (AD + 2) > part_floats) return false;
+  return true;
 }
 
 template <int MB>

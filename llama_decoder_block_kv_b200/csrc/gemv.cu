@@ -24,6 +24,9 @@
 // launches. A row block inside one range goes straight to the epilogue.
 #include "kernels.cuh"
 
+#include <algorithm>
+#include <vector>
+
 namespace llama {
 
 namespace {
@@ -274,6 +277,49 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
   p.S = smax;
   p.part_floats = smax > 1 ? (size_t)smax * M * N : 0;
   return p;
+}
+
+// Host-side walk of a plan with the kernel's own index functions: every
+// weight stage belongs to exactly one CTA's range; a row block split across
+// CTAs gets one partial slot per contributor, the slots are 0 .. count-1 with
+// count <= S, and the partial workspace holds S x M x N floats.
+bool check_gemv_plan(int M, int N, int K, int num_sms) {
+  const GemvPlan p = plan_gemv(M, N, K, num_sms);
+  if (p.grid < 1 || p.total < 1 || K % KB) return false;
+  std::vector<int> seen(p.total, 0);
+  std::vector<std::vector<int>> slots(p.row_blocks);
+  std::vector<int> counts(p.row_blocks, -1);
+  for (int cta = 0; cta < p.grid; ++cta) {
+    const int sbeg = sk_begin(cta, p.total, p.grid), send = sk_begin(cta + 1, p.total, p.grid);
+    if (sbeg >= send) return false;  // every CTA of the grid has work
+    for (int x = sbeg; x < send;) {
+      const int rb = x / p.nk, seg_beg = x, seg_end = std::min(send, (rb + 1) * p.nk);
+      if (rb >= p.row_blocks) return false;
+      for (int y = seg_beg; y < seg_end; ++y) ++seen[y];
+      if (!(seg_beg == rb * p.nk && seg_end == (rb + 1) * p.nk)) {
+        const int c_first = sk_owner(rb * p.nk, p.total, p.grid);
+        const int c_last = sk_owner((rb + 1) * p.nk - 1, p.total, p.grid);
+        const int count = c_last - c_first + 1, slot = cta - c_first;
+        if (slot < 0 || slot >= count || count > p.S) return false;
+        if (counts[rb] >= 0 && counts[rb] != count) return false;
+        counts[rb] = count;
+        slots[rb].push_back(slot);
+      }
+      x = seg_end;
+    }
+  }
+  for (int v : seen)
+    if (v != 1) return false;
+  for (int rb = 0; rb < p.row_blocks; ++rb) {
+    if (counts[rb] < 0) continue;
+    std::vector<int> sl = slots[rb];
+    std::sort(sl.begin(), sl.end());
+    if ((int)sl.size() != counts[rb]) return false;
+    for (int i = 0; i < counts[rb]; ++i)
+      if (sl[i] != i) return false;
+  }
+  if (p.S > 1 && p.part_floats < (size_t)p.S * M * N) return false;
+  return true;
 }
 
 template <int MB>

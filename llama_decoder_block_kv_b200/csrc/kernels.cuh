@@ -69,6 +69,7 @@ struct GemvPlan {
   size_t part_floats = 0;
 };
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
+bool check_gemv_plan(int M, int N, int K, int num_sms);  // host walk of a plan (see gemv.cu)
 // W: [N][K] row-major (tiled = 0) or the library's weight tiles (tiled = 1, tile_weights)
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
                              float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
@@ -149,6 +150,7 @@ DecodeBlockPlan plan_decode_block(int M, int dim, int H, int Hkv, int D, int F, 
 // maps: wqkv, wo, w1|w3, w2 (128-row x 64-k boxes), then the layer's K and V caches (64-row x 64 boxes)
 cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st);
 size_t decode_block_smem(int M);
+bool check_decode_block_plan(const DecodeBlockPlan& pl, int M, int H, size_t part_floats, int counters_n);
 // failure-detection self-tests (selftest.cu, decode_block.cu): a bounded wait that nothing completes
 cudaError_t launch_grid_barrier_selftest(void* gbar, int* err, unsigned long long* elapsed, cudaStream_t st);
 cudaError_t launch_mbarrier_selftest(int* err, unsigned long long* elapsed, cudaStream_t st);

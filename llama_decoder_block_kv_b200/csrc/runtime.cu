@@ -817,6 +817,7 @@ const char* llama_strerror(int code) {
     case LLAMA_ERR_CUDA: return "CUDA error";
     case LLAMA_ERR_NOT_READY: return "weights not set";
     case LLAMA_ERR_TOO_LARGE: return "size exceeds the fixed scratch of llama_linear_noalloc";
+    case LLAMA_ERR_INTERNAL: return "an internal consistency check failed";
     case LLAMA_ERR_TOKEN_RANGE: return "token id outside [0, vocab_size)";
     case LLAMA_ERR_POS_RANGE: return "position outside [0, max_seq_len)";
     case LLAMA_ERR_TIMEOUT: return "a bounded device wait timed out";
@@ -847,6 +848,24 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
                  cudaSuccess
              ? LLAMA_OK
              : LLAMA_ERR_CUDA;
+}
+
+int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, int max_seq_len, int num_sms) {
+  if (M < 1 || dim < 64 || n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || dim % n_heads || ffn < 64 ||
+      max_seq_len < 1 || num_sms < 1 || dim % 64 || ffn % 64)
+    return LLAMA_ERR_INVALID_ARGS;
+  const int D = dim / n_heads, n_qkv = (n_heads + 2 * n_kv_heads) * D;
+  // the decode GEMV of every linear, for the tokens given
+  if (M <= 32) {
+    const int Ns[4] = {n_qkv, dim, 2 * ffn, dim};
+    const int Ks[4] = {dim, n_heads * D, dim, ffn};
+    for (int i = 0; i < 4; ++i)
+      if (Ks[i] % 64 == 0 && !check_gemv_plan(M, Ns[i], Ks[i], num_sms)) return LLAMA_ERR_INTERNAL;
+  }
+  // the persistent decode kernel, with the workspace a context would hold
+  DecodeBlockPlan pl = plan_decode_block(M, dim, n_heads, n_kv_heads, D, ffn, max_seq_len, max_seq_len, num_sms);
+  if (pl.ok && !check_decode_block_plan(pl, M, n_heads, pl.part_floats, pl.counters)) return LLAMA_ERR_INTERNAL;
+  return LLAMA_OK;
 }
 
 int llama_set_alloc_limit(uint64_t bytes) {

@@ -1,0 +1,51 @@
+"""Host-only consistency of the decode kernels' work partitions
+(llama_selfcheck_plans walks them with the kernels' own index functions):
+every weight tile covered exactly once and in bounds, split-K partial slots
+distinct and inside the workspace, for the workloads' shapes, the test shapes,
+every batch of up to 32 tokens and several SM counts."""
+import os
+import random
+
+import pytest
+
+from llama_decoder_block_kv_b200 import binding as B
+import oracle as O
+
+pytestmark = pytest.mark.skipif(not os.path.exists(B.LIB_PATH), reason="library not built")
+
+SHAPES = [  # dim, heads, kv heads, ffn, max_seq_len
+    (4096, 32, 32, 11008, 2048),                          # LLaMA-7B layer
+    (8192, 64, 8, 28672, 8192),                           # LLaMA-2-70B layer
+    (4096, 32, 8, 14336, 8192),                           # LLaMA-3-8B
+    (512, 4, 2, O.ffn_hidden_dim(512, 256), 256),
+    (1024, 8, 1, O.ffn_hidden_dim(1024, 256), 4096),
+    (2048, 16, 2, O.ffn_hidden_dim(2048, 256), 256),
+    (2048, 32, 1, O.ffn_hidden_dim(2048, 256), 16384),
+    (256, 4, 1, 768, 64),                                 # head_dim 64: GEMV only
+]
+
+
+@pytest.mark.parametrize("dim,H,Hkv,F,S", SHAPES)
+def test_plans_of_the_workload_and_test_shapes(dim, H, Hkv, F, S):
+    for M in (1, 2, 5, 8, 9, 16, 17, 24, 25, 32):
+        for sms in (148, 132):
+            assert B.llama_selfcheck_plans(M, dim, H, Hkv, F, S, sms) == B.LLAMA_OK, (M, sms)
+
+
+def test_plans_of_random_shapes_and_grids():
+    rng = random.Random(7)
+    for _ in range(60):
+        D = rng.choice([64, 128])
+        Hkv = rng.choice([1, 2, 4, 8])
+        H = Hkv * rng.choice([1, 2, 4, 8, 16])
+        dim = H * D
+        F = 64 * rng.randint(2, 200)
+        M = rng.randint(1, 32)
+        sms = rng.choice([1, 3, 7, 64, 100, 148, 160])
+        assert B.llama_selfcheck_plans(M, dim, H, Hkv, F, 128 * rng.randint(1, 64), sms) == B.LLAMA_OK, \
+            (M, dim, H, Hkv, F, sms)
+
+
+def test_selfcheck_rejects_bad_sizes():
+    assert B.llama_selfcheck_plans(0, 4096, 32, 32, 11008, 2048, 148) == B.LLAMA_ERR_INVALID_ARGS
+    assert B.llama_selfcheck_plans(1, 4096, 32, 3, 11008, 2048, 148) == B.LLAMA_ERR_INVALID_ARGS
