@@ -183,9 +183,9 @@ __global__ void kv_to_logical_kernel(const T* __restrict__ src, T* __restrict__ 
 // host launchers
 
 template <typename T>
-void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
-                  int tok_stride, int* err, cudaStream_t st, const int* col, int* pos) {
-  launch_pdl(embed_gather_kernel<T>, dim3(n_tok), dim3(128), 0, st, tokens, reinterpret_cast<const T*>(table), h, dim,
+cudaError_t launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
+                         int tok_stride, int* err, cudaStream_t st, const int* col, int* pos) {
+  return launch_pdl(embed_gather_kernel<T>, dim3(n_tok), dim3(128), 0, st, tokens, reinterpret_cast<const T*>(table), h, dim,
              vocab, T_, tok_stride, err, col, pos);
 }
 
@@ -203,13 +203,13 @@ cudaError_t launch_step_counter(int* col, int value, int add, cudaStream_t st) {
 }
 
 template <typename T>
-void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
-                    int in_row_offset, cudaStream_t st) {
+cudaError_t launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps,
+                           int in_row_stride_T, int in_row_offset, cudaStream_t st) {
   if (dim >= 4096)  // one float4 per thread and pass at dim 4096 (a row is read in one round trip)
-    launch_pdl(rmsnorm_kernel<T, 1024>, dim3(rows), dim3(1024), 0, st, h, reinterpret_cast<const T*>(w),
+    return launch_pdl(rmsnorm_kernel<T, 1024>, dim3(rows), dim3(1024), 0, st, h, reinterpret_cast<const T*>(w),
                reinterpret_cast<T*>(out), dim, eps, in_row_stride_T, in_row_offset);
   else
-    launch_pdl(rmsnorm_kernel<T, 64>, dim3(rows), dim3(64), 0, st, h, reinterpret_cast<const T*>(w),
+    return launch_pdl(rmsnorm_kernel<T, 64>, dim3(rows), dim3(64), 0, st, h, reinterpret_cast<const T*>(w),
                reinterpret_cast<T*>(out), dim, eps, in_row_stride_T, in_row_offset);
 }
 
@@ -234,9 +234,10 @@ void launch_rope_rows_to_interleaved(const void* src, void* dst, int heads, int 
 }
 
 #define INST(T)                                                                                              \
-  template void launch_embed<T>(const int*, const void*, float*, int, int, int, int, int, int*, cudaStream_t, \
-                                const int*, int*);                                                          \
-  template void launch_rmsnorm<T>(const float*, const void*, void*, int, int, float, int, int, cudaStream_t); \
+  template cudaError_t launch_embed<T>(const int*, const void*, float*, int, int, int, int, int, int*,       \
+                                       cudaStream_t, const int*, int*);                                  \
+  template cudaError_t launch_rmsnorm<T>(const float*, const void*, void*, int, int, float, int, int,       \
+                                         cudaStream_t);                                                   \
   template void launch_pack_w13<T>(const void*, const void*, void*, int, int, cudaStream_t);                 \
   template void launch_kv_convert<T>(const void*, void*, int, int, int, int, int, int, cudaStream_t);   \
   template void launch_rope_rows_to_interleaved<T>(const void*, void*, int, int, int, cudaStream_t);

@@ -42,12 +42,12 @@ cudaError_t ensure_smem(void (*kernel)(KArgs...), size_t bytes, std::atomic<unsi
 
 // elementwise.cu
 template <typename T>
-void launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
-                  int tok_stride, int* err, cudaStream_t st, const int* col = nullptr, int* pos = nullptr);
+cudaError_t launch_embed(const int* tokens, const void* table, float* h, int n_tok, int dim, int vocab, int T_,
+                         int tok_stride, int* err, cudaStream_t st, const int* col = nullptr, int* pos = nullptr);
 cudaError_t launch_step_counter(int* col, int value, int add, cudaStream_t st);
 template <typename T>
-void launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps, int in_row_stride_T,
-                    int in_row_offset, cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* h, const void* w, void* out, int rows, int dim, float eps,
+                           int in_row_stride_T, int in_row_offset, cudaStream_t st);
 template <typename T>
 void launch_pack_w13(const void* w1, const void* w3, void* out, int F, int dim, cudaStream_t st);
 template <typename T>

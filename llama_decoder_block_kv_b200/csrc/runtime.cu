@@ -269,10 +269,9 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
     r = run_block_persistent(c, layer, h, B, sp_dev, sp_host, st);
     return r == 1 ? LLAMA_ERR_INVALID_ARGS : r;
   }
-  if (c->bf16)
-    launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
-  else
-    launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
+               : launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
+    return LLAMA_ERR_CUDA;
 
   EpiParams e = epi_base(c, EPI_QKV_ROPE, M, c->n_qkv);
   e.q_out = c->q;
@@ -310,10 +309,9 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.ld_out = c->dim;
   if ((r = gemm(c, c->o, Ly.wo, M, c->dim, HD, e, st))) return r;
 
-  if (c->bf16)
-    launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
-  else
-    launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st);
+  if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
+               : launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
+    return LLAMA_ERR_CUDA;
 
   e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
   e.g_out = c->g;
@@ -337,19 +335,19 @@ int run_model(llama_ctx* c, const int32_t* tokens, int tok_stride, int B, int T,
   int r;
   if ((r = reserve(c, M))) return r;
   int* pos_out = col ? const_cast<int*>(sp_dev) : nullptr;
-  if (c->bf16)
-    launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col, pos_out);
-  else
-    launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col, pos_out);
+  if ((c->bf16 ? launch_embed<bf16>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col, pos_out)
+               : launch_embed<float>(tokens, c->tok_emb, c->h, M, c->dim, c->V, T, tok_stride, c->err, st, col,
+                                     pos_out)) != cudaSuccess)
+    return LLAMA_ERR_CUDA;
   for (int l = 0; l < c->L; ++l)
     if ((r = run_block(c, l, c->h, B, T, sp_dev, sp_host, st))) return r;
   const int rows = all_positions ? M : B;
   const int stride = all_positions ? 1 : T;
   const int offset = all_positions ? 0 : T - 1;
-  if (c->bf16)
-    launch_rmsnorm<bf16>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
-  else
-    launch_rmsnorm<float>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st);
+  if ((c->bf16 ? launch_rmsnorm<bf16>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset, st)
+               : launch_rmsnorm<float>(c->h, c->final_norm, c->xn, rows, c->dim, c->a.norm_eps, stride, offset,
+                                       st)) != cudaSuccess)
+    return LLAMA_ERR_CUDA;
   EpiParams e = epi_base(c, EPI_STORE_F32, rows, c->V);
   e.out = logits;
   e.ld_out = c->V;
