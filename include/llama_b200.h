@@ -29,13 +29,18 @@
  *    The residual stream h is always fp32.
  *  - Calls that take a cuda_stream (a cudaStream_t, may be NULL for the
  *    legacy default stream) are asynchronous and stream-ordered; the library
- *    never synchronises inside them, so they can be captured in a CUDA graph
- *    once llama_reserve has sized the workspace for the largest call.
+ *    synchronises inside them only where it must allocate (workspace growth,
+ *    first use of a private scratch) and where llama_generate releases the
+ *    previous call's graph, so once llama_reserve has sized the workspace for
+ *    the largest call they can be captured in a CUDA graph.
  *  - Every int-returning call returns LLAMA_OK (0) or a negative error code;
  *    an error returned before any launch leaves all state unchanged.
  *    Problems only the device can see (a token id out of range, a position
  *    past the cache, a bounded wait that timed out) set a device flag that
  *    llama_get_error reads back.
+ *  - A context belongs to the device that was current at llama_create (its
+ *    calls make that device current) and is used by one host thread at a
+ *    time; calls on different contexts may run concurrently.
  */
 #ifndef LLAMA_B200_H
 #define LLAMA_B200_H
