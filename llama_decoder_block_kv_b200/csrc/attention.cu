@@ -390,7 +390,7 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
   int ck = (max_len + want - 1) / want;
   ck = (ck + KT - 1) / KT * KT;
   if (ck < 128) ck = 128;  // at least two tiles per CTA (measured: 128 beats 256 and 512 on short histories)
-  if (ck > 1024) ck = 1024;
+  if (ck > 2048) ck = 2048;  // measured: 2048 beats 1024 and 4096 on long ragged histories (8B decode)
   p.CK = ck;
   p.max_chunks = (S_max + ck - 1) / ck;
   p.part_floats = (size_t)B * H * p.max_chunks * 128 + (size_t)B * H * p.max_chunks * 2;
