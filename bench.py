@@ -222,6 +222,7 @@ class LayerBench:
         self.args = B.ModelArgs.from_workload(w)
         self.model = B.Llama(self.args)
         B.llama_set_decode_kernel(self.model.ctx, DECODE_KERNELS[DECODE_KERNEL])
+        B.llama_set_decode_attention(self.model.ctx, DECODE_ATTENTIONS[DECODE_ATTENTION])
         self.lw = synth.layer_weights(w, 0, device="cuda")
         B.llama_set_layer(self.model.ctx, 0, self.lw)
         dim = w.dim
@@ -450,7 +451,7 @@ def run_ours(args, world, rank, local):
            "config": {"workload": w.name, "batch": lb.Bsz, "prefill_tokens": lb.P, "decode_steps": lb.ND,
                       "decode_start_pos": lb.dec_pos0, "l2": "inputs larger than L2: %.0f MB of weights per pass"
                       % (wbytes / 1e6), "parallelism": "replicas" if world > 1 else "single GPU",
-                      "decode_kernel": DECODE_KERNEL},
+                      "decode_kernel": DECODE_KERNEL, "decode_attention": DECODE_ATTENTION},
            "phases": phases, "roofline": roof, "e2e": e2e,
            "gpu_launches": lb.kernels_per_step() * args.steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -499,6 +500,7 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
     m = B.Llama(B.ModelArgs.from_workload(w))
     ctx = m.ctx
     B.llama_set_decode_kernel(ctx, DECODE_KERNELS[DECODE_KERNEL])
+    B.llama_set_decode_attention(ctx, DECODE_ATTENTIONS[DECODE_ATTENTION])
     for i in range(w.n_layers):
         B.llama_set_layer(ctx, i, synth.layer_weights(w, i, device="cuda"))
     enh = synth.embed_norm_head(w, device="cuda")
@@ -547,7 +549,8 @@ def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL}, "clocks": clocks, "device_error": code,
+           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL,
+                                                "decode_attention": DECODE_ATTENTION}, "clocks": clocks, "device_error": code,
            "gpu_launches": launches_per_step * args.steps}
     m.close()
     return out
@@ -579,6 +582,8 @@ def run_reference(args, world, rank):
 DECODE_KERNELS = {"auto": B.LLAMA_DECODE_AUTO, "layered": B.LLAMA_DECODE_LAYERED,
                   "persistent": B.LLAMA_DECODE_PERSISTENT}
 DECODE_KERNEL = "auto"
+DECODE_ATTENTIONS = {"auto": B.LLAMA_ATTN_AUTO, "chunked": B.LLAMA_ATTN_CHUNKED, "streamk": B.LLAMA_ATTN_STREAMK}
+DECODE_ATTENTION = "auto"
 CLOCK_LOG_DIR = os.environ.get("TMPDIR", "/tmp")
 
 
@@ -593,9 +598,12 @@ def main():
     ap.add_argument("--clock-log", default=None, help="directory for the per-rank clock sample CSV")
     ap.add_argument("--decode-kernel", default="auto", choices=sorted(DECODE_KERNELS),
                     help="decode-step launch structure (llama_set_decode_kernel)")
+    ap.add_argument("--decode-attention", default="auto", choices=sorted(DECODE_ATTENTIONS),
+                    help="decode attention kernel of the per-step launches (llama_set_decode_attention)")
     args = ap.parse_args()
-    global DECODE_KERNEL, CLOCK_LOG_DIR
+    global DECODE_KERNEL, DECODE_ATTENTION, CLOCK_LOG_DIR
     DECODE_KERNEL = args.decode_kernel
+    DECODE_ATTENTION = args.decode_attention
     if args.clock_log:
         CLOCK_LOG_DIR = args.clock_log
     if args.warmup < 3:

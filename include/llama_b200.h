@@ -79,6 +79,11 @@ extern "C" {
 #define LLAMA_DECODE_LAYERED 1    /* a kernel per step: RMSNorm, GEMV, attention, GEMV, RMSNorm, GEMV, GEMV */
 #define LLAMA_DECODE_PERSISTENT 2 /* always the persistent launch; an ineligible decode call fails */
 
+/* Decode attention kernel of the per-step launches, llama_set_decode_attention */
+#define LLAMA_ATTN_AUTO 0    /* the library's choice by shape */
+#define LLAMA_ATTN_CHUNKED 1 /* a CTA per (sequence, kv head group, chunk of keys) */
+#define LLAMA_ATTN_STREAMK 2 /* the key tiles of all sequences dealt out evenly over two CTAs per SM */
+
 /*
  * ModelArgs of the notes' section 3 code plus rope_theta ("灵哥讲llama3(中)",
  * Transformer class) and the storage type.
@@ -273,6 +278,27 @@ int llama_reset(llama_ctx* ctx);
 int llama_set_decode_kernel(llama_ctx* ctx, int mode);
 
 /*
+ * Choose the attention kernel that decode calls (T == 1, bf16) run in the
+ * per-step launches (LLAMA_ATTN_*); the persistent decode launch has its own.
+ * Both compute, for every sequence b and query head h, the softmax over the
+ * cached keys 0 .. start_pos[b] of kv head h / n_rep ("LLaMA: Open and
+ * Efficient Foundation Language Models" notes, Attention.forward and
+ * repeat_kv); they differ only in the order of fp32 sums.
+ *  LLAMA_ATTN_CHUNKED: a CTA per (sequence, kv head group, chunk of up to
+ *   2048 keys), merged by the CTA that finishes last.
+ *  LLAMA_ATTN_STREAMK: the 64-key tiles of all (sequence, kv head group)
+ *   units form one list cut into equal contiguous ranges, one per CTA, two
+ *   CTAs per SM; a unit split between CTAs is merged by the last of them.
+ *   Served when max_batch_size <= 1024 and head_dim is 64 or 128; a decode
+ *   call of another shape returns LLAMA_ERR_INVALID_ARGS before any launch.
+ *  LLAMA_ATTN_AUTO (the default): the kernel measured faster on B200 for the
+ *   call's shape.
+ * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it
+ * applies to calls made after it.
+ */
+int llama_set_decode_attention(llama_ctx* ctx, int mode);
+
+/*
  * Synchronise the device, then return and clear the device flags: LLAMA_OK,
  * or the most severe of LLAMA_ERR_TIMEOUT, LLAMA_ERR_POS_RANGE,
  * LLAMA_ERR_TOKEN_RANGE. *flags (if not NULL) receives the raw flag bits
@@ -304,7 +330,11 @@ int llama_selftest_bounded_wait(int which, int* flags, double* seconds);
  * each decode linear and of the persistent decode kernel, and checks that
  * every weight tile is covered exactly once and in bounds, that each split
  * row block's partial slots are distinct and fit the workspace, and that the
- * attention partials fit. Returns LLAMA_OK, LLAMA_ERR_INTERNAL when a check
+ * attention partials fit; and, for M sequences at several ragged and uniform
+ * position patterns, the stream-K decode attention's split: every key tile in
+ * exactly one CTA's range, each split unit merged from one partial of each CTA
+ * it spans, in distinct slots inside the workspace (M up to 1024 there).
+ * Returns LLAMA_OK, LLAMA_ERR_INTERNAL when a check
  * fails, or LLAMA_ERR_INVALID_ARGS for sizes the library rejects. Needs no GPU.
  */
 int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, int max_seq_len, int num_sms);

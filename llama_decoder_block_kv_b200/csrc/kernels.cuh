@@ -91,6 +91,18 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
 cudaError_t launch_attn_decode(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                const DecodePlan& p, int* err, cudaStream_t st);
+// attn_decode_sk.cu: the same decode attention with the key tiles of all
+// (sequence, head group) units dealt out stream-K over two CTAs per SM
+struct DecodeSkPlan {
+  bool ok = false;  // shape served (B <= 1024, head_dim 64 or 128, 32-bit split arithmetic)
+  int hpc = 1, grid = 1, units = 0;
+  size_t part_floats = 0;
+};
+DecodeSkPlan plan_decode_sk(int B, int H, int Hkv, int D, int max_len, int num_sms);
+cudaError_t launch_attn_decode_sk(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
+                                  int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
+                                  const DecodeSkPlan& p, int* err, cudaStream_t st);
+bool check_decode_sk(const DecodeSkPlan& p, const int* start_pos, int B, int H, int Hkv, int D, int S_max);
 // sample.cu
 // col (optional, device): out, keep and the uniforms row are offset by column *col
 cudaError_t launch_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,

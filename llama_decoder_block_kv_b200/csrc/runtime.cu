@@ -74,6 +74,7 @@ struct llama_ctx {
   unsigned* gbar = nullptr;
   float* ssq = nullptr;
   int decode_mode = LLAMA_DECODE_AUTO;
+  int attn_mode = LLAMA_ATTN_AUTO;
   // generation: last-position logits and sampling scratch, [max_batch][vocab] each;
   // the captured decode step's column counter and positions; its executable graph
   float* gen_logits = nullptr;
@@ -259,6 +260,15 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
   return launch_decode_block(maps, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+// Which decode attention kernel a call runs (both compute the same attention).
+bool use_stream_k(int mode, int B, bool ragged, int max_len) {
+  if (mode != LLAMA_ATTN_AUTO) return mode == LLAMA_ATTN_STREAMK;
+  (void)B;
+  (void)ragged;
+  (void)max_len;
+  return false;
+}
+
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
   Layer& Ly = c->layers[layer];
   const int M = B * T;
@@ -293,11 +303,19 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
                                    c->S, st);
   } else if (T == 1) {
     const int max_len = sp_dev ? c->S : sp_host + 1;
-    DecodePlan p = plan_decode(B, c->H, c->Hkv, c->S, max_len, c->num_sms);
-    if (p.part_floats > c->part_floats) return LLAMA_ERR_INVALID_ARGS;
-    if (B * c->Hkv * (c->n_rep / p.hpc) > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H, c->Hkv,
-                            c->D, c->S, p, c->err, st);
+    DecodeSkPlan sk = plan_decode_sk(B, c->H, c->Hkv, c->D, max_len, c->num_sms);
+    if (c->attn_mode == LLAMA_ATTN_STREAMK && !sk.ok) return LLAMA_ERR_INVALID_ARGS;
+    if (sk.ok && use_stream_k(c->attn_mode, B, sp_dev != nullptr, max_len)) {
+      if (sk.part_floats > c->part_floats || sk.units > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
+      ce = launch_attn_decode_sk(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H,
+                                 c->Hkv, c->D, c->S, sk, c->err, st);
+    } else {
+      DecodePlan p = plan_decode(B, c->H, c->Hkv, c->S, max_len, c->num_sms);
+      if (p.part_floats > c->part_floats) return LLAMA_ERR_INVALID_ARGS;
+      if (B * c->Hkv * (c->n_rep / p.hpc) > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
+      ce = launch_attn_decode(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H,
+                              c->Hkv, c->D, c->S, p, c->err, st);
+    }
   } else {
     ce = launch_attn_prefill_tc(Ly.map_k, Ly.map_v, c->q, c->o, sp_dev, sp_host, B, T, c->H, c->Hkv, c->D, c->S,
                                 c->err, st);
@@ -487,6 +505,10 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     }
     const size_t dec = (size_t)c->Bm * c->H * ((c->S + 127) / 128) * (128 + 2);
     if (dec > need) need = dec;
+    for (int b = 1; b <= c->Bm; ++b) {  // the stream-K decode attention's partials
+      DecodeSkPlan sk = plan_decode_sk(b, c->H, c->Hkv, D, c->S, c->num_sms);
+      if (sk.ok && sk.part_floats > need) need = sk.part_floats;
+    }
     // the persistent decode kernel, for every batch it serves
     for (int m = 1; m <= c->Bm && m <= 32; ++m) {
       DecodeBlockPlan pl = plan_decode_block(m, c->dim, c->H, c->Hkv, D, F, c->S, c->S, c->num_sms);
@@ -780,6 +802,12 @@ int llama_reset(llama_ctx* c) {
   return LLAMA_OK;
 }
 
+int llama_set_decode_attention(llama_ctx* c, int mode) {
+  if (!c || mode < LLAMA_ATTN_AUTO || mode > LLAMA_ATTN_STREAMK) return LLAMA_ERR_INVALID_ARGS;
+  c->attn_mode = mode;
+  return LLAMA_OK;
+}
+
 int llama_set_decode_kernel(llama_ctx* c, int mode) {
   if (!c || mode < LLAMA_DECODE_AUTO || mode > LLAMA_DECODE_PERSISTENT) return LLAMA_ERR_INVALID_ARGS;
   c->decode_mode = mode;
@@ -863,6 +891,29 @@ int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, 
   // the persistent decode kernel, with the workspace a context would hold
   DecodeBlockPlan pl = plan_decode_block(M, dim, n_heads, n_kv_heads, D, ffn, max_seq_len, max_seq_len, num_sms);
   if (pl.ok && !check_decode_block_plan(pl, M, n_heads, pl.part_floats, pl.counters)) return LLAMA_ERR_INTERNAL;
+  // the stream-K decode attention: ragged device positions (planned for max_seq_len) ...
+  std::vector<int> pos(M);
+  const int S = max_seq_len;
+  DecodeSkPlan sk = plan_decode_sk(M, n_heads, n_kv_heads, D, S, num_sms);
+  uint32_t lcg = 12345u + (uint32_t)M;
+  for (int pattern = 0; pattern < 5; ++pattern) {
+    for (int b = 0; b < M; ++b) {
+      lcg = lcg * 1664525u + 1013904223u;
+      pos[b] = pattern == 0 ? S - 1
+             : pattern == 1 ? (int)(((long long)b * 977 + 13) % S)
+             : pattern == 2 ? (b == 0 ? S - 1 : 0)
+             : pattern == 3 ? 0
+                            : (int)((lcg >> 8) % (uint32_t)S);
+    }
+    if (!check_decode_sk(sk, pos.data(), M, n_heads, n_kv_heads, D, S)) return LLAMA_ERR_INTERNAL;
+  }
+  // ... and one position for the whole batch (planned for that length)
+  const int sps[5] = {0, 63, 64, S / 3, S - 1};
+  for (int sp : sps) {
+    DecodeSkPlan p1 = plan_decode_sk(M, n_heads, n_kv_heads, D, sp + 1, num_sms);
+    std::fill(pos.begin(), pos.end(), sp);
+    if (!check_decode_sk(p1, pos.data(), M, n_heads, n_kv_heads, D, S)) return LLAMA_ERR_INTERNAL;
+  }
   return LLAMA_OK;
 }
 

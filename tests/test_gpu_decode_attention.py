@@ -1,0 +1,194 @@
+"""The two decode attention kernels of the per-step launches (LLAMA_ATTN_CHUNKED
+and LLAMA_ATTN_STREAMK) against the oracle: MHA / GQA / MQA head maps, head_dim
+64 and 128, scalar and per-sequence positions, histories split over many CTAs
+(the stream-K split cuts one sequence's tiles over up to 16 CTAs), batches of
+up to 96 sequences, repeated launches through the same counters, CUDA-graph
+replay with device positions, and the mode switch's errors.
+The oracle's block (TransformerBlock.forward of the notes) is the reference;
+the two kernels' outputs are also compared with each other, which bounds a
+difference the block's output would dilute."""
+import numpy as np
+import pytest
+import torch
+
+from llama_decoder_block_kv_b200 import binding as B
+from llama_decoder_block_kv_b200 import synth
+from tests.gpu_util import BF16_HIDDEN_ABS, Pair, assert_abs_close, assert_cache_matches
+from tests.helpers import t2np
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [B.LLAMA_ATTN_CHUNKED, B.LLAMA_ATTN_STREAMK]
+
+
+def _wl(dim, H, Hkv, Bm, S=256, mo=256, seed=23):
+    F = O.ffn_hidden_dim(dim, mo)
+    return synth.Workload(name=f"decode attention dim {dim} H {H}/{Hkv}", dim=dim, n_layers=1, n_heads=H,
+                          n_kv_heads=Hkv, ffn_hidden=F, vocab_size=0, multiple_of=mo, ffn_dim_multiplier=None,
+                          norm_eps=1e-5, rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act="bf16", batch=Bm,
+                          seed=seed)
+
+
+def _run(pair, h, start_pos):
+    hd = h.to("cuda").contiguous()
+    sp = start_pos
+    if isinstance(start_pos, np.ndarray):
+        sp = torch.from_numpy(start_pos.astype(np.int32)).to("cuda")
+    B.llama_block_forward(pair.ctx, 0, hd, sp)
+    torch.cuda.synchronize()
+    pair.check_error()
+    return t2np(hd)
+
+
+def _step(pair, h, start_pos):
+    """One call through the library and the oracle (which keeps its own cache)."""
+    ref = pair.oracle.block(0, t2np(h), start_pos)
+    got = _run(pair, h, start_pos)
+    assert_abs_close(got, ref, BF16_HIDDEN_ABS, "call")
+    return got
+
+
+def _decode_both(pair, h, start_pos):
+    """One decode step through each kernel from the same cache (the step's own
+    slot is rewritten with the same values), each checked against the oracle;
+    returns the two outputs."""
+    ref = pair.oracle.block(0, t2np(h), start_pos)
+    outs = []
+    for k in KERNELS:
+        B.llama_set_decode_attention(pair.ctx, k)
+        got = _run(pair, h, start_pos)
+        assert_abs_close(got, ref, BF16_HIDDEN_ABS, f"kernel {k}")
+        outs.append(got)
+    return outs
+
+
+@pytest.mark.parametrize("dim,H,Hkv,Bsz", [(512, 4, 2, 1), (512, 4, 4, 2), (1024, 8, 1, 3), (2048, 16, 2, 5),
+                                           (1024, 8, 8, 9), (256, 4, 1, 4), (512, 8, 2, 6), (2048, 16, 4, 2)])
+def test_decode_steps_match_oracle(dim, H, Hkv, Bsz):
+    w = _wl(dim, H, Hkv, Bsz)
+    pair = Pair(w)
+    try:
+        h = synth.hidden(w, (Bsz, 70, dim), call=0)
+        _step(pair, h, 0)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:Bsz, :70] = True
+        for i in range(3):
+            h = synth.hidden(w, (Bsz, 1, dim), call=1 + i)
+            a, b = _decode_both(pair, h, 70 + i)
+            assert np.abs(a - b).max() <= BF16_HIDDEN_ABS / 2
+            written[:Bsz, 70 + i] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 1), (1024, 8, 2), (256, 4, 2)])
+def test_long_ragged_histories_split_over_many_ctas(dim, H, Hkv):
+    """Per-sequence device positions, one history of ~3.9k keys next to short
+    ones: the stream-K split gives a unit's tiles to many CTAs whose partials
+    the last of them merges."""
+    w = _wl(dim, H, Hkv, 4, S=4096)
+    pair = Pair(w)
+    try:
+        h = synth.hidden(w, (4, 5, dim), call=0)
+        _step(pair, h, 0)
+        pos = np.array([5, 3900, 130, 1000])   # skipped slots stay zero on both sides
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:4, :5] = True
+        for step in range(3):
+            h = synth.hidden(w, (4, 1, dim), call=1 + step)
+            a, b = _decode_both(pair, h, pos)
+            assert np.abs(a - b).max() <= BF16_HIDDEN_ABS / 2
+            for s in range(4):
+                written[s, pos[s]] = True
+            pos = pos + np.array([1, 64, 63, 129])
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+def test_single_sequence_long_history():
+    """One sequence, one kv head group, 4000 keys: every CTA of the stream-K grid
+    holds a piece of the same unit."""
+    w = _wl(512, 4, 1, 1, S=4096)
+    pair = Pair(w)
+    try:
+        _step(pair, synth.hidden(w, (1, 3, 512), call=0), 0)
+        for step, p in enumerate((3999, 4000, 4095)):
+            h = synth.hidden(w, (1, 1, 512), call=1 + step)
+            _decode_both(pair, h, np.array([p]))
+    finally:
+        pair.close()
+
+
+def test_wide_ragged_batch():
+    """96 sequences with lengths spread over 1 .. 1200 keys."""
+    w = _wl(512, 4, 2, 96, S=1280)
+    pair = Pair(w)
+    try:
+        _step(pair, synth.hidden(w, (96, 2, 512), call=0), 0)
+        rng = np.random.default_rng(5)
+        for step in range(2):
+            pos = rng.integers(2, 1200, size=96)
+            _decode_both(pair, synth.hidden(w, (96, 1, 512), call=1 + step), pos)
+    finally:
+        pair.close()
+
+
+def test_repeated_launches_rearm_counters():
+    """Forty launches through one workspace, alternating the kernels."""
+    w = _wl(512, 4, 2, 3, S=512)
+    pair = Pair(w)
+    try:
+        _step(pair, synth.hidden(w, (3, 200, 512), call=0), 0)
+        for i in range(40):
+            B.llama_set_decode_attention(pair.ctx, KERNELS[(i // 3) % 2])
+            h = synth.hidden(w, (3, 1, 512), call=1 + i)
+            pos = np.array([200 + i, 17 + i, 300 + 2 * i])
+            _step(pair, h, pos)
+    finally:
+        pair.close()
+
+
+def test_graph_replay_with_device_positions():
+    w = _wl(1024, 8, 2, 2, S=256)
+    pair = Pair(w)
+    try:
+        B.llama_set_decode_attention(pair.ctx, B.LLAMA_ATTN_STREAMK)
+        _step(pair, synth.hidden(w, (2, 100, 1024), call=0), 0)
+        _step(pair, synth.hidden(w, (2, 1, 1024), call=9), 100)   # first launch outside the capture
+        pos = torch.tensor([100, 100], dtype=torch.int32, device="cuda")
+        hd = torch.zeros((2, 1, 1024), device="cuda")
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            B.llama_block_forward(pair.ctx, 0, hd, pos, stream=s)
+        torch.cuda.synchronize()
+        for i in range(3):
+            hin = synth.hidden(w, (2, 1, 1024), call=1 + i)
+            hd.copy_(hin.to("cuda"))
+            p = np.array([100 + 30 * i, 101 + 60 * i])
+            pos.copy_(torch.from_numpy(p.astype(np.int32)))
+            g.replay()
+            torch.cuda.synchronize()
+            pair.check_error()
+            ref = pair.oracle.block(0, t2np(hin), p)
+            assert_abs_close(t2np(hd), ref, BF16_HIDDEN_ABS, f"replay {i}")
+        del g
+    finally:
+        pair.close()
+
+
+def test_mode_errors():
+    w = _wl(512, 4, 2, 2, S=64)
+    pair = Pair(w)
+    try:
+        with pytest.raises(B.LlamaError):
+            B.llama_set_decode_attention(pair.ctx, 3)
+        B.llama_set_decode_attention(pair.ctx, B.LLAMA_ATTN_AUTO)
+        _step(pair, synth.hidden(w, (2, 4, 512), call=0), 0)
+        _step(pair, synth.hidden(w, (2, 1, 512), call=1), 4)
+    finally:
+        pair.close()

@@ -49,3 +49,12 @@ def test_plans_of_random_shapes_and_grids():
 def test_selfcheck_rejects_bad_sizes():
     assert B.llama_selfcheck_plans(0, 4096, 32, 32, 11008, 2048, 148) == B.LLAMA_ERR_INVALID_ARGS
     assert B.llama_selfcheck_plans(1, 4096, 32, 3, 11008, 2048, 148) == B.LLAMA_ERR_INVALID_ARGS
+
+
+@pytest.mark.parametrize("M", [33, 96, 255, 1024])
+def test_stream_k_attention_split_of_wide_batches(M):
+    """The decode attention's stream-K split (walked inside llama_selfcheck_plans
+    at ragged and uniform positions) for batches past the GEMV range."""
+    for dim, H, Hkv, S in ((4096, 32, 8, 2048), (512, 4, 2, 1280), (2048, 32, 1, 512)):
+        for sms in (148, 7):
+            assert B.llama_selfcheck_plans(M, dim, H, Hkv, 1024, S, sms) == B.LLAMA_OK, (M, dim, H, Hkv, sms)
