@@ -80,7 +80,7 @@ extern "C" {
 #define LLAMA_DECODE_PERSISTENT 2 /* always the persistent launch; an ineligible decode call fails */
 
 /* Decode attention kernel of the per-step launches, llama_set_decode_attention */
-#define LLAMA_ATTN_AUTO 0    /* the library's choice by shape */
+#define LLAMA_ATTN_AUTO 0    /* the library's choice by size (see llama_set_decode_attention) */
 #define LLAMA_ATTN_CHUNKED 1 /* a CTA per (sequence, kv head group, chunk of keys) */
 #define LLAMA_ATTN_STREAMK 2 /* the key tiles of all sequences dealt out evenly over two CTAs per SM */
 
@@ -292,7 +292,9 @@ int llama_set_decode_kernel(llama_ctx* ctx, int mode);
  *   Served when max_batch_size <= 1024 and head_dim is 64 or 128; a decode
  *   call of another shape returns LLAMA_ERR_INVALID_ARGS before any launch.
  *  LLAMA_ATTN_AUTO (the default): the kernel measured faster on B200 for the
- *   call's shape.
+ *   call's size: STREAMK when the units times the 64-key tiles of the longest
+ *   history (max_seq_len for per-sequence positions) reach 8 per SM, else
+ *   CHUNKED.
  * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it
  * applies to calls made after it.
  */

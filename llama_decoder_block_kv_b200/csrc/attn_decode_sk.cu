@@ -78,20 +78,20 @@ __host__ __device__ __forceinline__ SkUnit sk_locate(const int* pb, const int* n
 __host__ __device__ __forceinline__ int sk_part_stride(int hpc, int D) { return hpc * D + ((2 * hpc + 3) & ~3); }
 
 template <int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(160, 2)
     attn_decode_sk_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                           const bf16* __restrict__ q, bf16* __restrict__ o, float* __restrict__ part,
                           int* __restrict__ counters, const int* __restrict__ start_pos, int sp_scalar, int B, int H,
                           int Hkv, int S_max, int hpc, int* err) {
   constexpr uint32_t TB = SKT * D * 2;  // one K or one V tile
   constexpr int HALVES = D / 64;
-  constexpr int DW = D / 4;  // output columns of one warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + SK_STAGES * 2 * TB);
   uint64_t* empty = full + SK_STAGES;
   int* nb = reinterpret_cast<int*>(empty + SK_STAGES);  // [B] tiles per unit of each sequence
   int* pb = nb + B;                                      // [B + 1] prefix sums of nb
+  __shared__ float s_m[64], s_l[64];  // (max, sum) of [4 warps][16 rows] at a segment's merge
   __shared__ int s_last;
   __shared__ int s_abort;
   volatile int* abort_flag = &s_abort;
@@ -184,7 +184,6 @@ __global__ void __launch_bounds__(160, 1)
   pdl_wait();
   pdl_trigger();
   const int g = lane >> 2, qd = lane & 3;
-  const int dw0 = warp * DW;
   const float sl2 = rsqrtf((float)D) * SK_LOG2E;
   const bool rv0 = g < hpc, rv1 = g + 8 < hpc;  // rows g, g + 8 are heads of the group
   int j = 0;
@@ -211,48 +210,44 @@ __global__ void __launch_bounds__(160, 1)
         qa[kk][3] = rv1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
       }
     }
-    float oacc[DW / 8][4];
+    float oacc[D / 8][4];
 #pragma unroll
-    for (int c = 0; c < DW / 8; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
+    for (int c = 0; c < D / 8; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
+    int st = 0;
     for (int i = 0; i < seg_len; ++i, ++j) {
-      const int st = j % SK_STAGES;
+      st = j % SK_STAGES;
       const bool ok = wait_or_abort(&full[st], (j / SK_STAGES) & 1, err, abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
+      const int key0 = (u.t + i) * SKT + 16 * warp;  // first of this warp's 16 keys
+      if (__all_sync(0xffffffffu, ok) && key0 < L) {
         const uint32_t kb = smem_u32(base + st * 2 * TB), vb = kb + TB;
-        const int key0 = (u.t + i) * SKT;
-        // scores of all 64 keys: n-tile n holds keys 8n .. 8n + 7
-        float s[8][4];
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-        for (int kq = 0; kq < 4; ++kq)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int mi = lane >> 3;
-            const int key = 16 * kq + 8 * (mi >> 1) + (lane & 7);
-            const int d = 16 * kk + 8 * (mi & 1);
-            uint32_t bf[4];
-            ldmatrix_x4(bf, sk_sw(kb + (d >> 6) * 8192, key, d & 63));
-            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-            mma_bf16_16816(s[2 * kq], qa[kk], b0);
-            mma_bf16_16816(s[2 * kq + 1], qa[kk], b1);
-          }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int mi = lane >> 3;
+          const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+          const int d = 16 * kk + 8 * (mi & 1);
+          uint32_t bf[4];
+          ldmatrix_x4(bf, sk_sw(kb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(s[0], qa[kk], b0);
+          mma_bf16_16816(s[1], qa[kk], b1);
+        }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int n = 0; n < 8; ++n)
+        for (int jn = 0; jn < 2; ++jn)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float v = s[n][e] * sl2;
-            if (key0 + 8 * n + 2 * qd + (e & 1) >= L) v = -INFINITY;
-            s[n][e] = v;
+            float v = s[jn][e] * sl2;
+            if (key0 + 8 * jn + 2 * qd + (e & 1) >= L) v = -INFINITY;
+            s[jn][e] = v;
             if (e < 2)
               mx0 = fmaxf(mx0, v);
             else
               mx1 = fmaxf(mx1, v);
           }
-        // key0 < L, so every tile holds a valid key and the maxima are finite
+        // key0 < L: the maxima are finite
         const float mn0 = fmaxf(m0, sk_quad_max(mx0)), mn1 = fmaxf(m1, sk_quad_max(mx1));
         const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
         m0 = mn0;
@@ -260,80 +255,98 @@ __global__ void __launch_bounds__(160, 1)
         l0 *= sc0;
         l1 *= sc1;
 #pragma unroll
-        for (int c = 0; c < DW / 8; ++c) {
+        for (int c = 0; c < D / 8; ++c) {
           oacc[c][0] *= sc0;
           oacc[c][1] *= sc0;
           oacc[c][2] *= sc1;
           oacc[c][3] *= sc1;
         }
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          s[n][0] = exp2f(s[n][0] - mn0);
-          s[n][1] = exp2f(s[n][1] - mn0);
-          s[n][2] = exp2f(s[n][2] - mn1);
-          s[n][3] = exp2f(s[n][3] - mn1);
-          l0 += s[n][0] + s[n][1];
-          l1 += s[n][2] + s[n][3];
+        for (int jn = 0; jn < 2; ++jn) {
+          s[jn][0] = exp2f(s[jn][0] - mn0);
+          s[jn][1] = exp2f(s[jn][1] - mn0);
+          s[jn][2] = exp2f(s[jn][2] - mn1);
+          s[jn][3] = exp2f(s[jn][3] - mn1);
+          l0 += s[jn][0] + s[jn][1];
+          l1 += s[jn][2] + s[jn][3];
         }
-        // O[:, this warp's columns] += P V, P as hi + lo bf16 parts, 16 keys per step
+        // O += P V over this warp's 16 keys, P as hi + lo bf16 parts
+        uint32_t ph[4], pl[4];
+        split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
+        split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
+        split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
+        split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t ph[4], pl[4];
-          split_bf16x2(s[2 * ks][0], s[2 * ks][1], ph[0], pl[0]);
-          split_bf16x2(s[2 * ks][2], s[2 * ks][3], ph[1], pl[1]);
-          split_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1], ph[2], pl[2]);
-          split_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3], ph[3], pl[3]);
-#pragma unroll
-          for (int jd = 0; jd < DW / 8; jd += 2) {
-            const int mi = lane >> 3;
-            const int key = 16 * ks + 8 * (mi & 1) + (lane & 7);
-            const int d = dw0 + 8 * (jd + (mi >> 1));
-            uint32_t bf[4];
-            ldmatrix_x4_trans(bf, sk_sw(vb + (d >> 6) * 8192, key, d & 63));
-            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-            mma_bf16_16816(oacc[jd], ph, b0);
-            mma_bf16_16816(oacc[jd], pl, b0);
-            mma_bf16_16816(oacc[jd + 1], ph, b1);
-            mma_bf16_16816(oacc[jd + 1], pl, b1);
-          }
+        for (int jd = 0; jd < D / 8; jd += 2) {
+          const int mi = lane >> 3;
+          const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
+          const int d = 8 * (jd + (mi >> 1));
+          uint32_t bf[4];
+          ldmatrix_x4_trans(bf, sk_sw(vb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(oacc[jd], ph, b0);
+          mma_bf16_16816(oacc[jd], pl, b0);
+          mma_bf16_16816(oacc[jd + 1], ph, b1);
+          mma_bf16_16816(oacc[jd + 1], pl, b1);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if (i + 1 < seg_len) {  // the segment's last stage is released after the merge below
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
     }
     l0 = sk_quad_sum(l0);
     l1 = sk_quad_sum(l1);
 
+    // Merge the four warps' states in the stage of the segment's last tile, which
+    // every warp has finished reading: [4 warps][16 rows][D] floats fill its
+    // 2 x 64 x D bf16 exactly; the (max, sum) pairs go to s_m, s_l.
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float* sm_o = reinterpret_cast<float*>(base + st * 2 * TB);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      *reinterpret_cast<float2*>(sm_o + (warp * 16 + g) * D + 8 * c + 2 * qd) = make_float2(oacc[c][0], oacc[c][1]);
+      *reinterpret_cast<float2*>(sm_o + (warp * 16 + g + 8) * D + 8 * c + 2 * qd) =
+          make_float2(oacc[c][2], oacc[c][3]);
+    }
+    if (qd == 0) {
+      s_m[warp * 16 + g] = m0;
+      s_m[warp * 16 + g + 8] = m1;
+      s_l[warp * 16 + g] = l0;
+      s_l[warp * 16 + g + 8] = l1;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     const uint32_t P = (uint32_t)pb[u.b] * (uint32_t)HG + (uint32_t)u.zl * (uint32_t)n_u;  // the unit's first tile
-    if (u.t == 0 && seg_len == n_u) {
-      // the whole unit is in this range: normalise and store
-      const float i0 = 1.f / l0, i1 = 1.f / l1;
+    const bool whole = u.t == 0 && seg_len == n_u;
+    // Partial state of this CTA for a split unit: slot 2 cta when the unit began
+    // before this range (the range's first segment), else slot 2 cta + 1 (the
+    // unit runs past the range's end: its last segment).
+    float* pp = part + (size_t)(2 * cta + (P <= sbeg ? 0 : 1)) * pstride;
+    for (int e = tid; e < hpc * D; e += 128) {
+      const int r = e / D, d = e - r * D;
+      float mm = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < DW / 8; ++c) {
-        const int col = dw0 + 8 * c + 2 * qd;
-        if (rv0)
-          *reinterpret_cast<uint32_t*>(o + ((size_t)u.b * H + h0 + g) * D + col) =
-              pack_bf16x2(oacc[c][0] * i0, oacc[c][1] * i0);
-        if (rv1)
-          *reinterpret_cast<uint32_t*>(o + ((size_t)u.b * H + h0 + g + 8) * D + col) =
-              pack_bf16x2(oacc[c][2] * i1, oacc[c][3] * i1);
-      }
-    } else {
-      // Partial state of this CTA for the unit: slot 2 cta when the unit began
-      // before this range (the range's first segment), else slot 2 cta + 1
-      // (the unit runs past the range's end: its last segment).
-      float* pp = part + (size_t)(2 * cta + (P <= sbeg ? 0 : 1)) * pstride;
+      for (int w = 0; w < 4; ++w) mm = fmaxf(mm, s_m[w * 16 + r]);
+      float acc = 0.f, ll = 0.f;
 #pragma unroll
-      for (int c = 0; c < DW / 8; ++c) {
-        const int col = dw0 + 8 * c + 2 * qd;
-        if (rv0) __stcg(reinterpret_cast<float2*>(pp + g * D + col), make_float2(oacc[c][0], oacc[c][1]));
-        if (rv1) __stcg(reinterpret_cast<float2*>(pp + (g + 8) * D + col), make_float2(oacc[c][2], oacc[c][3]));
+      for (int w = 0; w < 4; ++w) {
+        const float mw = s_m[w * 16 + r];
+        const float f = mw == -INFINITY ? 0.f : exp2f(mw - mm);  // a warp without valid keys in the segment
+        acc += sm_o[(w * 16 + r) * D + d] * f;
+        ll += s_l[w * 16 + r] * f;
       }
-      if (warp == 0 && qd == 0) {  // every warp holds the same (max, sum)
-        if (rv0) __stcg(reinterpret_cast<float2*>(pp + hpc * D + 2 * g), make_float2(m0, l0));
-        if (rv1) __stcg(reinterpret_cast<float2*>(pp + hpc * D + 2 * (g + 8)), make_float2(m1, l1));
+      if (whole) {  // the whole unit is in this range: normalise and store
+        o[((size_t)u.b * H + h0 + r) * D + d] = __float2bfloat16_rn(acc / ll);
+      } else {
+        __stcg(pp + r * D + d, acc);
+        if (d == 0) __stcg(reinterpret_cast<float2*>(pp + hpc * D + 2 * r), make_float2(mm, ll));
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+    fence_proxy_async_smem();  // these generic writes come before the next TMA write into the stage
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (lane == 0) mbar_arrive(&empty[st]);
+
+    if (!whole) {
       const uint32_t c0 = sk_own(P, W, G), c1 = sk_own(P + n_u - 1, W, G);
       if (tid == 0) s_last = (atomic_add_acq_rel(&counters[z], 1) == (int)(c1 - c0));
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -385,8 +398,8 @@ DecodeSkPlan plan_decode_sk(int B, int H, int Hkv, int D, int max_len, int num_s
   p.hpc = n_rep < 16 ? n_rep : 16;
   const long long HG = (long long)Hkv * (n_rep / p.hpc);
   const long long W_max = (long long)B * HG * ((max_len + SKT - 1) / SKT);
-  // two resident CTAs per SM; at least four tiles per CTA on short histories
-  const long long G = std::min<long long>(2LL * num_sms, std::max<long long>(1, W_max / 4));
+  // two resident CTAs per SM; at least two tiles per CTA on short histories
+  const long long G = std::min<long long>(2LL * num_sms, std::max<long long>(1, W_max / 2));
   p.grid = (int)G;
   p.units = (int)(B * HG);
   p.part_floats = (size_t)2 * p.grid * sk_part_stride(p.hpc, D);

@@ -261,12 +261,16 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
 }
 
 // Which decode attention kernel a call runs (both compute the same attention).
-bool use_stream_k(int mode, int B, bool ragged, int max_len) {
+// AUTO takes the stream-K split once the call can hold at least 8 key tiles per
+// SM (the longest history counted for every unit). Measured on B200: the
+// LLaMA-2-70B layer at batch 16 x 4096 keys runs 0.343 ms per step against
+// 0.360 chunked, the LLaMA-3-8B ragged batch-32 decode 436 ms per 64 steps
+// against 446; a batch-1 LLaMA-7B layer over ~600 keys (about 2 tiles per SM)
+// runs 90.8 us against 89.2 chunked.
+bool use_stream_k(int mode, const DecodeSkPlan& sk, int max_len, int num_sms) {
   if (mode != LLAMA_ATTN_AUTO) return mode == LLAMA_ATTN_STREAMK;
-  (void)B;
-  (void)ragged;
-  (void)max_len;
-  return false;
+  const long long w_max = (long long)sk.units * ((max_len + 63) / 64);
+  return w_max >= 8LL * num_sms;
 }
 
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
@@ -305,7 +309,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
     const int max_len = sp_dev ? c->S : sp_host + 1;
     DecodeSkPlan sk = plan_decode_sk(B, c->H, c->Hkv, c->D, max_len, c->num_sms);
     if (c->attn_mode == LLAMA_ATTN_STREAMK && !sk.ok) return LLAMA_ERR_INVALID_ARGS;
-    if (sk.ok && use_stream_k(c->attn_mode, B, sp_dev != nullptr, max_len)) {
+    if (sk.ok && use_stream_k(c->attn_mode, sk, max_len, c->num_sms)) {
       if (sk.part_floats > c->part_floats || sk.units > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
       ce = launch_attn_decode_sk(Ly.map_k, Ly.map_v, c->q, c->o, c->part, c->counters, sp_dev, sp_host, B, c->H,
                                  c->Hkv, c->D, c->S, sk, c->err, st);
