@@ -15,11 +15,12 @@
 //               3-stage ring (128-byte swizzle, no multicast), crossing
 //               segment edges without pausing; tiles of positions written by
 //               earlier calls are fetched before griddepcontrol.wait;
-//   warps 0..3  every warp computes the scores of all 64 keys of a tile for
-//               the unit's query heads (redundantly: the kernel is bound by
-//               the cache stream) and its own quarter of the head dimension of
-//               P.V, so the warps never merge states; P is split into two bf16
-//               parts for the MMA (~16 bits kept).
+//   warps 0..3  warp w takes keys 16w .. 16w + 15 of every tile on the
+//               warp-level bf16 tensor-core MMA with its own online-softmax
+//               state (max, sum, O over the whole head dimension); P is split
+//               into two bf16 parts for the MMA (~16 bits kept). At the end of
+//               a segment the four states merge in the ring stage of the
+//               segment's last tile, which is released only after the merge.
 // A segment that covers its whole unit writes the output; otherwise it writes
 // an unnormalised partial (max, sum, O) and the CTA that arrives last for the
 // unit merges the partials of its contributing CTAs in CTA order with the
