@@ -24,6 +24,8 @@
 //    scores in shared memory, plain two-pass softmax.
 #include "kernels.cuh"
 
+#include <vector>
+
 namespace llama {
 
 namespace {
@@ -383,7 +385,7 @@ __global__ void attn_simple_kernel(const T* __restrict__ q, const T* __restrict_
 DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sms) {
   DecodePlan p;
   const int n_rep = H / Hkv;
-  p.hpc = n_rep < 16 ? n_rep : 16;
+  p.hpc = decode_heads_per_cta(n_rep);
   const int units = B * Hkv * (n_rep / p.hpc);
   // chunks per unit so that the grid covers the SMs about twice (at least one tile each)
   int want = (2 * num_sms + units - 1) / units;
@@ -395,6 +397,22 @@ DecodePlan plan_decode(int B, int H, int Hkv, int S_max, int max_len, int num_sm
   p.max_chunks = (S_max + ck - 1) / ck;
   p.part_floats = (size_t)B * H * p.max_chunks * 128 + (size_t)B * H * p.max_chunks * 2;
   return p;
+}
+
+bool check_decode_heads(int H, int Hkv, int hpc) {
+  if (Hkv < 1 || H % Hkv || hpc < 1 || hpc > 16) return false;
+  const int n_rep = H / Hkv, groups = n_rep / hpc;
+  std::vector<int> seen(H, 0);
+  for (int kvh = 0; kvh < Hkv; ++kvh)
+    for (int grp = 0; grp < groups; ++grp)
+      for (int r = 0; r < hpc; ++r) {  // the kernels' head index h0 + r
+        const int h = kvh * n_rep + grp * hpc + r;
+        if (h < 0 || h >= H || h / n_rep != kvh) return false;
+        ++seen[h];
+      }
+  for (int v : seen)
+    if (v != 1) return false;
+  return true;
 }
 
 template <int D>

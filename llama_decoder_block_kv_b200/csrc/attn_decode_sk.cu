@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(160, 2)
 DecodeSkPlan plan_decode_sk(int B, int H, int Hkv, int D, int max_len, int num_sms) {
   DecodeSkPlan p;
   const int n_rep = H / Hkv;
-  p.hpc = n_rep < 16 ? n_rep : 16;
+  p.hpc = decode_heads_per_cta(n_rep);
   const long long HG = (long long)Hkv * (n_rep / p.hpc);
   const long long W_max = (long long)B * HG * ((max_len + SKT - 1) / SKT);
   // two resident CTAs per SM; at least two tiles per CTA on short histories
@@ -438,6 +438,7 @@ cudaError_t launch_attn_decode_sk(const CUtensorMap& mk, const CUtensorMap& mv, 
 // no slot used twice or outside the plan's workspace.
 bool check_decode_sk(const DecodeSkPlan& p, const int* start_pos, int B, int H, int Hkv, int D, int S_max) {
   if (!p.ok) return true;  // the kernel is not used for this shape
+  if (!check_decode_heads(H, Hkv, p.hpc)) return false;
   const int n_rep = H / Hkv, HG = Hkv * (n_rep / p.hpc);
   std::vector<int> nb(B), pb(B + 1);
   int acc = 0;

@@ -82,6 +82,14 @@ bool make_tmap_weights(CUtensorMap* map, const void* ptr, int tiled, uint64_t N,
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
                            int num_sms, cudaStream_t st);
 
+// Query heads one decode-attention CTA serves (one kv head's group of n_rep
+// query heads, split into n_rep / hpc groups; an MMA row block holds 16): all of
+// them up to 16, else 16 or 8, whichever divides n_rep (bf16 contexts have
+// n_rep <= 8 or n_rep % 8 == 0).
+inline int decode_heads_per_cta(int n_rep) { return n_rep <= 16 ? n_rep : (n_rep % 16 == 0 ? 16 : 8); }
+// Every query head of every kv head in exactly one group of the split above.
+bool check_decode_heads(int H, int Hkv, int hpc);
+
 // attention.cu
 struct DecodePlan {
   int hpc = 1, CK = 256, max_chunks = 1;

@@ -882,6 +882,7 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
 
 int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, int max_seq_len, int num_sms) {
   if (M < 1 || dim < 64 || n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || dim % n_heads || ffn < 64 ||
+      (n_heads / n_kv_heads > 8 && (n_heads / n_kv_heads) % 8) ||
       max_seq_len < 1 || num_sms < 1 || dim % 64 || ffn % 64)
     return LLAMA_ERR_INVALID_ARGS;
   const int D = dim / n_heads, n_qkv = (n_heads + 2 * n_kv_heads) * D;
@@ -895,6 +896,9 @@ int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, 
   // the persistent decode kernel, with the workspace a context would hold
   DecodeBlockPlan pl = plan_decode_block(M, dim, n_heads, n_kv_heads, D, ffn, max_seq_len, max_seq_len, num_sms);
   if (pl.ok && !check_decode_block_plan(pl, M, n_heads, pl.part_floats, pl.counters)) return LLAMA_ERR_INTERNAL;
+  // the chunked decode attention's head groups
+  if (!check_decode_heads(n_heads, n_kv_heads, plan_decode(M, n_heads, n_kv_heads, max_seq_len, max_seq_len, num_sms).hpc))
+    return LLAMA_ERR_INTERNAL;
   // the stream-K decode attention: ragged device positions (planned for max_seq_len) ...
   std::vector<int> pos(M);
   const int S = max_seq_len;

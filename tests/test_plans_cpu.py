@@ -58,3 +58,17 @@ def test_stream_k_attention_split_of_wide_batches(M):
     for dim, H, Hkv, S in ((4096, 32, 8, 2048), (512, 4, 2, 1280), (2048, 32, 1, 512)):
         for sms in (148, 7):
             assert B.llama_selfcheck_plans(M, dim, H, Hkv, 1024, S, sms) == B.LLAMA_OK, (M, dim, H, Hkv, sms)
+
+
+@pytest.mark.parametrize("H,Hkv", [(24, 1), (48, 2), (40, 1), (56, 7), (64, 2), (16, 1), (12, 3), (6, 2)])
+def test_decode_attention_head_groups_cover_every_head(H, Hkv):
+    """More than 16 query heads per kv head, not a multiple of 16 (groups of 8),
+    next to the usual ratios: every query head in exactly one group of both
+    decode attention kernels (checked inside llama_selfcheck_plans)."""
+    for D in (64, 128):
+        for M in (1, 7, 32):
+            assert B.llama_selfcheck_plans(M, H * D, H, Hkv, 1024, 2048, 148) == B.LLAMA_OK, (H, Hkv, D, M)
+
+
+def test_selfcheck_rejects_head_ratios_the_library_rejects():
+    assert B.llama_selfcheck_plans(1, 20 * 64, 20, 1, 1024, 256, 148) == B.LLAMA_ERR_INVALID_ARGS  # n_rep 20
