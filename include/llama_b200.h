@@ -293,8 +293,9 @@ int llama_set_decode_kernel(llama_ctx* ctx, int mode);
  *   call of another shape returns LLAMA_ERR_INVALID_ARGS before any launch.
  *  LLAMA_ATTN_AUTO (the default): the kernel measured faster on B200 for the
  *   call's size: STREAMK when the units times the 64-key tiles of the longest
- *   history (max_seq_len for per-sequence positions) reach 8 per SM, else
- *   CHUNKED.
+ *   history (max_seq_len for per-sequence positions) reach 8 per SM and a CTA
+ *   serves at most 8 query heads (n_rep <= 8, or a multiple of 8 that is not
+ *   a multiple of 16), else CHUNKED.
  * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it
  * applies to calls made after it.
  */

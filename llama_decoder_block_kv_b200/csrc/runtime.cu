@@ -266,11 +266,12 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
 // LLaMA-2-70B layer at batch 16 x 4096 keys runs 0.343 ms per step against
 // 0.360 chunked, the LLaMA-3-8B ragged batch-32 decode 436 ms per 64 steps
 // against 446; a batch-1 LLaMA-7B layer over ~600 keys (about 2 tiles per SM)
-// runs 90.8 us against 89.2 chunked.
+// runs 90.8 us against 89.2 chunked. AUTO keeps groups of up to 8 query heads
+// per CTA (the configurations timed above); 16 runs when chosen explicitly.
 bool use_stream_k(int mode, const DecodeSkPlan& sk, int max_len, int num_sms) {
   if (mode != LLAMA_ATTN_AUTO) return mode == LLAMA_ATTN_STREAMK;
   const long long w_max = (long long)sk.units * ((max_len + 63) / 64);
-  return w_max >= 8LL * num_sms;
+  return sk.hpc <= 8 && w_max >= 8LL * num_sms;
 }
 
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
