@@ -4,7 +4,8 @@
   python -m llama_decoder_block_kv_b200.profile_case tc   M N K [--reps R]
   python -m llama_decoder_block_kv_b200.profile_case simt M N K [--reps R]
   python -m llama_decoder_block_kv_b200.profile_case prefill-attn T   (LLaMA-7B layer shape, one block call)
-  python -m llama_decoder_block_kv_b200.profile_case decode-attn B L  (LLaMA-2-70B layer shape, one block call)
+  python -m llama_decoder_block_kv_b200.profile_case decode-attn B L [--decode-attention chunked|streamk|auto]
+                                                     (LLaMA-2-70B layer shape, one block call)
 
 GEMM cases call llama_linear on seeded bf16 inputs; the block cases call
 llama_block_forward. Prints the mean CUDA-event time per launch.
@@ -25,6 +26,8 @@ def main():
     ap.add_argument("sizes", type=int, nargs="+")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--graph", action="store_true", help="time the launches inside one CUDA graph")
+    ap.add_argument("--decode-attention", default="auto", choices=["auto", "chunked", "streamk"],
+                    help="decode-attn: the attention kernel of the call (llama_set_decode_attention)")
     ap.add_argument("--row-major", action="store_true",
                     help="gemv / tc: pass the weights row-major instead of in the library's tile layout")
     a = ap.parse_args()
@@ -79,6 +82,8 @@ def main():
         w = synth.LLAMA70B_LAYER
         Bsz, L = a.sizes
         m = B.Llama(B.ModelArgs.from_workload(w.with_(max_batch_size=Bsz)))
+        B.llama_set_decode_attention(m.ctx, {"auto": B.LLAMA_ATTN_AUTO, "chunked": B.LLAMA_ATTN_CHUNKED,
+                                             "streamk": B.LLAMA_ATTN_STREAMK}[a.decode_attention])
         B.llama_set_layer(m.ctx, 0, synth.layer_weights(w, 0, device="cuda"))
         h0 = synth.hidden(w, (Bsz, 1, w.dim), 0, "cuda")
         pos = L
