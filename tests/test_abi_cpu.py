@@ -30,6 +30,16 @@ def test_library_exports_every_declared_symbol():
     assert set(declared) == set(B.EXPORTED)
 
 
+def test_binding_constants_equal_the_header_defines():
+    """Every integer #define LLAMA_* of the header has the same value in the binding."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    defines = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+(LLAMA_[A-Z0-9_]+)\s+(-?\d+)\b", src)}
+    assert len(defines) >= 20
+    for name, value in defines.items():
+        assert hasattr(B, name), name
+        assert getattr(B, name) == value, (name, getattr(B, name), value)
+
+
 def test_ffn_hidden_matches_oracle_rule():
     if not os.path.exists(B.LIB_PATH):
         pytest.skip("library not built")
