@@ -4,16 +4,20 @@ heads per kv head: one CTA group of 16; 24 at head_dim 64: three groups of 8), h
 (the stream-K split cuts one sequence's tiles over up to 16 CTAs), batches of
 up to 96 sequences, repeated launches through the same counters, CUDA-graph
 replay with device positions, and the mode switch's errors.
-The oracle's block (TransformerBlock.forward of the notes) is the reference;
-the two kernels' outputs are also compared with each other, which bounds a
-difference the block's output would dilute."""
+The oracle's block (TransformerBlock.forward of the notes) is the reference,
+with the bound of the full-size tests: max(2e-2, 3 x the oracle's own response
+to a 2^-17 relative perturbation of the input), which is never tighter than the
+flat 2e-2 and widens it only where the oracle itself moves by more. The two
+kernels' outputs are also compared with each other (half that bound), which
+bounds a difference the block's output would dilute."""
 import numpy as np
 import pytest
 import torch
 
 from llama_decoder_block_kv_b200 import binding as B
 from llama_decoder_block_kv_b200 import synth
-from tests.gpu_util import BF16_HIDDEN_ABS, Pair, assert_abs_close, assert_cache_matches
+from tests.gpu_util import (BF16_HIDDEN_ABS, FLOOR_FACTOR, CacheSnapshot, Pair, assert_abs_close,
+                            assert_cache_matches, assert_hidden_close_floor, oracle_floor)
 from tests.helpers import t2np
 import oracle as O
 
@@ -41,25 +45,38 @@ def _run(pair, h, start_pos):
     return t2np(hd)
 
 
+def _oracle(pair, h, start_pos):
+    """The oracle's output for this call and its conditioning floor; the oracle's
+    cache ends in the unperturbed state."""
+    snap = CacheSnapshot(pair.oracle, [0])
+
+    def run(x):
+        snap.restore()
+        return pair.oracle.block(0, x, start_pos)
+    return oracle_floor(run, t2np(h))
+
+
 def _step(pair, h, start_pos):
     """One call through the library and the oracle (which keeps its own cache)."""
-    ref = pair.oracle.block(0, t2np(h), start_pos)
+    ref, floor = _oracle(pair, h, start_pos)
     got = _run(pair, h, start_pos)
-    assert_abs_close(got, ref, BF16_HIDDEN_ABS, "call")
+    assert_hidden_close_floor(got, ref, floor, "call")
     return got
 
 
 def _decode_both(pair, h, start_pos):
     """One decode step through each kernel from the same cache (the step's own
     slot is rewritten with the same values), each checked against the oracle;
-    returns the two outputs."""
-    ref = pair.oracle.block(0, t2np(h), start_pos)
+    compares the two outputs with each other."""
+    ref, floor = _oracle(pair, h, start_pos)
     outs = []
     for k in KERNELS:
         B.llama_set_decode_attention(pair.ctx, k)
         got = _run(pair, h, start_pos)
-        assert_abs_close(got, ref, BF16_HIDDEN_ABS, f"kernel {k}")
+        assert_hidden_close_floor(got, ref, floor, f"kernel {k}")
         outs.append(got)
+    diff = np.abs(outs[0] - outs[1]).max()
+    assert diff <= max(BF16_HIDDEN_ABS, FLOOR_FACTOR * float(floor.max())) / 2, f"kernels differ by {diff:.4g}"
     return outs
 
 
@@ -76,8 +93,7 @@ def test_decode_steps_match_oracle(dim, H, Hkv, Bsz):
         written[:Bsz, :70] = True
         for i in range(3):
             h = synth.hidden(w, (Bsz, 1, dim), call=1 + i)
-            a, b = _decode_both(pair, h, 70 + i)
-            assert np.abs(a - b).max() <= BF16_HIDDEN_ABS / 2
+            _decode_both(pair, h, 70 + i)
             written[:Bsz, 70 + i] = True
         assert_cache_matches(pair, 0, written, 2e-2)
     finally:
@@ -99,8 +115,7 @@ def test_long_ragged_histories_split_over_many_ctas(dim, H, Hkv):
         written[:4, :5] = True
         for step in range(3):
             h = synth.hidden(w, (4, 1, dim), call=1 + step)
-            a, b = _decode_both(pair, h, pos)
-            assert np.abs(a - b).max() <= BF16_HIDDEN_ABS / 2
+            _decode_both(pair, h, pos)
             for s in range(4):
                 written[s, pos[s]] = True
             pos = pos + np.array([1, 64, 63, 129])
