@@ -8,7 +8,9 @@
 //
 // One CTA owns 128 query rows of one (sequence, kv head): hpc query heads of
 // that group x 128/hpc consecutive positions (row r = position r / hpc, head
-// r % hpc), so every K/V tile is loaded once for the group.
+// r % hpc), so every K/V tile is loaded once for those heads. hpc is the
+// largest power of two (at most 8) dividing n_rep, so the rows hold whole
+// positions and a kv head's n_rep query heads take n_rep / hpc CTAs.
 //   warp 0      TMA: the Q tile once (a 3-D box over [token][head][d]), then
 //               64-key K and V tiles of the cache into a 3-stage ring;
 //   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of two
@@ -367,7 +369,7 @@ template <int D>
 static cudaError_t prefill_tc_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
                                 int sp_scalar, int B, int T, int H, int Hkv, int S_max, int* err, cudaStream_t st) {
   const int n_rep = H / Hkv;
-  const int hpc = n_rep < 8 ? n_rep : 8;
+  const int hpc = prefill_heads_per_cta(n_rep);
   const int BQ = 128 / hpc;
   CUtensorMap mq;
   if (!make_q_map(&mq, q, B * T, H, D, hpc)) return cudaErrorInvalidValue;

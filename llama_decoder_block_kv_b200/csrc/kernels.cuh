@@ -87,6 +87,14 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int
 // them up to 16, else 16 or 8, whichever divides n_rep (bf16 contexts have
 // n_rep <= 8 or n_rep % 8 == 0).
 inline int decode_heads_per_cta(int n_rep) { return n_rep <= 16 ? n_rep : (n_rep % 16 == 0 ? 16 : 8); }
+// Query heads one prefill-attention CTA serves: its 128 MMA rows hold 128 / hpc
+// positions x hpc heads, so hpc must divide 128 as well as n_rep: the largest
+// power of two dividing n_rep, at most 8 (n_rep 6 -> 2, n_rep 3, 5, 7 -> 1).
+inline int prefill_heads_per_cta(int n_rep) {
+  int hpc = 1;
+  while (hpc < 8 && n_rep % (2 * hpc) == 0) hpc *= 2;
+  return hpc;
+}
 // Every query head of every kv head in exactly one group of the split above.
 bool check_decode_heads(int H, int Hkv, int hpc);
 

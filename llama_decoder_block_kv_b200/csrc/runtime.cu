@@ -897,6 +897,11 @@ int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, 
   // the persistent decode kernel, with the workspace a context would hold
   DecodeBlockPlan pl = plan_decode_block(M, dim, n_heads, n_kv_heads, D, ffn, max_seq_len, max_seq_len, num_sms);
   if (pl.ok && !check_decode_block_plan(pl, M, n_heads, pl.part_floats, pl.counters)) return LLAMA_ERR_INTERNAL;
+  // the prefill attention's head groups: whole heads, and 128 rows of whole positions
+  {
+    const int hp = prefill_heads_per_cta(n_heads / n_kv_heads);
+    if (128 % hp || !check_decode_heads(n_heads, n_kv_heads, hp)) return LLAMA_ERR_INTERNAL;
+  }
   // the chunked decode attention's head groups
   if (!check_decode_heads(n_heads, n_kv_heads, plan_decode(M, n_heads, n_kv_heads, max_seq_len, max_seq_len, num_sms).hpc))
     return LLAMA_ERR_INTERNAL;

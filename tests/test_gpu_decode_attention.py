@@ -1,6 +1,7 @@
 """The two decode attention kernels of the per-step launches (LLAMA_ATTN_CHUNKED
 and LLAMA_ATTN_STREAMK) against the oracle: MHA / GQA / MQA head maps (16 query
-heads per kv head: one CTA group of 16; 24 at head_dim 64: three groups of 8), head_dim 64 and 128, scalar and per-sequence positions, histories split over many CTAs
+heads per kv head: one CTA group of 16; 24 at head_dim 64: three groups of 8;
+3 and 6, where the prefill attention takes groups of 1 and 2), head_dim 64 and 128, scalar and per-sequence positions, histories split over many CTAs
 (the stream-K split cuts one sequence's tiles over up to 16 CTAs), batches of
 up to 96 sequences, repeated launches through the same counters, CUDA-graph
 replay with device positions, and the mode switch's errors.
@@ -82,7 +83,7 @@ def _decode_both(pair, h, start_pos):
 
 @pytest.mark.parametrize("dim,H,Hkv,Bsz", [(512, 4, 2, 1), (512, 4, 4, 2), (1024, 8, 1, 3), (2048, 16, 2, 5),
                                            (1024, 8, 8, 9), (256, 4, 1, 4), (512, 8, 2, 6), (2048, 16, 4, 2),
-                                           (1536, 24, 1, 2), (2048, 16, 1, 3)])
+                                           (1536, 24, 1, 2), (2048, 16, 1, 3), (768, 6, 2, 2), (768, 12, 2, 3)])
 def test_decode_steps_match_oracle(dim, H, Hkv, Bsz):
     w = _wl(dim, H, Hkv, Bsz)
     pair = Pair(w)

@@ -72,3 +72,12 @@ def test_decode_attention_head_groups_cover_every_head(H, Hkv):
 
 def test_selfcheck_rejects_head_ratios_the_library_rejects():
     assert B.llama_selfcheck_plans(1, 20 * 64, 20, 1, 1024, 256, 148) == B.LLAMA_ERR_INVALID_ARGS  # n_rep 20
+
+
+@pytest.mark.parametrize("H,Hkv", [(3, 1), (5, 1), (6, 1), (7, 1), (12, 4), (24, 8), (30, 5), (48, 6)])
+def test_head_groups_of_every_ratio_up_to_eight(H, Hkv):
+    """Ratios of 3, 5, 6 and 7 query heads per kv head: the prefill attention's
+    128 MMA rows must hold whole positions (heads per CTA dividing 128) and
+    every head must fall in exactly one group of each attention kernel."""
+    for D in (64, 128):
+        assert B.llama_selfcheck_plans(4, H * D, H, Hkv, 1024, 512, 148) == B.LLAMA_OK, (H, Hkv, D)
