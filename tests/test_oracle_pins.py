@@ -194,6 +194,52 @@ def test_rmsnorm_unit_weight_closed_form_and_scale_invariance():
     np.testing.assert_array_equal(yb, O.bf16_round(y))
 
 
+def _golden_fields(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if line:
+                out[line[0]] = np.array([float(v) for v in line[1:]])
+    return out
+
+
+def test_rmsnorm_bf16_weight_after_cast_back_golden():
+    """The notes' RMSNorm.forward casts the normalised row back, then multiplies by
+    the weight in the activation type; the HuggingFace order (weight first, one
+    cast) gives a different bf16 result on the hand-worked row of the golden file."""
+    g = _golden_fields("rmsnorm_bf16_order.txt")
+    eps = float(g["eps"][0])
+    got = O.rmsnorm(g["h"][None], g["w"], eps, O.ACT_BF16)[0]
+    np.testing.assert_array_equal(got, g["bf16_notes_order"])
+    assert np.all(got != g["bf16_hf_order"])
+    np.testing.assert_allclose(O.rmsnorm(g["h"][None], g["w"], eps, O.ACT_FP32)[0], g["fp32"], rtol=1e-8)
+
+
+def test_rmsnorm_bf16_non_unit_weight_rounding_points():
+    """bf16 mode with non-unit weights: every output is a bf16 value, equals the
+    (rounded) product of a bf16 value and the weight, and the weight is applied
+    per column (a row of equal inputs reproduces the weight vector's pattern)."""
+    rng = np.random.default_rng(9)
+    dim = 512
+    w = O.bf16_round(1.0 + 0.1 * rng.standard_normal(dim))
+    x = rng.standard_normal((6, dim)) * 2.0
+    y = O.rmsnorm(x, w, 1e-5, O.ACT_BF16)
+    np.testing.assert_array_equal(y, O.bf16_round(y))
+    # a constant row normalises to 1 (up to eps) in every column: the output is bf16(w)
+    c = O.rmsnorm(np.full((1, dim), 3.0), w, 0.0, O.ACT_BF16)[0]
+    np.testing.assert_array_equal(c, w)
+    # the result differs from the weight-first (one-rounding) order somewhere on random data
+    yhf = O.bf16_round(x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-5) * w)
+    assert np.any(y != yhf)
+    # a permuted weight vector permutes nothing else: swapping two columns of x and w swaps the output
+    xs, ws = x.copy(), w.copy()
+    xs[:, [3, 77]] = xs[:, [77, 3]]
+    ws[[3, 77]] = ws[[77, 3]]
+    ys = O.rmsnorm(xs, ws, 1e-5, O.ACT_BF16)
+    np.testing.assert_array_equal(ys[:, [3, 77]], y[:, [77, 3]])
+
+
 def test_silu_identities_and_library():
     a = np.linspace(-30, 30, 601)
     s = O.silu(a)
