@@ -8,6 +8,13 @@ through llama_block_forward. The 128 decode steps of a pass are captured in
 one CUDA graph together with the prefill; the graph also restores the step's
 inputs first, so every step does identical work. Prints one JSON line.
 
+At one GPU the line also carries a "configs" object with the other
+workloads (the tiny fp32 model, the LLaMA-2-70B-shaped layer decode, the
+LLaMA-3-8B-shaped ragged decode and 4 x 8192 prefill), each with its
+device-timed throughput, clocks, the roofline of its dominant kernel, an
+end-to-end number with host buffers and the oracle's CPU baseline on a
+stated sample (--configs none skips them).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload llama7b-layer|llama70b-layer|llama3-8b-decode|llama3-8b-prefill]
 
@@ -275,14 +282,7 @@ class LayerBench:
 
     def decode_gemms(self):
         """(x, w) pairs of the decode linears, same shapes and kernel as the decode path."""
-        lw, w = self.lw, self.w
-        M = self.Bsz
-        wqkv = torch.cat([lw["wq"], lw["wk"], lw["wv"]], 0).contiguous()
-        w13 = torch.stack([lw["w1"], lw["w3"]], 1).reshape(2 * w.ffn_hidden, w.dim).contiguous()
-        xs = {K: synth.normal((M, K), 1.0, 7 + K, torch.bfloat16, "cuda") for K in (w.dim, w.ffn_hidden,
-                                                                                  w.n_heads * w.head_dim)}
-        return [(xs[w.dim], wqkv), (xs[w.n_heads * w.head_dim], lw["wo"]), (xs[w.dim], w13),
-                (xs[w.ffn_hidden], lw["w2"])]
+        return layer_pairs(self.w, self.Bsz)
 
     def close(self):
         self.model.close()
@@ -310,17 +310,21 @@ def time_graph(g, steps, warmup, world):
 GEMV_TRAFFIC_RATIO = (180.45e6 + 3.53e6) / (22016 * 4096 * 2 + 4096 * 2 + 22016 * 4)
 
 
-def gemv_roofline(lb: LayerBench, peaks, reps=10):
-    """Average bandwidth of the decode GEMV kernel: the layer's four decode linears
-    (wqkv, wo, w1|w3, w2: 405 MB together, larger than L2) launched back to back
-    `reps` times inside one CUDA graph, timed with CUDA events around the replay.
-    Algorithmic bytes: weights + activations in + fp32 outputs."""
-    pairs = lb.decode_gemms()
+def linear_roofline(pairs, path, peaks, reps, kernel, bound="hbm", peak_key="hbm_gbs", traffic_ratio=None,
+                    traffic_source=None):
+    """Average rate of one GEMM kernel of the library: the (x, w) pairs (a layer's
+    linears, the weights in the tile layout the library keeps) launched back to
+    back ``reps`` times inside one CUDA graph, timed with CUDA events around the
+    replay on the launching stream. Algorithmic work per launch: for an HBM-bound
+    kernel the weights + activations in + fp32 outputs, for a tensor-bound one
+    2*M*N*K FLOP."""
     ys = [torch.empty((x.shape[0], w.shape[0]), device="cuda") for x, w in pairs]
-    byts = sum(w.numel() * 2 + x.numel() * 2 + x.shape[0] * w.shape[0] * 4 for x, w in pairs)
-    # the weights in the tile layout the library keeps for its own linears
+    if bound == "hbm":
+        work = sum(w.numel() * 2 + x.numel() * 2 + x.shape[0] * w.shape[0] * 4 for x, w in pairs)
+    else:
+        work = sum(2.0 * x.shape[0] * w.shape[0] * x.shape[1] for x, w in pairs)
     tiles = [(x, B.llama_tile_weights(w), w.shape[0]) for x, w in pairs]
-    path = B.LLAMA_PATH_GEMV | B.LLAMA_WEIGHTS_TILED
+    path = path | B.LLAMA_WEIGHTS_TILED
     for (x, wt, n), y in zip(tiles, ys):
         B.llama_linear(x, wt, y, path, n=n)
     torch.cuda.synchronize()
@@ -339,16 +343,43 @@ def gemv_roofline(lb: LayerBench, peaks, reps=10):
     e1.synchronize()
     launches = reps * len(pairs)
     t_ms = e0.elapsed_time(e1) / launches          # average launch duration
-    per_launch = byts / len(pairs)
-    achieved = per_launch / (t_ms * 1e-3) / 1e9
-    traffic = None if GEMV_TRAFFIC_RATIO is None else int(round(GEMV_TRAFFIC_RATIO * per_launch))
-    return {"kernel": "gemv_bf16_kernel (decode linears: wqkv, wo, w1|w3, w2)", "bound": "hbm",
-            "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-            "traffic_source": "ncu dram read+write of the w1|w3 launch scaled by algorithmic bytes "
-                              "(M=1, N=22016, K=4096)",
-            "bytes_per_launch": int(per_launch), "avg_launch_us": round(t_ms * 1e3, 2),
-            "launches_timed": launches}
+    per_launch = work / len(pairs)
+    if bound == "hbm":
+        achieved, unit = per_launch / (t_ms * 1e-3) / 1e9, "GB/s"
+    else:
+        achieved, unit = per_launch / (t_ms * 1e-3) / 1e12, "TFLOP/s"
+    peak = peaks[peak_key]
+    out = {"kernel": kernel, "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+           "frac": round(achieved / peak, 4),
+           "traffic": None if traffic_ratio is None else int(round(traffic_ratio * per_launch)),
+           ("bytes_per_launch" if bound == "hbm" else "flop_per_launch"): int(per_launch),
+           "avg_launch_us": round(t_ms * 1e3, 2), "launches_timed": launches, "peak_key": peak_key}
+    if traffic_source:
+        out["traffic_source"] = traffic_source
+    del g
+    return out
+
+
+def gemv_roofline(lb: "LayerBench", peaks, reps=10):
+    """The decode GEMV over the layer's four decode linears (wqkv, wo, w1|w3, w2),
+    larger than L2 together (405 MB for the LLaMA-7B layer)."""
+    return linear_roofline(lb.decode_gemms(), B.LLAMA_PATH_GEMV, peaks, reps,
+                           "llama_decode_linear_kernel (decode linears: wqkv, wo, w1|w3, w2)",
+                           traffic_ratio=GEMV_TRAFFIC_RATIO,
+                           traffic_source="ncu dram read+write of the w1|w3 launch scaled by algorithmic bytes "
+                                          "(M=1, N=22016, K=4096)")
+
+
+def layer_pairs(w: synth.Workload, M: int, layer: int = 0):
+    """(x, w) pairs of one block's linears as the library packs them: wq|wk|wv,
+    wo, w1|w3 row-interleaved, w2; x seeded N(0, 1) bf16 with M rows."""
+    lw = synth.layer_weights(w, layer, device="cuda")
+    wqkv = torch.cat([lw["wq"], lw["wk"], lw["wv"]], 0).contiguous()
+    w13 = torch.stack([lw["w1"], lw["w3"]], 1).reshape(2 * w.ffn_hidden, w.dim).contiguous()
+    xs = {K: synth.normal((M, K), 1.0, 7 + K, torch.bfloat16, "cuda")
+          for K in (w.dim, w.ffn_hidden, w.n_heads * w.head_dim)}
+    return [(xs[w.dim], wqkv), (xs[w.n_heads * w.head_dim], lw["wo"]), (xs[w.dim], w13),
+            (xs[w.ffn_hidden], lw["w2"])]
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
@@ -394,6 +425,150 @@ def oracle_layer_sample(w: synth.Workload, n_decode: int = 4):
     sample = (f"oracle (numpy float64) on one layer: prefill of {w.prefill_len} tokens timed in full, "
               f"{n_decode} of {w.decode_steps} decode steps timed and extrapolated linearly")
     return total, threads, sample
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def _f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _bits(t):
+    """bf16 tensor -> raw uint16 patterns (the oracle widens them slice by slice)."""
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _oracle_model(w: synth.Workload, n_layers: int, **over):
+    import oracle as O
+    a = O.ModelArgs(dim=w.dim, n_layers=n_layers, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads,
+                    vocab_size=w.vocab_size, multiple_of=w.multiple_of, ffn_dim_multiplier=w.ffn_dim_multiplier,
+                    norm_eps=w.norm_eps, rope_theta=w.rope_theta, max_batch_size=w.max_batch_size,
+                    max_seq_len=w.max_seq_len, act=w.act)
+    for k, v in over.items():
+        setattr(a, k, v)
+    m = O.OracleModel(a)
+    for i in range(n_layers):
+        m.layers[i] = {k: _f64(v) for k, v in synth.layer_weights(w, i, device="cuda").items()}
+    if w.vocab_size:
+        enh = synth.embed_norm_head(w, device="cuda")
+        m.tok_embeddings, m.norm, m.output = _bits(enh["tok_embeddings"]), _f64(enh["norm"]), _bits(enh["output"])
+        if w.act == "fp32":
+            m.tok_embeddings, m.output = _f64(enh["tok_embeddings"]), _f64(enh["output"])
+    return m
+
+
+def oracle_sample(name: str, w: synth.Workload):
+    """The oracle (numpy float64, as it stands) timed on the host cores on a bounded
+    sample of a workload; returns the cpu_baseline object (tokens/s)."""
+    import oracle as O
+    threads = _oracle_threads()
+    if name == "tiny-fp32":
+        m = _oracle_model(w, w.n_layers)
+        tok = _f64(synth.tokens(w, (w.batch, w.prefill_len + w.decode_steps), 0, "cuda")).astype(np.int64)
+        t0 = time.perf_counter()
+        m.forward(tok[:, :w.prefill_len], 0)
+        for s in range(w.decode_steps):
+            p = w.prefill_len + s
+            m.forward(tok[:, p:p + 1], p)
+        t = time.perf_counter() - t0
+        return {"value": round(w.batch * (w.prefill_len + w.decode_steps) / t, 2), "unit": "tokens/s",
+                "cores": threads, "kind": "oracle", "sample": "the whole run: prefill of 32 tokens and 16 decode steps"}
+    if name == "llama70b-layer":
+        t, threads, sample = oracle_layer_sample(w, n_decode=1)
+        return {"value": round(w.batch * w.decode_steps / t, 2), "unit": "tokens/s", "cores": threads,
+                "kind": "oracle", "sample": "one decode step of batch 16 over the 4096-position cache (the full step)"}
+    if name == "llama3-8b-decode":
+        L = 2
+        m = _oracle_model(w, L)
+        lens = _f64(synth.ragged_lengths(w, "cuda")).astype(np.int64)
+        shape = (w.max_batch_size, w.max_seq_len, w.n_kv_heads, w.head_dim)
+        for i in range(L):
+            m.cache_k[i][...] = _f64(synth.cache_values(w, i, 0, shape, "cuda"))
+            m.cache_v[i][...] = _f64(synth.cache_values(w, i, 1, shape, "cuda"))
+        tok = _f64(synth.tokens(w, (w.decode_steps, w.batch), 0, "cuda")).astype(np.int64)[0]
+        t0 = time.perf_counter()
+        h = O.as_f64(m.tok_embeddings[tok]).reshape(w.batch, 1, w.dim)
+        t_embed = time.perf_counter() - t0
+        t_layers = []
+        for i in range(L):
+            t0 = time.perf_counter()
+            h = m.block(i, h, lens)
+            t_layers.append(time.perf_counter() - t0)
+        t0 = time.perf_counter()
+        m._lm_head(O.rmsnorm(h, m.norm, w.norm_eps, w.act))
+        t_head = time.perf_counter() - t0
+        t_step = t_embed + w.n_layers * (sum(t_layers) / L) + t_head
+        return {"value": round(w.batch / t_step, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": "one decode step of the 32 sequences (ragged, first of the 64 steps) over 2 of the 32 "
+                          "layers + the final norm and LM head, timed; the per-layer time scaled to 32 layers"}
+    if name == "llama3-8b-prefill":
+        L, T = 2, 1024
+        m = _oracle_model(w, L, max_batch_size=1, max_seq_len=T)
+        tok = _f64(synth.tokens(w, (w.batch, w.prefill_len), 0, "cuda")).astype(np.int64)[:1, :T]
+        t0 = time.perf_counter()
+        m.forward(tok, 0, all_positions=False)
+        t = time.perf_counter() - t0
+        return {"value": round(T / t, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": "a reduced prefill: 1 x 1024 tokens through 2 layers of the same dims + the final norm "
+                          "and last-position LM head (the full 4 x 8192 x 32-layer prefill is ~528 TFLOP)"}
+    raise ValueError(name)
+
+
+CONFIG_STEPS = {"tiny-fp32": (20, 3), "llama70b-layer": (50, 3), "llama3-8b-decode": (3, 3),
+                "llama3-8b-prefill": (3, 3)}
+
+
+def run_configs(args, world, local, peaks, peak_kind, names):
+    """The other workloads, one object each: device-timed value, clocks, the
+    dominant kernel's roofline, end to end with host buffers, and the oracle's
+    CPU baseline (rank 0 at one GPU)."""
+    out = {}
+    for name in names:
+        w = synth.WORKLOADS[name]
+        steps, warmup = CONFIG_STEPS[name]
+        if w.n_layers == 1:
+            lb = LayerBench(w)
+            g = lb.capture("all")
+            sampler = NvmlClockSampler(local)
+            barrier(world)
+            sampler.start()
+            ms = max_over_ranks(time_graph(g, steps, warmup, world), world)
+            clocks = sampler.stop()
+            ms_step = ms / steps
+            wbytes = 2 * (w.dim * (w.n_heads + 2 * w.n_kv_heads) * w.head_dim + w.n_heads * w.head_dim * w.dim +
+                          3 * w.dim * w.ffn_hidden)
+            kv = w.batch * (w.cache_len + 1) * 2 * w.n_kv_heads * w.head_dim * 2
+            r = {"workload": w.name, "value": round(world * lb.tokens_per_step * steps / (ms * 1e-3), 1),
+                 "unit": "tokens/s", "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
+                 "clocks": clocks, "gpu_launches": lb.kernels_per_step() * steps,
+                 "phases": {"weights_gb": round(wbytes / 1e9, 3), "kv_gb": round(kv / 1e9, 4),
+                            "hbm_gbs": round((wbytes + kv) / (ms_step * 1e-3) / 1e9, 1),
+                            "hbm_frac": round((wbytes + kv) / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}}
+            r["roofline"] = linear_roofline(lb.decode_gemms(), B.LLAMA_PATH_GEMV, peaks, 5,
+                                            "llama_decode_linear_kernel (the 70B layer's decode linears at 16 "
+                                            "tokens: wqkv, wo, w1|w3, w2)")
+            r["roofline"]["peak_kind"] = peak_kind
+            r["e2e"] = run_e2e(lb, g, argparse.Namespace(steps=steps, warmup=warmup), world)
+            del g
+            lb.close()
+        else:
+            mb = ModelBench(w)
+            r = model_config_entry(mb, steps, warmup, world, local, peaks, peak_kind)
+            r["e2e"] = run_e2e_graph(mb.graph, mb.inputs, mb.outputs(), mb.tokens_per_step,
+                                     argparse.Namespace(steps=steps, warmup=warmup), world)
+            mb.close()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        if world == 1 and not args.no_cpu_baseline:
+            r["cpu_baseline"] = oracle_sample(name, w)
+        out[name] = r
+    return out
 
 
 # ----------------------------------------------------------------------------- main
@@ -447,18 +622,24 @@ def run_ours(args, world, rank, local):
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic: seeded N(0,1) hidden states, N(0,0.02) weights, RMSNorm weights 1",
+           "data": "synthetic: seeded N(0,1) hidden states, N(0,0.02) weights, RMSNorm weights 1 (as the workloads state)",
            "config": {"workload": w.name, "batch": lb.Bsz, "prefill_tokens": lb.P, "decode_steps": lb.ND,
                       "decode_start_pos": lb.dec_pos0, "l2": "inputs larger than L2: %.0f MB of weights per pass"
                       % (wbytes / 1e6), "parallelism": "replicas" if world > 1 else "single GPU",
                       "decode_kernel": DECODE_KERNEL, "decode_attention": DECODE_ATTENTION},
            "phases": phases, "roofline": roof, "e2e": e2e,
            "gpu_launches": lb.kernels_per_step() * args.steps, "clocks": clocks}
+    del g
+    lb.close()
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, threads, sample = oracle_layer_sample(w)
         out["cpu_baseline"] = {"value": round(lb.tokens_per_step / t_cpu, 2), "unit": "tokens/s", "cores": threads,
                                "kind": "oracle", "sample": sample}
-    lb.close()
+    if world == 1 and args.configs != "none":
+        names = [n for n in ("tiny-fp32", "llama70b-layer", "llama3-8b-decode", "llama3-8b-prefill")
+                 if n != args.workload and (args.configs == "all" or n in args.configs.split(","))]
+        out["configs"] = run_configs(args, world, local, peaks, peak_kind, names)
     return out
 
 
@@ -495,65 +676,191 @@ def run_e2e(lb: LayerBench, g, args, world):
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bi}
 
 
-def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
-    """Whole-model workloads (LLaMA-3-8B shape): ragged decode or long prefill."""
-    m = B.Llama(B.ModelArgs.from_workload(w))
-    ctx = m.ctx
-    B.llama_set_decode_kernel(ctx, DECODE_KERNELS[DECODE_KERNEL])
-    B.llama_set_decode_attention(ctx, DECODE_ATTENTIONS[DECODE_ATTENTION])
-    for i in range(w.n_layers):
-        B.llama_set_layer(ctx, i, synth.layer_weights(w, i, device="cuda"))
-    enh = synth.embed_norm_head(w, device="cuda")
-    B.llama_set_embed_norm_head(ctx, enh["tok_embeddings"], enh["norm"], enh["output"])
-    del enh
-    if w.decode_steps:
-        lens = synth.ragged_lengths(w, "cuda")
-        shape = (w.max_batch_size, w.max_seq_len, w.n_kv_heads, w.head_dim)
+class ModelBench:
+    """A whole model (embedding, blocks, final norm, LM head) through llama_forward /
+    llama_forward_ragged, one step captured in a CUDA graph:
+      - the tiny fp32 model: a 32-token prefill then 16 decode steps, all-position logits;
+      - the LLaMA-3-8B shape, ragged decode: 64 decode steps of a batch of 32 at
+        per-sequence positions (caches prefilled with N(0,1) to uniform lengths);
+      - the LLaMA-3-8B shape, prefill: 4 x 8192 tokens from start_pos 0, last-position logits."""
+
+    def __init__(self, w: synth.Workload):
+        self.w = w
+        self.m = B.Llama(B.ModelArgs.from_workload(w))
+        ctx = self.ctx = self.m.ctx
+        B.llama_set_decode_kernel(ctx, DECODE_KERNELS[DECODE_KERNEL])
+        B.llama_set_decode_attention(ctx, DECODE_ATTENTIONS[DECODE_ATTENTION])
         for i in range(w.n_layers):
-            k = synth.cache_values(w, i, 0, shape, "cuda")
-            v = synth.cache_values(w, i, 1, shape, "cuda")
-            B.llama_kv_write(ctx, i, k, v)
-            del k, v
-        toks = synth.tokens(w, (w.decode_steps, w.batch), 0, "cuda")
-        pos = (lens[None, :] + torch.arange(w.decode_steps, device="cuda", dtype=torch.int32)[:, None]).contiguous()
-        logits = torch.empty((w.batch, w.vocab_size), device="cuda")
-        B.llama_reserve(ctx, w.batch)
-
-        def enqueue():
-            for s in range(w.decode_steps):
-                B.llama_forward_ragged(ctx, toks[s], pos[s], logits)
-        tokens_per_step = w.batch * w.decode_steps
-        # per forward: embedding, the blocks, final RMSNorm, LM head
+            B.llama_set_layer(ctx, i, synth.layer_weights(w, i, device="cuda"))
+        enh = synth.embed_norm_head(w, device="cuda")
+        B.llama_set_embed_norm_head(ctx, enh["tok_embeddings"], enh["norm"], enh["output"])
+        del enh
         per_block = 1 if DECODE_KERNEL == "persistent" else 7
-        launches_per_step = w.decode_steps * (1 + w.n_layers * per_block + 2)
-    else:
-        toks = synth.tokens(w, (w.batch, w.prefill_len), 0, "cuda")
-        logits = torch.empty((w.batch, w.vocab_size), device="cuda")
-        B.llama_reserve(ctx, w.batch * w.prefill_len)
+        if w.ragged_hi:                      # ragged decode from prefilled caches
+            self.kind = "ragged-decode"
+            self.lens = synth.ragged_lengths(w, "cuda")
+            shape = (w.max_batch_size, w.max_seq_len, w.n_kv_heads, w.head_dim)
+            for i in range(w.n_layers):
+                k = synth.cache_values(w, i, 0, shape, "cuda")
+                v = synth.cache_values(w, i, 1, shape, "cuda")
+                B.llama_kv_write(ctx, i, k, v)
+                del k, v
+            self.toks = synth.tokens(w, (w.decode_steps, w.batch), 0, "cuda")
+            steps = torch.arange(w.decode_steps, device="cuda", dtype=torch.int32)[:, None]
+            self.pos = (self.lens[None, :] + steps).contiguous()
+            self.logits = torch.empty((w.batch, w.vocab_size), device="cuda")
+            B.llama_reserve(ctx, w.batch)
+            self.tokens_per_step = w.batch * w.decode_steps
+            self.launches_per_step = w.decode_steps * (1 + w.n_layers * per_block + 2)
+            self.inputs = [self.toks, self.pos]
+        elif w.decode_steps:                 # prefill then decode steps, all-position logits
+            self.kind = "prefill+decode"
+            P, ND = w.prefill_len, w.decode_steps
+            self.toks = synth.tokens(w, (w.batch, P + ND), 0, "cuda")
+            self.logits_pre = torch.empty((w.batch, P, w.vocab_size), device="cuda")
+            self.logits_dec = torch.empty((ND, w.batch, 1, w.vocab_size), device="cuda")
+            if w.batch != 1:
+                raise ValueError("the prefill+decode model step reads its decode tokens as views (batch 1)")
+            B.llama_reserve(ctx, w.batch * P)
+            self.tokens_per_step = w.batch * (P + ND)
+            blocks = 1 + w.n_layers * 7 + 2
+            self.launches_per_step = blocks + ND * (1 + w.n_layers * (per_block if w.act == "bf16" else 7) + 2)
+            self.inputs = [self.toks]
+        else:                                # one long prefill, last-position logits
+            self.kind = "prefill"
+            self.toks = synth.tokens(w, (w.batch, w.prefill_len), 0, "cuda")
+            self.logits = torch.empty((w.batch, w.vocab_size), device="cuda")
+            B.llama_reserve(ctx, w.batch * w.prefill_len)
+            self.tokens_per_step = w.batch * w.prefill_len
+            self.launches_per_step = 1 + w.n_layers * 7 + 2
+            self.inputs = [self.toks]
+        self.enqueue()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.enqueue()
+        torch.cuda.synchronize()
 
-        def enqueue():
-            B.llama_forward(ctx, toks, 0, logits, False)
-        tokens_per_step = w.batch * w.prefill_len
-        launches_per_step = 1 + w.n_layers * 7 + 2
-    enqueue()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        enqueue()
-    sampler = NvmlClockSampler(local)
-    sampler.start()
-    ms = max_over_ranks(time_graph(g, args.steps, args.warmup, world), world)
-    clocks = sampler.stop()
-    code, flags = B.llama_get_error(ctx)
-    out = {"metric": METRIC, "value": round(world * tokens_per_step * args.steps / (ms * 1e-3), 1),
-           "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL,
-                                                "decode_attention": DECODE_ATTENTION}, "clocks": clocks, "device_error": code,
-           "gpu_launches": launches_per_step * args.steps}
-    m.close()
+    def enqueue(self):
+        w, ctx = self.w, self.ctx
+        if self.kind == "ragged-decode":
+            for s in range(w.decode_steps):
+                B.llama_forward_ragged(ctx, self.toks[s], self.pos[s], self.logits)
+        elif self.kind == "prefill+decode":
+            P = w.prefill_len
+            B.llama_forward(ctx, self.toks[:, :P], 0, self.logits_pre, True)
+            for s in range(w.decode_steps):
+                B.llama_forward(ctx, self.toks[:, P + s:P + s + 1], P + s, self.logits_dec[s], True)
+        else:
+            B.llama_forward(ctx, self.toks, 0, self.logits, False)
+
+    def outputs(self):
+        if self.kind == "prefill+decode":
+            return [self.logits_pre, self.logits_dec]
+        return [self.logits]
+
+    def close(self):
+        del self.graph
+        self.m.close()
+
+
+def run_e2e_graph(g, inputs, outputs, tokens_per_step, args, world, steps=None):
+    """The step through the C ABI with host buffers: every step copies its inputs
+    from pinned host memory to the device, replays the step, and copies its
+    result back to pinned host memory, all inside the timed region."""
+    steps = args.steps if steps is None else steps
+    hin = [t.cpu().pin_memory() for t in inputs]
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outputs]
+    st = torch.cuda.current_stream()
+
+    def step():
+        for d, h in zip(inputs, hin):
+            d.copy_(h, non_blocking=True)
+        g.replay()
+        for h, d in zip(hout, outputs):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        step()
+    e1.record(st)
+    e1.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": round(world * tokens_per_step * steps / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in inputs)),
+            "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outputs))}
+
+
+def run_model_bench(args, world, rank, local, w, peaks, peak_kind):
+    """A whole-model workload as the headline line (--workload llama3-8b-*)."""
+    mb = ModelBench(w)
+    r = model_config_entry(mb, args.steps, args.warmup, world, local, peaks, peak_kind)
+    out = {"metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32" if w.act == "fp32" else "bf16", "data": "synthetic",
+           "config": {"workload": w.name, "decode_kernel": DECODE_KERNEL, "decode_attention": DECODE_ATTENTION},
+           "phases": r.get("phases", {}), "roofline": r["roofline"], "clocks": r["clocks"],
+           "gpu_launches": r["gpu_launches"]}
+    out["e2e"] = run_e2e_graph(mb.graph, mb.inputs, mb.outputs(), mb.tokens_per_step, args, world)
+    mb.close()
     return out
+
+
+def model_config_entry(mb: ModelBench, steps, warmup, world, local, peaks, peak_kind):
+    """Time a whole-model step and measure its dominant kernel."""
+    w = mb.w
+    sampler = NvmlClockSampler(local)
+    barrier(world)
+    sampler.start()
+    ms = max_over_ranks(time_graph(mb.graph, steps, warmup, world), world)
+    clocks = sampler.stop()
+    code, flags = B.llama_get_error(mb.ctx)
+    if code != B.LLAMA_OK:
+        raise RuntimeError(f"device flag raised during the timed steps: {B.strerror(code)} ({flags})")
+    ms_step = ms / steps
+    r = {"workload": w.name, "value": round(world * mb.tokens_per_step * steps / (ms * 1e-3), 1),
+         "unit": "tokens/s", "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
+         "clocks": clocks, "gpu_launches": mb.launches_per_step * steps}
+    D, H, Hkv, F = w.head_dim, w.n_heads, w.n_kv_heads, w.ffn_hidden
+    layer_params = w.dim * (H + 2 * Hkv) * D + H * D * w.dim + 3 * w.dim * F
+    if mb.kind == "ragged-decode":
+        wbytes = 2 * (w.n_layers * layer_params + w.vocab_size * w.dim)
+        lens = mb.lens.double()
+        kv = sum(float((lens + s + 1).sum()) for s in range(w.decode_steps)) * w.n_layers * 2 * Hkv * D * 2
+        byts = w.decode_steps * wbytes + kv
+        r["phases"] = {"weights_gb_per_decode_step": round(wbytes / 1e9, 3),
+                       "kv_gb_per_decode_step": round(kv / w.decode_steps / 1e9, 3),
+                       "hbm_gbs": round(byts / (ms_step * 1e-3) / 1e9, 1),
+                       "hbm_frac": round(byts / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+        r["roofline"] = linear_roofline(layer_pairs(w, w.batch), B.LLAMA_PATH_GEMV, peaks, 5,
+                                        "llama_decode_linear_kernel (the 8B layer's decode linears at 32 tokens)")
+    elif mb.kind == "prefill":
+        T = w.prefill_len
+        flops = 2.0 * w.batch * T * w.n_layers * layer_params
+        flops += w.n_layers * w.batch * 4.0 * H * D * (T * (T + 1) / 2)
+        flops += 2.0 * w.batch * w.dim * w.vocab_size
+        r["phases"] = {"tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
+                       "tensor_frac_sustained": round(flops / (ms_step * 1e-3) / 1e12
+                                                      / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4)}
+        r["roofline"] = linear_roofline(layer_pairs(w, w.batch * T), B.LLAMA_PATH_TCGEN05, peaks, 2,
+                                        "gemm_tc_kernel (the 8B layer's prefill linears at 32768 tokens)",
+                                        bound="tensor", peak_key="bf16_tflops_sustained"
+                                        if "bf16_tflops_sustained" in peaks else "bf16_tflops")
+    else:   # the tiny fp32 model: latency-bound, 2.08 M parameters
+        n_fwd = 1 + w.decode_steps
+        wbytes = 4 * (w.n_layers * layer_params + 2 * w.vocab_size * w.dim)
+        achieved = n_fwd * wbytes / (ms_step * 1e-3) / 1e9
+        r["roofline"] = {"kernel": "whole step (latency-bound: %d launches of a 2-layer dim-256 model)"
+                         % mb.launches_per_step, "bound": "hbm", "achieved": round(achieved, 2),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 5),
+                         "traffic": None, "bytes_per_step": n_fwd * wbytes}
+    r["roofline"]["peak_kind"] = peak_kind
+    return r
 
 
 def run_reference(args, world, rank):
@@ -595,6 +902,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b-layer", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="all",
+                    help="the other workloads reported under 'configs' at one GPU: all, none, or a comma list")
     ap.add_argument("--clock-log", default=None, help="directory for the per-rank clock sample CSV")
     ap.add_argument("--decode-kernel", default="auto", choices=sorted(DECODE_KERNELS),
                     help="decode-step launch structure (llama_set_decode_kernel)")

@@ -402,12 +402,29 @@ int llama_linear(const void* x_dev, const void* w_dev, float* y_dev, int M, int 
  * LLAMA_ERR_TOO_LARGE before anything is launched.
  * The first call on a device (with that device current) looks up the array's
  * device address; make that first call before any stream capture.
+ * cudaDeviceReset unloads the array: the address looked up before it is not
+ * valid afterwards, so do not call this entry point on a device after
+ * resetting it (a call whose CUDA work fails forgets the address, and the
+ * next call looks it up again).
  * All calls on one device share the array and it keeps the last call's
  * contents; calls whose kernels overlap on the GPU (different streams without
  * ordering between them) race. The arrival counters are cleared on
- * cuda_stream before each launch. Stream-ordered, asynchronous.
+ * cuda_stream before each launch. Stream-ordered, asynchronous: the return
+ * code covers only what the host can check. A bounded in-kernel wait that
+ * gives up sets a bit in an error word inside the array, which stays set
+ * until llama_linear_noalloc_status reads it.
  */
 int llama_linear_noalloc(const void* x_dev, const void* w_dev, float* y_dev, int M, int N, int K, void* cuda_stream);
+
+/*
+ * Status of llama_linear_noalloc on the current device (the pages have no
+ * counterpart): synchronises the device, copies the error word out of the
+ * fixed array into a host variable, clears it, and returns LLAMA_OK or
+ * LLAMA_ERR_TIMEOUT (a bounded wait of some call since the last status read
+ * gave up, so that call's y is not valid); LLAMA_ERR_CUDA when the copy fails.
+ * *flags (if not NULL) receives the raw bits (4 = timeout). Allocates nothing.
+ */
+int llama_linear_noalloc_status(int* flags);
 
 #ifdef __cplusplus
 }

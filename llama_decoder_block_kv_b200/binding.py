@@ -37,7 +37,7 @@ LLAMA_ATTN_AUTO, LLAMA_ATTN_CHUNKED, LLAMA_ATTN_STREAMK = 0, 1, 2
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
-            "llama_linear_noalloc", "llama_sample", "llama_generate", "llama_set_decode_kernel",
+            "llama_linear_noalloc", "llama_linear_noalloc_status", "llama_sample", "llama_generate", "llama_set_decode_kernel",
             "llama_set_decode_attention", "llama_tile_weights",
             "llama_selftest_bounded_wait", "llama_set_alloc_limit", "llama_allocated_bytes",
             "llama_selfcheck_plans")
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.llama_strerror.restype = ctypes.c_char_p
         L.llama_linear.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
         L.llama_linear_noalloc.argtypes = [vp, vp, vp, i, i, i, vp]
+        L.llama_linear_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.llama_sample.argtypes = [vp, i, i, f, f, vp, vp, vp]
         L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
         L.llama_set_decode_kernel.argtypes = [vp, i]
@@ -296,6 +297,13 @@ def llama_linear_noalloc(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, stre
     M, K = x.shape
     N = w.shape[0]
     return lib().llama_linear_noalloc(_ptr(x), _ptr(w), _ptr(y), M, N, K, _stream(stream))
+
+
+def llama_linear_noalloc_status():
+    """(code, raw error bits) of llama_linear_noalloc on the current device; clears them."""
+    flags = ctypes.c_int(0)
+    code = lib().llama_linear_noalloc_status(ctypes.byref(flags))
+    return code, flags.value
 
 
 class Llama:

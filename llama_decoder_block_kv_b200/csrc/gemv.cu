@@ -67,7 +67,7 @@ __host__ __device__ __forceinline__ int sk_owner(int x, int total, int grid) {
 
 template <int MB>
 __global__ void __launch_bounds__(160, 1)
-    gemv_bf16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
+    llama_decode_linear_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
                      int N, int nk, int total, int tiled, float* __restrict__ part, int* __restrict__ counters,
                      EpiParams ep) {
   constexpr int STAGES = stages(MB);
@@ -327,9 +327,9 @@ static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M
                              int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
   constexpr size_t smem = gemv_smem(MB);
   static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(gemv_bf16_kernel<MB>, smem, attr);
+  cudaError_t e = ensure_smem(llama_decode_linear_kernel<MB>, smem, attr);
   if (e != cudaSuccess) return e;
-  return launch_pdl(gemv_bf16_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
+  return launch_pdl(llama_decode_linear_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
                     counters, ep);
 }
 

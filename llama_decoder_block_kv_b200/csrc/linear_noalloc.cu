@@ -17,7 +17,11 @@
 // any stream capture. All calls on a device share the one array: calls whose
 // kernels overlap on the GPU (e.g. on two streams) race and corrupt each
 // other's partial sums. The counters are cleared on the caller's stream before
-// each launch.
+// each launch. The error word is not: a bounded wait that gave up leaves its bit
+// there until llama_linear_noalloc_status reads and clears it. cudaDeviceReset
+// unloads the array with the rest of the device code, so the address found at
+// set-up is no longer valid on that device afterwards; a failed CUDA call in
+// this path forgets the address, so the next call looks it up again.
 #include <cstring>
 #include <mutex>
 
@@ -56,6 +60,15 @@ int scratch_on_current_device(unsigned char** out) {
   return LLAMA_OK;
 }
 
+// After a failed CUDA call the cached address may be stale (e.g. the device was
+// reset): look it up again on the next call.
+void forget_scratch_of_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  g_scratch[dev].ready = false;
+}
+
 }  // namespace
 }  // namespace llama
 
@@ -74,8 +87,12 @@ extern "C" int llama_linear_noalloc(const void* x, const void* w, float* y, int 
   int* counters = reinterpret_cast<int*>(base + NOALLOC_PART_FLOATS * 4);
   int* err = counters + NOALLOC_COUNTERS;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
-  // the arrival counters and the error word must start at zero
-  if (cudaMemsetAsync(counters, 0, (NOALLOC_COUNTERS + 1) * sizeof(int), st) != cudaSuccess) return LLAMA_ERR_CUDA;
+  // the arrival counters must start at zero; the error word (bit 4: a bounded
+  // wait timed out) is left as it is until llama_linear_noalloc_status clears it
+  if (cudaMemsetAsync(counters, 0, NOALLOC_COUNTERS * sizeof(int), st) != cudaSuccess) {
+    forget_scratch_of_current_device();
+    return LLAMA_ERR_CUDA;
+  }
   EpiParams e;
   memset(&e, 0, sizeof(e));
   e.kind = EPI_STORE_F32;
@@ -84,6 +101,27 @@ extern "C" int llama_linear_noalloc(const void* x, const void* w, float* y, int 
   e.out = y;
   e.ld_out = N;
   e.err = err;
-  if (launch_gemv_bf16(x, w, 0, M, N, K, p, part, counters, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+  if (launch_gemv_bf16(x, w, 0, M, N, K, p, part, counters, e, sms, st) != cudaSuccess) {
+    forget_scratch_of_current_device();
+    return LLAMA_ERR_CUDA;
+  }
   return LLAMA_OK;
+}
+
+extern "C" int llama_linear_noalloc_status(int* flags) {
+  using namespace llama;
+  if (flags) *flags = 0;
+  unsigned char* base = nullptr;
+  int r = scratch_on_current_device(&base);
+  if (r != LLAMA_OK) return r;
+  int* err = reinterpret_cast<int*>(base + NOALLOC_PART_FLOATS * 4) + NOALLOC_COUNTERS;
+  int word = 0;
+  // a plain synchronous copy into a host variable: nothing is allocated
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpy(&word, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(err, 0, sizeof(int)) != cudaSuccess) {
+    forget_scratch_of_current_device();
+    return LLAMA_ERR_CUDA;
+  }
+  if (flags) *flags = word;
+  return (word & LLAMA_DEV_TIMEOUT) ? LLAMA_ERR_TIMEOUT : LLAMA_OK;
 }

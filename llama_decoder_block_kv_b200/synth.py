@@ -5,7 +5,10 @@ casts them to a storage dtype. It holds no arithmetic of the model: sizes such
 as the FFN width are stated per workload, not derived here.
 
 Recipe (all workloads): linear weights ~ N(0, 0.02^2) drawn in fp32 and cast
-(round-to-nearest-even) to the storage dtype; RMSNorm weights are 1; hidden
+(round-to-nearest-even) to the storage dtype; RMSNorm weights are 1 (the
+workloads' statement), or, for parity cases that must exercise the learned
+norm weight, 1 + N(0, 0.1^2) drawn per layer and per norm and cast to the
+storage dtype (``Workload.norm_weights = "random"``); hidden
 states ~ N(0, 1) cast to the activation dtype and handed over as fp32; token ids
 uniform in [0, vocab); prefilled cache entries ~ N(0, 1) in the cache dtype;
 ragged cache lengths uniform over an inclusive integer range. Every tensor has
@@ -20,6 +23,7 @@ from typing import Optional
 import torch
 
 WEIGHT_STD = 0.02
+NORM_WEIGHT_STD = 0.1
 LAYER_WEIGHT_NAMES = ("wq", "wk", "wv", "wo", "w1", "w2", "w3")
 
 
@@ -47,6 +51,7 @@ class Workload:
     ragged_lo: int = 0       # ragged cache lengths, inclusive range
     ragged_hi: int = 0
     seed: int = 0
+    norm_weights: str = "unit"   # "unit" (all 1) or "random" (1 + N(0, 0.1^2), per layer and per norm)
 
     @property
     def head_dim(self) -> int:
@@ -128,25 +133,38 @@ def storage_dtype(w: Workload) -> torch.dtype:
 _ROLE_LAYER, _ROLE_EMBED, _ROLE_NORM, _ROLE_HEAD, _ROLE_TOKENS, _ROLE_HIDDEN, _ROLE_CACHE, _ROLE_LENS = range(8)
 
 
+def norm_weight(w: Workload, which: int, layer: int = 0, device="cpu") -> torch.Tensor:
+    """One RMSNorm weight vector [dim]: all 1, or 1 + N(0, 0.1^2) with its own seed
+    (which = 0 attention_norm, 1 ffn_norm, 2 the final norm)."""
+    dt = storage_dtype(w)
+    if w.norm_weights == "unit":
+        return torch.ones(w.dim, dtype=dt, device=device)
+    if w.norm_weights != "random":
+        raise ValueError(f"unknown norm_weights {w.norm_weights!r}")
+    x = torch.randn((w.dim,), generator=_gen(sub_seed(w.seed, _ROLE_NORM, layer, which), device),
+                    dtype=torch.float32, device=device)
+    return (1.0 + NORM_WEIGHT_STD * x).to(dt)
+
+
 def layer_weights(w: Workload, layer: int, device="cpu") -> dict:
-    """Weights of one block as [out, in] tensors (the nn.Linear layout), norms = 1."""
+    """Weights of one block as [out, in] tensors (the nn.Linear layout) and its two norm weights."""
     D, H, Hkv, F = w.head_dim, w.n_heads, w.n_kv_heads, w.ffn_hidden
     shapes = {"wq": (H * D, w.dim), "wk": (Hkv * D, w.dim), "wv": (Hkv * D, w.dim),
               "wo": (w.dim, H * D), "w1": (F, w.dim), "w2": (w.dim, F), "w3": (F, w.dim)}
     dt = storage_dtype(w)
     out = {name: normal(shapes[name], WEIGHT_STD, sub_seed(w.seed, _ROLE_LAYER, layer, i), dt, device)
            for i, name in enumerate(LAYER_WEIGHT_NAMES)}
-    out["attn_norm"] = torch.ones(w.dim, dtype=dt, device=device)
-    out["ffn_norm"] = torch.ones(w.dim, dtype=dt, device=device)
+    out["attn_norm"] = norm_weight(w, 0, layer, device)
+    out["ffn_norm"] = norm_weight(w, 1, layer, device)
     return out
 
 
 def embed_norm_head(w: Workload, device="cpu") -> dict:
-    """Token embedding [vocab, dim], final norm weight [dim] (= 1), LM head [vocab, dim]."""
+    """Token embedding [vocab, dim], final norm weight [dim], LM head [vocab, dim]."""
     dt = storage_dtype(w)
     return {
         "tok_embeddings": normal((w.vocab_size, w.dim), WEIGHT_STD, sub_seed(w.seed, _ROLE_EMBED), dt, device),
-        "norm": torch.ones(w.dim, dtype=dt, device=device),
+        "norm": norm_weight(w, 2, 0, device),
         "output": normal((w.vocab_size, w.dim), WEIGHT_STD, sub_seed(w.seed, _ROLE_HEAD), dt, device),
     }
 

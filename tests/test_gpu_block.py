@@ -19,7 +19,8 @@ def _wl(dim, H, Hkv, act="bf16", Bm=2, S=256, mo=256, seed=5):
     F = O.ffn_hidden_dim(dim, mo)
     return synth.Workload(name=f"block dim {dim} H {H}/{Hkv}", dim=dim, n_layers=1, n_heads=H, n_kv_heads=Hkv,
                           ffn_hidden=F, vocab_size=0, multiple_of=mo, ffn_dim_multiplier=None, norm_eps=1e-5,
-                          rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act=act, batch=Bm, seed=seed)
+                          rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act=act, batch=Bm, seed=seed,
+                          norm_weights="random")
 
 
 def _run(pair: Pair, h: torch.Tensor, start_pos, tol_hidden):
@@ -146,6 +147,40 @@ def test_long_context_prefill_rows_and_decode():
         written[0, :1000] = True
         written[0, 12000:16096] = True
         written[0, 16383] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("dim,H,Hkv", [(512, 4, 2), (1024, 8, 1)])
+def test_chunked_prefill_with_per_sequence_positions(dim, H, Hkv):
+    """T > 1 with a device vector of start positions (chunked prefill of sequences
+    at different offsets in one call). Query s of sequence b sits at position
+    start_pos[b] + s and sees keys j <= start_pos[b] + s ("灵哥讲llama3(中)",
+    Transformer class, mask comment). The offsets are chosen so that query blocks
+    start mid-tile, the diagonal crosses key tiles, and one sequence starts at 0."""
+    w = _wl(dim, H, Hkv, Bm=3, S=512)
+    pair = Pair(w)
+    try:
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        h = synth.hidden(w, (3, 150, dim), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        written[:3, :150] = True
+        sp = np.array([150, 37, 0])          # sequence 1 and 2 rewrite part of their history
+        h = synth.hidden(w, (3, 70, dim), call=1)
+        _run(pair, h, sp, BF16_HIDDEN_ABS)
+        for b in range(3):
+            written[b, sp[b]:sp[b] + 70] = True
+        sp = np.array([220, 300, 70])        # a jump: positions 107..299 of sequence 1 stay as they are
+        h = synth.hidden(w, (3, 129, dim), call=2)
+        _run(pair, h, sp, BF16_HIDDEN_ABS)
+        for b in range(3):
+            written[b, sp[b]:sp[b] + 129] = True
+        # a decode step after the ragged chunks
+        pos = np.array([349, 429, 199])
+        _run(pair, synth.hidden(w, (3, 1, dim), call=3), pos, BF16_HIDDEN_ABS)
+        for b in range(3):
+            written[b, pos[b]] = True
         assert_cache_matches(pair, 0, written, 2e-2)
     finally:
         pair.close()

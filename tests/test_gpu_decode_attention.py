@@ -32,7 +32,7 @@ def _wl(dim, H, Hkv, Bm, S=256, mo=256, seed=23):
     return synth.Workload(name=f"decode attention dim {dim} H {H}/{Hkv}", dim=dim, n_layers=1, n_heads=H,
                           n_kv_heads=Hkv, ffn_hidden=F, vocab_size=0, multiple_of=mo, ffn_dim_multiplier=None,
                           norm_eps=1e-5, rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act="bf16", batch=Bm,
-                          seed=seed)
+                          seed=seed, norm_weights="random")
 
 
 def _run(pair, h, start_pos):
@@ -96,6 +96,26 @@ def test_decode_steps_match_oracle(dim, H, Hkv, Bsz):
             h = synth.hidden(w, (Bsz, 1, dim), call=1 + i)
             _decode_both(pair, h, 70 + i)
             written[:Bsz, 70 + i] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
+@pytest.mark.parametrize("dim,H,Hkv", [(768, 6, 2), (768, 12, 2)])
+def test_long_prefill_then_decode_odd_head_ratios(dim, H, Hkv):
+    """3 and 6 query heads per kv head: the prefill attention serves one or two
+    heads per CTA, so a CTA holds 128 or 64 positions. A 300-token prefill of
+    two sequences spans several query blocks, puts the causal diagonal inside
+    later blocks, and has Q boxes that run past one sequence's end."""
+    w = _wl(dim, H, Hkv, 2, S=512)
+    pair = Pair(w)
+    try:
+        _step(pair, synth.hidden(w, (2, 300, dim), call=0), 0)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:2, :300] = True
+        for i in range(2):
+            _decode_both(pair, synth.hidden(w, (2, 1, dim), call=1 + i), 300 + i)
+            written[:2, 300 + i] = True
         assert_cache_matches(pair, 0, written, 2e-2)
     finally:
         pair.close()

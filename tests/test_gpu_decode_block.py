@@ -22,7 +22,8 @@ def _wl(dim, H, Hkv, Bm, S=256, mo=256, seed=11):
     F = O.ffn_hidden_dim(dim, mo)
     return synth.Workload(name=f"decode block dim {dim} H {H}/{Hkv}", dim=dim, n_layers=1, n_heads=H, n_kv_heads=Hkv,
                           ffn_hidden=F, vocab_size=0, multiple_of=mo, ffn_dim_multiplier=None, norm_eps=1e-5,
-                          rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act="bf16", batch=Bm, seed=seed)
+                          rope_theta=10000.0, max_batch_size=Bm, max_seq_len=S, act="bf16", batch=Bm, seed=seed,
+                          norm_weights="random")
 
 
 def _step(pair, h, start_pos):

@@ -69,7 +69,7 @@ def _small_model(act, seed=21):
     return synth.Workload(name="generation model", dim=256, n_layers=2, n_heads=4, n_kv_heads=2,
                           ffn_hidden=O.ffn_hidden_dim(256, 256), vocab_size=512, multiple_of=256,
                           ffn_dim_multiplier=None, norm_eps=1e-5, rope_theta=10000.0, max_batch_size=3,
-                          max_seq_len=64, act=act, batch=3, seed=seed)
+                          max_seq_len=64, act=act, batch=3, seed=seed, norm_weights="random")
 
 
 def _load(w):

@@ -26,8 +26,11 @@ def _forward(pair, tok, start_pos, all_positions=True):
     return t2np(out), ref
 
 
-def test_tiny_fp32_prefill_then_decode():
-    w = synth.TINY_FP32
+@pytest.mark.parametrize("norms", ["unit", "random"])
+def test_tiny_fp32_prefill_then_decode(norms):
+    """The tiny fp32 workload as stated (norm weights 1), and with learned-looking
+    norm weights so the weight multiply of every RMSNorm is checked too."""
+    w = synth.TINY_FP32.with_(norm_weights=norms)
     pair = Pair(w)
     try:
         tok = synth.tokens(w, (1, 32 + 16))
@@ -47,7 +50,8 @@ def test_tiny_fp32_prefill_then_decode():
 def _small_bf16(**kw):
     base = dict(name="small bf16 model", dim=512, n_layers=2, n_heads=8, n_kv_heads=2,
                 ffn_hidden=O.ffn_hidden_dim(512, 256), vocab_size=1000, multiple_of=256, ffn_dim_multiplier=None,
-                norm_eps=1e-5, rope_theta=500000.0, max_batch_size=3, max_seq_len=256, act="bf16", batch=3, seed=9)
+                norm_eps=1e-5, rope_theta=500000.0, max_batch_size=3, max_seq_len=256, act="bf16", batch=3, seed=9,
+                norm_weights="random")
     base.update(kw)
     return synth.Workload(**base)
 

@@ -30,7 +30,7 @@ def test_half_split_weights_match_interleaved_oracle(act):
     w = synth.Workload(name="half-split rope model", dim=256, n_layers=2, n_heads=4, n_kv_heads=2,
                        ffn_hidden=O.ffn_hidden_dim(256, 256), vocab_size=512, multiple_of=256,
                        ffn_dim_multiplier=None, norm_eps=1e-5, rope_theta=10000.0, max_batch_size=2, max_seq_len=64,
-                       act=act, batch=2, seed=13)
+                       act=act, batch=2, seed=13, norm_weights="random")
     D = w.head_dim
     lws = [synth.layer_weights(w, i) for i in range(w.n_layers)]
     enh = synth.embed_norm_head(w)

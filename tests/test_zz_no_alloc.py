@@ -1,10 +1,18 @@
 """llama_linear_noalloc through the C ABI: the decode GEMV with its scratch in a
 fixed array compiled into the library, for callers that cannot allocate device
-memory when they call (an application whose memory belongs to its own pool
-allocator, a loop where cudaMalloc/cudaFree and their possible device
-synchronisation are not acceptable). It must give the same result as
-llama_linear's GEMV path, call after call, and refuse shapes whose scratch
-would not fit. Collected last so a failure here leaves every other test run."""
+memory when they call (an application whose device memory belongs to its own
+pool allocator, so a cudaMalloc behind its back could fail or fragment it; a
+loop where cudaMalloc/cudaFree and the device synchronisation they can cause
+are not acceptable).
+
+Checked here: the result against a float64 matmul of the same bf16 inputs,
+call after call (the fixed array keeps the previous call's contents, so the
+second call checks that the counters were cleared); that the calls take no
+device memory (the library's tracked total and the device's free memory do
+not move, and the calls still run under an allocation cap set to what the
+library already holds); that the error word reads back clear; and that shapes
+whose scratch would not fit are refused. Collected last so that a failure here
+leaves every other test run."""
 import numpy as np
 import pytest
 import torch
@@ -14,24 +22,50 @@ from llama_decoder_block_kv_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-REL = 2e-5  # the GEMM-core tolerance of test_gpu_linear.py
+REL = 2e-5  # the GEMM-core tolerance of test_gpu_linear.py: of the largest output, fp32 accumulation
+
+
+def _inputs(M, N, K, seed):
+    x = synth.normal((M, K), 1.0, seed, torch.bfloat16, "cuda")
+    w = synth.normal((N, K), 0.02, seed + 1, torch.bfloat16, "cuda")
+    ref = x.double().cpu().numpy() @ w.double().cpu().numpy().T
+    return x, w, ref
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (7, 12288, 4096), (32, 4096, 11008), (3, 136, 192)])
-def test_noalloc_matches_linear_twice_in_a_row(M, N, K):
-    x = synth.normal((M, K), 1.0, 41, torch.bfloat16, "cuda")
-    w = synth.normal((N, K), 0.02, 42, torch.bfloat16, "cuda")
-    ref = torch.empty((M, N), device="cuda")
-    B.llama_linear(x, w, ref, B.LLAMA_PATH_GEMV)
-    torch.cuda.synchronize()
-    r = ref.double().cpu().numpy()
+def test_noalloc_matches_float64_matmul_twice_in_a_row(M, N, K):
+    x, w, ref = _inputs(M, N, K, 41)
+    scale = np.abs(ref).max()
     for _ in range(2):
         y = torch.full((M, N), float("nan"), device="cuda")
         assert B.llama_linear_noalloc(x, w, y) == B.LLAMA_OK
         torch.cuda.synchronize()
         got = y.double().cpu().numpy()
         assert np.all(np.isfinite(got))
-        assert np.abs(got - r).max() <= REL * np.abs(r).max()
+        err = np.abs(got - ref).max()
+        assert err <= REL * scale, (err, scale)
+    assert B.llama_linear_noalloc_status() == (B.LLAMA_OK, 0)
+
+
+def test_noalloc_takes_no_device_memory():
+    x, w, ref = _inputs(16, 8192, 4096, 43)
+    y = torch.empty((16, 8192), device="cuda")
+    assert B.llama_linear_noalloc(x, w, y) == B.LLAMA_OK     # warm-up (the per-device set-up)
+    torch.cuda.synchronize()
+    held, (free0, _) = B.llama_allocated_bytes(), torch.cuda.mem_get_info()
+    try:
+        B.llama_set_alloc_limit(max(held, 1))                # any allocation by the library would now fail
+        for _ in range(3):
+            y.fill_(float("nan"))
+            assert B.llama_linear_noalloc(x, w, y) == B.LLAMA_OK
+            torch.cuda.synchronize()
+            got = y.cpu().double().numpy()   # copied out first: no device-side temporary
+            assert np.abs(got - ref).max() <= REL * np.abs(ref).max()
+    finally:
+        B.llama_set_alloc_limit(0)
+    assert B.llama_allocated_bytes() == held
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert B.llama_linear_noalloc_status() == (B.LLAMA_OK, 0)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
