@@ -118,56 +118,34 @@ def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float
             assert_bf16_cache_close(got[written], ref[written], f"cache {name}")
 
 
-# ----------------------------------------------------------------------------- conditioning floor
+# ----------------------------------------------------------------------------- full-size bound
 #
-# The bf16 rounding points (norm outputs, q/k/v, attention output, silu*mul)
-# make the block ill-conditioned at its full sizes: a perturbation as small as
-# the rounding error of an fp32 accumulation flips a few bf16 roundings, and
-# the flips fan out through 4096..28672-wide sums. The oracle itself, fed
-# hidden states perturbed by a relative 2^-17 (the size of an fp32
-# accumulation error over ~2^14 terms), moves by up to ~0.04 (LLaMA-7B layer
-# prefill) and ~0.09 (LLaMA-2-70B layer decode) in max-abs. No
-# fp32-accumulating implementation can be held below that. At those sizes the
-# hidden-state check is: max and 99th percentile of |error| each within
-# max(2e-2, 3 x the same statistic of the oracle's own floor on the same inputs).
+# At the workloads' full sizes the bf16 rounding points (norm outputs, q/k/v,
+# attention output, silu*mul) make the block ill-conditioned: the rounding
+# error of an fp32 accumulation flips a few bf16 roundings, and each flip fans
+# out through 4096..28672-wide sums, so no fp32-accumulating implementation
+# stays within a flat 2e-2 of the float64 oracle everywhere. The bound there is
+# measured, not assumed: tests/emulation.py computes the same block with the
+# same rounding points and fp32 sums on the CPU, and the GPU result must be
+# within the flat bound, or within EMU_FACTOR x the emulation's own distance
+# from the oracle on the same inputs, for the maximum and for the 99th
+# percentile of |error| separately.
 
-PERTURB_REL = 2.0 ** -17
-FLOOR_FACTOR = 3.0
-
-
-def oracle_floor(run, h: np.ndarray, seed: int = 0):
-    """(run(h), floor) where floor = |run(h) - run(h * (1 + 2^-17 r))|, r ~ N(0, 1), as an array.
-
-    ``run`` must start from the same state each call; the unperturbed run is made
-    last so the oracle's caches end in the unperturbed state."""
-    r = np.random.default_rng(seed).standard_normal(h.shape)
-    pert = run(h * (1.0 + PERTURB_REL * r))
-    ref = run(h)
-    return ref, np.abs(ref - pert)
+EMU_FACTOR = 1.5
 
 
-def assert_hidden_close_floor(got: np.ndarray, ref: np.ndarray, floor: np.ndarray, what: str = ""):
+def assert_close_emulated(got: np.ndarray, ref: np.ndarray, emu: np.ndarray, flat: float, what: str = ""):
+    """|got - ref| within max(flat, EMU_FACTOR x |emu - ref|) in max and in p99; prints both."""
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     err = np.abs(got - ref)
-    p99, fp99 = float(np.quantile(err, 0.99)), float(np.quantile(floor, 0.99))
-    tol_max = max(BF16_HIDDEN_ABS, FLOOR_FACTOR * float(floor.max()))
-    tol_p99 = max(BF16_HIDDEN_ABS, FLOOR_FACTOR * fp99)
-    assert p99 <= tol_p99, f"{what}: p99 abs err {p99:.4g} > {tol_p99:.4g} (oracle floor p99 {fp99:.4g})"
-    assert err.max() <= tol_max, \
-        f"{what}: max abs err {err.max():.4g} > {tol_max:.4g} (oracle floor max {floor.max():.4g})"
-    return float(err.max()), p99
-
-
-def assert_logits_close_floor(got: np.ndarray, ref: np.ndarray, floor: np.ndarray, what: str = ""):
-    """Logits of a deep model: as assert_hidden_close_floor with the 5e-2 logits bound."""
-    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    err = np.abs(got - ref)
-    p99, fp99 = float(np.quantile(err, 0.99)), float(np.quantile(floor, 0.99))
-    tol_max = max(BF16_LOGITS_ABS, FLOOR_FACTOR * float(floor.max()))
-    tol_p99 = max(BF16_LOGITS_ABS, FLOOR_FACTOR * fp99)
-    assert p99 <= tol_p99, f"{what}: p99 abs err {p99:.4g} > {tol_p99:.4g} (oracle floor p99 {fp99:.4g})"
-    assert err.max() <= tol_max, \
-        f"{what}: max abs err {err.max():.4g} > {tol_max:.4g} (oracle floor max {floor.max():.4g})"
+    eemu = np.abs(emu - ref)
+    p99, ep99 = float(np.quantile(err, 0.99)), float(np.quantile(eemu, 0.99))
+    tol_max = max(flat, EMU_FACTOR * float(eemu.max()))
+    tol_p99 = max(flat, EMU_FACTOR * ep99)
+    print(f"[parity] {what}: GPU max {err.max():.4g} p99 {p99:.4g}; fp32 emulation max {eemu.max():.4g} "
+          f"p99 {ep99:.4g}; bound max {tol_max:.4g} p99 {tol_p99:.4g}")
+    assert p99 <= tol_p99, f"{what}: p99 abs err {p99:.4g} > {tol_p99:.4g} (emulation p99 {ep99:.4g})"
+    assert err.max() <= tol_max, f"{what}: max abs err {err.max():.4g} > {tol_max:.4g} (emulation {eemu.max():.4g})"
     return float(err.max()), p99
 
 

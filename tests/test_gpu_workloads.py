@@ -1,14 +1,17 @@
 """Parity at the workloads' full sizes, in the launch configuration the bench
 times (llama_block_forward, batch and positions of the workload), against
-the oracle run on the same seeded inputs."""
+the oracle run on the same seeded inputs. The bound is the flat one (2e-2 on
+hidden states, 5e-2 on logits), or 1.5 x the distance from the oracle of an
+fp32 CPU emulation with the same rounding points (tests/emulation.py) where
+fp32 accumulation alone exceeds the flat bound; both numbers are printed."""
 import numpy as np
 import pytest
 import torch
 
 from llama_decoder_block_kv_b200 import binding as B
 from llama_decoder_block_kv_b200 import synth
-from tests.gpu_util import (PERTURB_REL, CacheSnapshot, Pair, assert_bf16_cache_close, assert_hidden_close_floor,
-                            assert_logits_close_floor, oracle_floor)
+from tests import emulation as E
+from tests.gpu_util import (BF16_HIDDEN_ABS, BF16_LOGITS_ABS, Pair, assert_bf16_cache_close, assert_close_emulated)
 from tests.helpers import t2np
 
 pytestmark = pytest.mark.gpu
@@ -20,31 +23,26 @@ def test_llama7b_layer_prefill_512_then_decode():
     w = synth.LLAMA7B_LAYER
     pair = Pair(w)
     try:
+        em = E.EmuBlock(pair.oracle.layers[0], pair.oracle.args, pair.oracle.cos, pair.oracle.sin)
+        ek = torch.zeros((1, w.max_seq_len, w.n_kv_heads, w.head_dim))
+        ev = torch.zeros_like(ek)
         h = synth.hidden(w, (1, 512, w.dim), 0)
         hd = h.cuda()
         B.llama_block_forward(pair.ctx, 0, hd, 0)
         torch.cuda.synchronize()
         pair.check_error()
-        snap = CacheSnapshot(pair.oracle, [0])
-
-        def run(x):
-            snap.restore()
-            return pair.oracle.block(0, x, 0)
-        ref, floor = oracle_floor(run, t2np(h))
-        assert_hidden_close_floor(t2np(hd), ref, floor, "prefill hidden")
+        ref = pair.oracle.block(0, t2np(h), 0)
+        emu = em.forward(h, ek, ev, 0).double().numpy()
+        assert_close_emulated(t2np(hd), ref, emu, BF16_HIDDEN_ABS, "7B layer prefill 512 hidden")
         hdec = synth.hidden(w, (128, 1, 1, w.dim), 1)
         for i in range(4):
             x = hdec[i].cuda().contiguous()
             B.llama_block_forward(pair.ctx, 0, x, 512 + i)
             torch.cuda.synchronize()
             pair.check_error()
-            snap = CacheSnapshot(pair.oracle, [0])
-
-            def run(xx):
-                snap.restore()
-                return pair.oracle.block(0, xx, 512 + i)
-            r, floor = oracle_floor(run, t2np(hdec[i]))
-            assert_hidden_close_floor(t2np(x), r, floor, f"decode hidden at {512 + i}")
+            r = pair.oracle.block(0, t2np(hdec[i]), 512 + i)
+            e = em.forward(hdec[i], ek, ev, 512 + i).double().numpy()
+            assert_close_emulated(t2np(x), r, e, BF16_HIDDEN_ABS, f"7B layer decode hidden at {512 + i}")
         # the cache rows the calls wrote: slots 0..515 of sequence 0, nothing else
         k, v = pair.kv(0)
         for got, refc in ((k, pair.oracle.cache_k[0]), (v, pair.oracle.cache_v[0])):
@@ -79,13 +77,12 @@ def test_llama70b_layer_decode_batch16_at_4096():
         B.llama_block_forward(pair.ctx, 0, hd, w.cache_len)
         torch.cuda.synchronize()
         pair.check_error()
-        snap = CacheSnapshot(pair.oracle, [0])
-
-        def run(x):
-            snap.restore()
-            return pair.oracle.block(0, x, w.cache_len)
-        ref, floor = oracle_floor(run, t2np(h))
-        assert_hidden_close_floor(t2np(hd), ref, floor, "decode hidden")
+        em = E.EmuBlock(pair.oracle.layers[0], pair.oracle.args, pair.oracle.cos, pair.oracle.sin)
+        ek = torch.from_numpy(pair.oracle.cache_k[0])
+        ev = torch.from_numpy(pair.oracle.cache_v[0])
+        emu = em.forward(h, ek.clone(), ev.clone(), w.cache_len).double().numpy()
+        ref = pair.oracle.block(0, t2np(h), w.cache_len)
+        assert_close_emulated(t2np(hd), ref, emu, BF16_HIDDEN_ABS, "70B layer decode hidden")
         # repeating the step rewrites the same slot: identical result
         hd2 = h.cuda()
         B.llama_block_forward(pair.ctx, 0, hd2, w.cache_len)
@@ -134,26 +131,26 @@ def test_llama3_8b_ragged_decode_sampled_sequences():
     om = O.OracleModel(args)
     h0 = _cpu_f64(enh["tok_embeddings"][toks[seqs].long().cuda()])[:, None, :]
     n = int(L.max()) + 1
-    # the oracle runs the unperturbed embedding and, for the conditioning floor, the
-    # embedding perturbed by 2^-17 relative, layer by layer (weights regenerated per layer)
-    r = np.random.default_rng(0).standard_normal(h0.shape)
-    hs = [h0 * (1.0 + PERTURB_REL * r), h0]
+    # the oracle and the fp32 emulation, layer by layer (weights regenerated per layer),
+    # each over its own copy of the three sequences' histories
+    h = h0
+    he = torch.from_numpy(h0).float()
     for i in range(w.n_layers):
-        om.layers[0] = {k: _cpu_f64(v) for k, v in synth.layer_weights(w, i, device="cuda").items()}
-        ck = synth.cache_values(w, i, 0, full, "cuda")[seqs, :n].float().cpu().numpy()
-        cv = synth.cache_values(w, i, 1, full, "cuda")[seqs, :n].float().cpu().numpy()
-        for j in range(2):
-            om.cache_k[0] = ck.copy()
-            om.cache_v[0] = cv.copy()
-            hs[j] = om.block(0, hs[j], L)
+        lw = synth.layer_weights(w, i, device="cuda")
+        om.layers[0] = {k: _cpu_f64(v) for k, v in lw.items()}
+        ck = synth.cache_values(w, i, 0, full, "cuda")[seqs, :n].float().cpu()
+        cv = synth.cache_values(w, i, 1, full, "cuda")[seqs, :n].float().cpu()
+        om.cache_k[0] = ck.double().numpy()
+        om.cache_v[0] = cv.double().numpy()
+        h = om.block(0, h, L)
+        em = E.EmuBlock(lw, args, om.cos, om.sin)
+        he = em.forward(he, ck, cv, L)
     out = enh["output"]
-    refs = []
-    for hj in hs:
-        xn = O.rmsnorm(hj[:, 0], _cpu_f64(enh["norm"]), w.norm_eps, "bf16")
-        refs.append(np.concatenate([xn @ _cpu_f64(out[v0:v0 + 16384]).T for v0 in range(0, w.vocab_size, 16384)],
-                                   axis=1))
+    xn = O.rmsnorm(h[:, 0], _cpu_f64(enh["norm"]), w.norm_eps, "bf16")
+    ref = np.concatenate([xn @ _cpu_f64(out[v0:v0 + 16384]).T for v0 in range(0, w.vocab_size, 16384)], axis=1)
+    emu = E.lm_head(he[:, 0], enh["norm"], out, w.norm_eps).double().numpy()
     assert np.all(np.isfinite(got))
-    assert_logits_close_floor(got[seqs], refs[1], np.abs(refs[1] - refs[0]), "ragged decode logits")
+    assert_close_emulated(got[seqs], ref, emu, BF16_LOGITS_ABS, "8B ragged decode logits (sequences 0, 1, 31)")
 
 
 def test_llama3_8b_prefill_layer0_sampled_rows():
@@ -184,10 +181,11 @@ def test_llama3_8b_prefill_layer0_sampled_rows():
     lw = {k: _cpu_f64(v) for k, v in lw_dev.items()}
     h64 = _cpu_f64(h)
 
-    def run(x):
-        return O.block_forward_rows(x, lw, 0, args, cos, sin, rows)
-    ref, floor = oracle_floor(run, h64)
-    assert_hidden_close_floor(got, ref, floor, "prefill rows")
+    ref = O.block_forward_rows(h64, lw, 0, args, cos, sin, rows)
+    em = E.EmuBlock(lw_dev, args, cos, sin)
+    ck = torch.zeros((4, 8192, w.n_kv_heads, args.head_dim))
+    emu = em.forward(h.cpu(), ck, torch.zeros_like(ck), 0, rows=rows).double().numpy()
+    assert_close_emulated(got, ref, emu, BF16_HIDDEN_ABS, "8B layer-0 prefill rows")
 
 
 def test_llama3_8b_shapes_reduced_prefill_logits():
@@ -203,6 +201,7 @@ def test_llama3_8b_shapes_reduced_prefill_logits():
         pair.check_error()
         ref = pair.oracle.forward(t2np(tok).astype(np.int64), 0, all_positions=False)
         err = np.abs(t2np(out) - ref)
-        assert err.max() <= 5e-2, f"logits max abs err {err.max():.4g}"
+        print(f"[parity] 8B shapes, 2 layers, 1024-token prefill logits: max {err.max():.4g}")
+        assert err.max() <= BF16_LOGITS_ABS, f"logits max abs err {err.max():.4g}"
     finally:
         pair.close()
