@@ -99,8 +99,9 @@ extern "C" {
  *  interleaved order at load time (dot products q.k are unchanged) and
  *  llama_kv_read/llama_kv_write present K in the half-split order.
  * Rules: dim % n_heads == 0; head_dim = dim / n_heads in {64, 128};
- *  n_heads % n_kv_heads == 0; n_heads / n_kv_heads <= 8 when dtype == LLAMA_BF16,
- *  or a multiple of 8; dim % 64 == 0; all sizes positive.
+ *  n_heads % n_kv_heads == 0 (any ratio n_rep = n_heads / n_kv_heads, as the
+ *  notes' repeat_kv allows; the attention kernels serve a kv head's n_rep query
+ *  heads in groups that divide n_rep); dim % 64 == 0; all sizes positive.
  */
 typedef struct {
   int32_t dim;

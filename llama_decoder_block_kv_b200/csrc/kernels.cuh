@@ -71,22 +71,33 @@ struct GemvPlan {
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
 bool check_gemv_plan(int M, int N, int K, int num_sms);  // host walk of a plan (see gemv.cu)
 // W: [N][K] row-major (tiled = 0) or the library's weight tiles (tiled = 1, tile_weights)
+// wmap (optional): a tensor map of W encoded once by the caller (tiled layout, 128-row boxes); else encoded here
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
-                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st);
+                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
+                             const CUtensorMap* wmap = nullptr);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                        uint32_t b1, uint32_t b2);
 bool make_tmap_weights(CUtensorMap* map, const void* ptr, int tiled, uint64_t N, uint64_t K, uint32_t box_rows);
+// bmap (optional, tiled B only): a tensor map of B encoded once by the caller (128-row boxes)
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
-                           int num_sms, cudaStream_t st);
+                           int num_sms, cudaStream_t st, const CUtensorMap* bmap = nullptr);
 
 // Query heads one decode-attention CTA serves (one kv head's group of n_rep
 // query heads, split into n_rep / hpc groups; an MMA row block holds 16): all of
-// them up to 16, else 16 or 8, whichever divides n_rep (bf16 contexts have
-// n_rep <= 8 or n_rep % 8 == 0).
-inline int decode_heads_per_cta(int n_rep) { return n_rep <= 16 ? n_rep : (n_rep % 16 == 0 ? 16 : 8); }
+// them up to 16, else 16 or 8 when one of them divides n_rep, else the largest
+// divisor of n_rep below 16 (n_rep 20 -> 10, 17 -> 1), so every ratio the pages'
+// repeat_kv allows is served.
+inline int decode_heads_per_cta(int n_rep) {
+  if (n_rep <= 16) return n_rep;
+  if (n_rep % 16 == 0) return 16;
+  if (n_rep % 8 == 0) return 8;
+  int hpc = 15;
+  while (n_rep % hpc) --hpc;
+  return hpc;
+}
 // Query heads one prefill-attention CTA serves: its 128 MMA rows hold 128 / hpc
 // positions x hpc heads, so hpc must divide 128 as well as n_rep: the largest
 // power of two dividing n_rep, at most 8 (n_rep 6 -> 2, n_rep 3, 5, 7 -> 1).

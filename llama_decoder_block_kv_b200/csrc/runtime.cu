@@ -55,6 +55,7 @@ struct llama_ctx {
   void* tok_emb = nullptr;
   void* final_norm = nullptr;
   void* output = nullptr;
+  CUtensorMap map_out;  // the LM head as 128-row x 64-k TMA tiles (bf16)
   bool head_set = false;
   float2* rope = nullptr;
   int* err = nullptr;
@@ -198,7 +199,9 @@ EpiParams epi_base(llama_ctx* c, int kind, int M, int N) {
 // C[M][N] = A[M][K] * W[N][K]^T through the path that suits the shape.
 // W is one of the library's weight matrices: row-major fp32 in fp32 mode,
 // 128 x 64 bf16 tiles (tile_weights) in bf16 mode.
-int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st) {
+// wmap: W's tensor map (tiled layout, 128-row boxes), encoded when the weights were set.
+int gemm(llama_ctx* c, const void* A, const void* W, const CUtensorMap* wmap, int M, int N, int K, const EpiParams& ep,
+         cudaStream_t st) {
   if (!c->bf16) {
     launch_gemm_simt<float>(A, W, M, N, K, ep, st);
     return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -206,11 +209,11 @@ int gemm(llama_ctx* c, const void* A, const void* W, int M, int N, int K, const 
   if (M <= 32 && K % 64 == 0) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st) == cudaSuccess
+    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st, wmap) == cudaSuccess
                ? LLAMA_OK
                : LLAMA_ERR_CUDA;
   }
-  return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st, wmap) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 // elements of one stored weight matrix [N][K]: tiles in bf16 mode, row-major in fp32 mode
@@ -300,7 +303,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.Hkv = c->Hkv;
   e.D = c->D;
   e.S_max = c->S;
-  if ((r = gemm(c, c->xn, Ly.wqkv, M, c->n_qkv, c->dim, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.wqkv, &Ly.map_w[0], M, c->n_qkv, c->dim, e, st))) return r;
 
   cudaError_t ce;
   if (!c->bf16) {
@@ -330,7 +333,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;
   e.ld_out = c->dim;
-  if ((r = gemm(c, c->o, Ly.wo, M, c->dim, HD, e, st))) return r;
+  if ((r = gemm(c, c->o, Ly.wo, &Ly.map_w[1], M, c->dim, HD, e, st))) return r;
 
   if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
                : launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
@@ -338,12 +341,12 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
 
   e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
   e.g_out = c->g;
-  if ((r = gemm(c, c->xn, Ly.w13, M, 2 * c->F, c->dim, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.w13, &Ly.map_w[2], M, 2 * c->F, c->dim, e, st))) return r;
 
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;
   e.ld_out = c->dim;
-  return gemm(c, c->g, Ly.w2, M, c->dim, c->F, e, st);
+  return gemm(c, c->g, Ly.w2, &Ly.map_w[3], M, c->dim, c->F, e, st);
 }
 
 // embedding -> blocks -> final norm -> LM head
@@ -374,7 +377,7 @@ int run_model(llama_ctx* c, const int32_t* tokens, int tok_stride, int B, int T,
   EpiParams e = epi_base(c, EPI_STORE_F32, rows, c->V);
   e.out = logits;
   e.ld_out = c->V;
-  return gemm(c, c->xn, c->output, rows, c->V, c->dim, e, st);
+  return gemm(c, c->xn, c->output, &c->map_out, rows, c->V, c->dim, e, st);
 }
 
 int check_ctx_call(llama_ctx* c, int B, int T) {
@@ -415,7 +418,6 @@ int llama_create(const llama_args* args, llama_ctx** out) {
   const int D = a.dim / a.n_heads;
   if (D != 64 && D != 128) return LLAMA_ERR_INVALID_ARGS;
   const int n_rep = a.n_heads / a.n_kv_heads;
-  if (a.dtype == LLAMA_BF16 && n_rep > 8 && n_rep % 8) return LLAMA_ERR_INVALID_ARGS;
   const int F = ffn_hidden(&a);
   if (F < 0 || F % 64) return LLAMA_ERR_INVALID_ARGS;
   if (a.dtype == LLAMA_FP32 && (size_t)(a.max_seq_len + D) * 4 > 200 * 1024) return LLAMA_ERR_INVALID_ARGS;
@@ -485,6 +487,7 @@ int llama_create(const llama_args* args, llama_ctx** out) {
     if ((r = alloc(&c->tok_emb, (size_t)c->V * c->dim * es))) return fail(r);
     if ((r = alloc(&c->final_norm, round256((size_t)c->dim * es)))) return fail(r);
     if ((r = alloc(&c->output, weight_elems(c, c->V, c->dim) * es))) return fail(r);
+    if (c->bf16 && !make_tmap_weights(&c->map_out, c->output, 1, c->V, c->dim, 128)) return fail(LLAMA_ERR_CUDA);
   }
   std::vector<float2> rt = rope_table(D, 2 * c->S, (double)a.rope_theta);
   if ((r = alloc(reinterpret_cast<void**>(&c->rope), rt.size() * sizeof(float2)))) return fail(r);
@@ -638,10 +641,11 @@ int llama_set_embed_norm_head(llama_ctx* c, const void* tok, const void* norm, c
   const size_t es = c->esz;
   CK(cudaMemcpy(c->tok_emb, tok, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
   CK(cudaMemcpy(c->final_norm, norm, (size_t)c->dim * es, cudaMemcpyDeviceToDevice));
-  if (c->bf16)
+  if (c->bf16) {
     launch_tile_weights(output, c->output, c->V, c->dim, 0);
-  else
+  } else {
     CK(cudaMemcpy(c->output, output, (size_t)c->V * c->dim * es, cudaMemcpyDeviceToDevice));
+  }
   CK(cudaGetLastError());
   CK(cudaDeviceSynchronize());
   c->head_set = true;
@@ -883,7 +887,6 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
 
 int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, int max_seq_len, int num_sms) {
   if (M < 1 || dim < 64 || n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || dim % n_heads || ffn < 64 ||
-      (n_heads / n_kv_heads > 8 && (n_heads / n_kv_heads) % 8) ||
       max_seq_len < 1 || num_sms < 1 || dim % 64 || ffn % 64)
     return LLAMA_ERR_INVALID_ARGS;
   const int D = dim / n_heads, n_qkv = (n_heads + 2 * n_kv_heads) * D;

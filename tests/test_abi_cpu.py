@@ -64,8 +64,9 @@ def test_ffn_hidden_matches_oracle_rule():
     dict(vocab_size=1001),         # vocab % 8
     dict(dtype="fp16"),
     dict(n_heads=32, n_kv_heads=2, dim=4096),  # bf16 GQA group of 16 is fine (multiple of 8)
-    dict(n_heads=12, n_kv_heads=1, dim=768),   # bf16 group of 12: above 8 and not a multiple of 8
+    dict(n_heads=12, n_kv_heads=1, dim=768),   # bf16 group of 12 is fine (any ratio)
     dict(n_heads=24, n_kv_heads=1, dim=1536),  # bf16 group of 24 is fine (three CTA groups of 8)
+    dict(n_heads=20, n_kv_heads=1, dim=1280),  # bf16 group of 20 is fine (two CTA groups of 10)
 ])
 def test_create_rejects_invalid_args_on_host(bad):
     if not os.path.exists(B.LIB_PATH):
@@ -80,7 +81,8 @@ def test_create_rejects_invalid_args_on_host(bad):
         c.dtype = 7
     ctx = ctypes.c_void_p()
     code = B.lib().llama_create(ctypes.byref(c), ctypes.byref(ctx))
-    if bad in (dict(n_heads=32, n_kv_heads=2, dim=4096), dict(n_heads=24, n_kv_heads=1, dim=1536)):
+    if bad in (dict(n_heads=32, n_kv_heads=2, dim=4096), dict(n_heads=24, n_kv_heads=1, dim=1536),
+               dict(n_heads=12, n_kv_heads=1, dim=768), dict(n_heads=20, n_kv_heads=1, dim=1280)):
         # valid shape: without a GPU the failure (if any) comes from CUDA, not validation
         assert code != B.LLAMA_ERR_INVALID_ARGS
         if code == B.LLAMA_OK:

@@ -1,7 +1,8 @@
 """The two decode attention kernels of the per-step launches (LLAMA_ATTN_CHUNKED
 and LLAMA_ATTN_STREAMK) against the oracle: MHA / GQA / MQA head maps (16 query
 heads per kv head: one CTA group of 16; 24 at head_dim 64: three groups of 8;
-3 and 6, where the prefill attention takes groups of 1 and 2), head_dim 64 and
+3 and 6, where the prefill attention takes groups of 1 and 2; 12, 20 and 17,
+served in groups of 12, 10 and 1), head_dim 64 and
 128, scalar and per-sequence positions, histories split over many CTAs (the
 stream-K split cuts one sequence's tiles over up to 16 CTAs), batches of up to
 96 sequences, repeated launches through the same counters, CUDA-graph replay
@@ -75,7 +76,8 @@ def _decode_both(pair, h, start_pos):
 
 @pytest.mark.parametrize("dim,H,Hkv,Bsz", [(512, 4, 2, 1), (512, 4, 4, 2), (1024, 8, 1, 3), (2048, 16, 2, 5),
                                            (1024, 8, 8, 9), (256, 4, 1, 4), (512, 8, 2, 6), (2048, 16, 4, 2),
-                                           (1536, 24, 1, 2), (2048, 16, 1, 3), (768, 6, 2, 2), (768, 12, 2, 3)])
+                                           (1536, 24, 1, 2), (2048, 16, 1, 3), (768, 6, 2, 2), (768, 12, 2, 3),
+                                           (768, 12, 1, 2), (1280, 20, 1, 2), (1088, 17, 1, 2)])
 def test_decode_steps_match_oracle(dim, H, Hkv, Bsz):
     w = _wl(dim, H, Hkv, Bsz)
     pair = Pair(w)
@@ -219,5 +221,38 @@ def test_mode_errors():
         B.llama_set_decode_attention(pair.ctx, B.LLAMA_ATTN_AUTO)
         _step(pair, synth.hidden(w, (2, 4, 512), call=0), 0)
         _step(pair, synth.hidden(w, (2, 1, 512), call=1), 4)
+    finally:
+        pair.close()
+
+
+def test_24_query_heads_per_kv_head_at_head_dim_128():
+    """dim 3072, 24 query heads on one kv head, head_dim 128 (three decode groups
+    of 8, prefill groups of 8): a 70-token prefill and three decode steps through
+    both kernels. At ffn 8192 the fp32 accumulation alone comes near the flat
+    2e-2, so the bound is the one of the full-size tests: the flat one, or 1.5 x
+    the fp32 emulation's distance from the oracle on the same inputs."""
+    from tests import emulation as E
+    from tests.gpu_util import assert_close_emulated
+    w = _wl(3072, 24, 1, 2)
+    pair = Pair(w)
+    try:
+        em = E.EmuBlock(pair.oracle.layers[0], pair.oracle.args, pair.oracle.cos, pair.oracle.sin)
+        ek = torch.zeros((2, w.max_seq_len, 1, 128))
+        ev = torch.zeros_like(ek)
+        h = synth.hidden(w, (2, 70, 3072), call=0)
+        ref = _oracle(pair, h, 0)
+        emu = em.forward(h, ek, ev, 0).double().numpy()
+        assert_close_emulated(_run(pair, h, 0), ref, emu, BF16_HIDDEN_ABS, "dim 3072, 24/1 heads, prefill 70")
+        for i in range(3):
+            h = synth.hidden(w, (2, 1, 3072), call=1 + i)
+            ref = _oracle(pair, h, 70 + i)
+            emu = em.forward(h, ek, ev, 70 + i).double().numpy()
+            outs = []
+            for k in KERNELS:
+                B.llama_set_decode_attention(pair.ctx, k)
+                got = _run(pair, h, 70 + i)
+                assert_close_emulated(got, ref, emu, BF16_HIDDEN_ABS, f"dim 3072 decode {70 + i}, kernel {k}")
+                outs.append(got)
+            assert np.abs(outs[0] - outs[1]).max() <= BF16_HIDDEN_ABS / 2
     finally:
         pair.close()

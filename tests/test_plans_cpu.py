@@ -70,8 +70,14 @@ def test_decode_attention_head_groups_cover_every_head(H, Hkv):
             assert B.llama_selfcheck_plans(M, H * D, H, Hkv, 1024, 2048, 148) == B.LLAMA_OK, (H, Hkv, D, M)
 
 
-def test_selfcheck_rejects_head_ratios_the_library_rejects():
-    assert B.llama_selfcheck_plans(1, 20 * 64, 20, 1, 1024, 256, 148) == B.LLAMA_ERR_INVALID_ARGS  # n_rep 20
+@pytest.mark.parametrize("H,Hkv", [(20, 1), (17, 1), (34, 2), (36, 3), (44, 1), (12, 1), (10, 1), (9, 3)])
+def test_head_groups_of_ratios_that_are_not_multiples_of_eight(H, Hkv):
+    """Ratios above 8 that 8 does not divide (20 -> groups of 10, 17 -> groups
+    of 1, 22 -> 11): every query head in exactly one group of each attention
+    kernel, the prefill's rows holding whole positions."""
+    for D in (64, 128):
+        for M in (1, 5, 32):
+            assert B.llama_selfcheck_plans(M, H * D, H, Hkv, 1024, 512, 148) == B.LLAMA_OK, (H, Hkv, D, M)
 
 
 @pytest.mark.parametrize("H,Hkv", [(3, 1), (5, 1), (6, 1), (7, 1), (12, 4), (24, 8), (30, 5), (48, 6)])
