@@ -276,9 +276,12 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t 
 
 template <int BN>
 static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
-                             int num_sms, cudaStream_t st) {
+                             int num_sms, cudaStream_t st, const CUtensorMap* bmap) {
   CUtensorMap ma, mb;
-  if (!make_tmap_bf16(&ma, A, M, K, BM) || !make_tmap_weights(&mb, B, b_tiled, N, K, b_tiled ? 128 : BN))
+  if (!make_tmap_bf16(&ma, A, M, K, BM)) return cudaErrorInvalidValue;
+  if (bmap && b_tiled)
+    mb = *bmap;  // the library's weights: encoded once when they were set
+  else if (!make_tmap_weights(&mb, B, b_tiled, N, K, b_tiled ? 128 : BN))
     return cudaErrorInvalidValue;
   static std::atomic<unsigned long long> attr{0};
   cudaError_t e = ensure_smem(gemm_tc_kernel<bf16, BN>, TcCfg<BN>::SMEM, attr);
@@ -291,7 +294,7 @@ static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, i
 
 // BN = 256 unless that leaves the last wave badly filled.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
-                           int num_sms, cudaStream_t st) {
+                           int num_sms, cudaStream_t st, const CUtensorMap* bmap) {
   const int num_m = (M + BM - 1) / BM;
   const int t256 = num_m * ((N + 255) / 256);
   const int t128 = num_m * ((N + 127) / 128);
@@ -300,8 +303,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int
     return (double)waves * cost;  // time ~ waves x per-tile cost
   };
   const bool use256 = (N % 256 == 0) && eff(t256, 2.0) <= eff(t128, 1.0) * 1.05;
-  return use256 ? launch_tc<256>(A, B, b_tiled, M, N, K, ep, num_sms, st)
-                : launch_tc<128>(A, B, b_tiled, M, N, K, ep, num_sms, st);
+  return use256 ? launch_tc<256>(A, B, b_tiled, M, N, K, ep, num_sms, st, bmap)
+                : launch_tc<128>(A, B, b_tiled, M, N, K, ep, num_sms, st, bmap);
 }
 
 }  // namespace llama

@@ -334,12 +334,16 @@ static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M
 }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
-                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st) {
+                             float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
+                             const CUtensorMap* wmap) {
   (void)num_sms;
   const int MB = (M + 7) / 8;
   CUtensorMap mw, mx;
-  if (!make_tmap_weights(&mw, W, tiled, N, K, RPC) || !make_tmap_bf16(&mx, X, M, K, 8 * MB))
+  if (wmap && tiled)
+    mw = *wmap;  // the library's weights: encoded once when they were set
+  else if (!make_tmap_weights(&mw, W, tiled, N, K, RPC))
     return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
   switch (MB) {
     case 1: return launch_mb<1>(mw, mx, M, N, p, tiled, part, counters, ep, st);
     case 2: return launch_mb<2>(mw, mx, M, N, p, tiled, part, counters, ep, st);
