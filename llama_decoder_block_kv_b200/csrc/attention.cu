@@ -68,7 +68,20 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* mk, const CUtens
 
 // ============================================================================ decode
 
-template <int D>
+// Transpose of an 8 x 8 matrix of 16-bit values held as a warp fragment (thread
+// t holds row t / 4, columns 2 (t % 4), 2 (t % 4) + 1): afterwards thread t holds
+// row t / 4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// NARROW (a CTA serves at most 8 query heads): S^T = K q^T with the warp's 16
+// keys as the MMA rows and the heads as its 8 columns, and O^T = V^T P^T, so
+// no MMA row is spent on a missing head (half the MMAs and exponentials of the
+// heads-as-rows form kept for groups of 9..16 heads).
+template <int D, bool NARROW>
 __global__ void __launch_bounds__(160)
     attn_decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                        const bf16* __restrict__ q, bf16* __restrict__ o, float* __restrict__ part_o,
@@ -138,134 +151,243 @@ __global__ void __launch_bounds__(160)
   pdl_wait();
   pdl_trigger();
 
-  // query rows: g and g + 8 are heads h0 + g, h0 + g + 8 when inside the group of hpc
-  uint32_t qa[D / 16][4];
-  {
-    const bool v0 = g < hpc, v1 = g + 8 < hpc;
-    const bf16* r0 = q + ((size_t)b * H + h0 + (v0 ? g : 0)) * D;
-    const bf16* r1 = q + ((size_t)b * H + h0 + (v1 ? g + 8 : 0)) * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      qa[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
-      qa[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd) : 0u;
-      qa[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
-      qa[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
-    }
-  }
-  float oacc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const float sl2 = rsqrtf((float)D) * LOG2E;
-
   __shared__ int s_abort;
   if (threadIdx.x == 0) s_abort = 0;
   asm volatile("bar.sync 1, 128;" ::: "memory");
-  for (int j = 0; j < n_tiles; ++j) {
-    const int st = j % STAGES;
-    const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
-    if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) atomicExch(&s_abort, 1);
-      break;
-    }
-    const int key0 = k_begin + j * KT + 16 * warp;  // first key of this warp's 16
-    if (key0 < k_end) {
-      const uint32_t kb = smem_u32(base + st * 2 * TB);
-      const uint32_t vb = kb + TB;
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int mi = lane >> 3;
-        const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
-        const int d = 16 * kk + 8 * (mi & 1);
-        uint32_t bf[4];
-        ldmatrix_x4(bf, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
-        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-        mma_bf16_16816(s[0], qa[kk], b0);
-        mma_bf16_16816(s[1], qa[kk], b1);
-      }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int jn = 0; jn < 2; ++jn)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = s[jn][e] * sl2;
-          if (key0 + 8 * jn + 2 * qd + (e & 1) >= k_end) v = -INFINITY;
-          s[jn][e] = v;
-          if (e < 2)
-            mx0 = fmaxf(mx0, v);
-          else
-            mx1 = fmaxf(mx1, v);
-        }
-      mx0 = quad_max(mx0);
-      mx1 = quad_max(mx1);
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      l0 *= sc0;
-      l1 *= sc1;
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        oacc[i][0] *= sc0;
-        oacc[i][1] *= sc0;
-        oacc[i][2] *= sc1;
-        oacc[i][3] *= sc1;
-      }
-#pragma unroll
-      for (int jn = 0; jn < 2; ++jn) {
-        s[jn][0] = exp2f(s[jn][0] - mn0);
-        s[jn][1] = exp2f(s[jn][1] - mn0);
-        s[jn][2] = exp2f(s[jn][2] - mn1);
-        s[jn][3] = exp2f(s[jn][3] - mn1);
-        l0 += s[jn][0] + s[jn][1];
-        l1 += s[jn][2] + s[jn][3];
-      }
-      // P as a sum of two bf16 parts (hi + lo): the decode kernel is bound by
-      // the cache stream, so the second MMA is free and P keeps ~16 bits.
-      uint32_t ph[4], pl[4];
-      split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
-      split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
-      split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
-      split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
-#pragma unroll
-      for (int jd = 0; jd < D / 8; jd += 2) {
-        const int mi = lane >> 3;
-        const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
-        const int d = 8 * (jd + (mi >> 1));
-        uint32_t bf[4];
-        ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
-        const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-        mma_bf16_16816(oacc[jd], ph, b0);
-        mma_bf16_16816(oacc[jd], pl, b0);
-        mma_bf16_16816(oacc[jd + 1], ph, b1);
-        mma_bf16_16816(oacc[jd + 1], pl, b1);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-  }
-
-  // merge the 4 warps' states through shared memory (the ring is idle now)
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (*(volatile int*)&s_abort) return;  // CTA-uniform
-  l0 = quad_sum(l0);
-  l1 = quad_sum(l1);
   float* sm_o = reinterpret_cast<float*>(base);     // [4][16][D]
   float* sm_m = sm_o + 4 * 16 * D;                  // [4][16]
   float* sm_l = sm_m + 4 * 16;                      // [4][16]
+
+  if constexpr (NARROW) {
+    // ---- keys as MMA rows: thread (g, qd) holds heads 2qd, 2qd + 1 of keys g and g + 8
+    const bool v0 = g < hpc;
+    uint32_t qb[D / 16][2];  // B fragments of q^T: head g, d pairs 2qd (+8) of each 16-d step
+    {
+      const bf16* r0 = q + ((size_t)b * H + h0 + (v0 ? g : 0)) * D;
 #pragma unroll
-  for (int i = 0; i < D / 8; ++i) {
-    sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd] = oacc[i][0];
-    sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd + 1] = oacc[i][1];
-    sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd] = oacc[i][2];
-    sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd + 1] = oacc[i][3];
-  }
-  if (qd == 0) {
-    sm_m[warp * 16 + g] = m0;
-    sm_m[warp * 16 + g + 8] = m1;
-    sm_l[warp * 16 + g] = l0;
-    sm_l[warp * 16 + g + 8] = l1;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qb[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
+        qb[kk][1] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
+      }
+    }
+    float ot[D / 16][4];  // O^T: rows d = 16 i + g (+8), columns heads 2qd, 2qd + 1
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) ot[i][0] = ot[i][1] = ot[i][2] = ot[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2qd, 2qd + 1
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % STAGES;
+      const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) atomicExch(&s_abort, 1);
+        break;
+      }
+      const int key0 = k_begin + j * KT + 16 * warp;  // first key of this warp's 16
+      if (key0 < k_end) {
+        const uint32_t kb = smem_u32(base + st * 2 * TB);
+        const uint32_t vb = kb + TB;
+        float sv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int key = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int d = 16 * kk + 8 * (lane >> 4);
+          uint32_t a[4];
+          ldmatrix_x4(a, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
+          mma_bf16_16816(sv, a, qb[kk]);
+        }
+        sv[0] = key0 + g >= k_end ? -INFINITY : sv[0] * sl2;
+        sv[1] = key0 + g >= k_end ? -INFINITY : sv[1] * sl2;
+        sv[2] = key0 + g + 8 >= k_end ? -INFINITY : sv[2] * sl2;
+        sv[3] = key0 + g + 8 >= k_end ? -INFINITY : sv[3] * sl2;
+        float mx0 = fmaxf(sv[0], sv[2]), mx1 = fmaxf(sv[1], sv[3]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {  // over the 8 key rows g
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        // key0 < k_end: key0 itself is valid, so the maxima are finite
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        l0 *= sc0;
+        l1 *= sc1;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          ot[c][0] *= sc0;
+          ot[c][1] *= sc1;
+          ot[c][2] *= sc0;
+          ot[c][3] *= sc1;
+        }
+        sv[0] = exp2f(sv[0] - mn0);
+        sv[1] = exp2f(sv[1] - mn1);
+        sv[2] = exp2f(sv[2] - mn0);
+        sv[3] = exp2f(sv[3] - mn1);
+        l0 += sv[0] + sv[2];
+        l1 += sv[1] + sv[3];
+        // P^T as B fragments (key pairs 2qd (+8), head g), hi + lo bf16 parts (~16 bits of P)
+        uint32_t h01, l01, h23, l23;
+        split_bf16x2(sv[0], sv[1], h01, l01);
+        split_bf16x2(sv[2], sv[3], h23, l23);
+        const uint32_t bh[2] = {movmatrix_t(h01), movmatrix_t(h23)};
+        const uint32_t bl[2] = {movmatrix_t(l01), movmatrix_t(l23)};
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          const int mi = lane >> 3;
+          const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+          const int d = 16 * c + 8 * (mi & 1);
+          uint32_t a[4];
+          ldmatrix_x4_trans(a, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
+          mma_bf16_16816(ot[c], a, bh);
+          mma_bf16_16816(ot[c], a, bl);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    // merge the 4 warps' states through shared memory (the ring is idle now)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (*(volatile int*)&s_abort) return;  // CTA-uniform
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      sm_o[(warp * 16 + 2 * qd) * D + 16 * c + g] = ot[c][0];
+      sm_o[(warp * 16 + 2 * qd + 1) * D + 16 * c + g] = ot[c][1];
+      sm_o[(warp * 16 + 2 * qd) * D + 16 * c + g + 8] = ot[c][2];
+      sm_o[(warp * 16 + 2 * qd + 1) * D + 16 * c + g + 8] = ot[c][3];
+    }
+    if (g == 0) {
+      sm_m[warp * 16 + 2 * qd] = m0;
+      sm_m[warp * 16 + 2 * qd + 1] = m1;
+      sm_l[warp * 16 + 2 * qd] = l0;
+      sm_l[warp * 16 + 2 * qd + 1] = l1;
+    }
+  } else {
+    // query rows: g and g + 8 are heads h0 + g, h0 + g + 8 when inside the group of hpc
+    uint32_t qa[D / 16][4];
+    {
+      const bool v0 = g < hpc, v1 = g + 8 < hpc;
+      const bf16* r0 = q + ((size_t)b * H + h0 + (v0 ? g : 0)) * D;
+      const bf16* r1 = q + ((size_t)b * H + h0 + (v1 ? g + 8 : 0)) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qa[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
+        qa[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd) : 0u;
+        qa[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
+        qa[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
+      }
+    }
+    float oacc[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % STAGES;
+      const bool ok = mbar_wait(&full[st], (j / STAGES) & 1, err);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) atomicExch(&s_abort, 1);
+        break;
+      }
+      const int key0 = k_begin + j * KT + 16 * warp;  // first key of this warp's 16
+      if (key0 < k_end) {
+        const uint32_t kb = smem_u32(base + st * 2 * TB);
+        const uint32_t vb = kb + TB;
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int mi = lane >> 3;
+          const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+          const int d = 16 * kk + 8 * (mi & 1);
+          uint32_t bf[4];
+          ldmatrix_x4(bf, sw_addr(kb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(s[0], qa[kk], b0);
+          mma_bf16_16816(s[1], qa[kk], b1);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int jn = 0; jn < 2; ++jn)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = s[jn][e] * sl2;
+            if (key0 + 8 * jn + 2 * qd + (e & 1) >= k_end) v = -INFINITY;
+            s[jn][e] = v;
+            if (e < 2)
+              mx0 = fmaxf(mx0, v);
+            else
+              mx1 = fmaxf(mx1, v);
+          }
+        mx0 = quad_max(mx0);
+        mx1 = quad_max(mx1);
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        l0 *= sc0;
+        l1 *= sc1;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          oacc[i][0] *= sc0;
+          oacc[i][1] *= sc0;
+          oacc[i][2] *= sc1;
+          oacc[i][3] *= sc1;
+        }
+#pragma unroll
+        for (int jn = 0; jn < 2; ++jn) {
+          s[jn][0] = exp2f(s[jn][0] - mn0);
+          s[jn][1] = exp2f(s[jn][1] - mn0);
+          s[jn][2] = exp2f(s[jn][2] - mn1);
+          s[jn][3] = exp2f(s[jn][3] - mn1);
+          l0 += s[jn][0] + s[jn][1];
+          l1 += s[jn][2] + s[jn][3];
+        }
+        // P as a sum of two bf16 parts (hi + lo): the decode kernel is bound by
+        // the cache stream, so the second MMA is free and P keeps ~16 bits.
+        uint32_t ph[4], pl[4];
+        split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
+        split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
+        split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
+        split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
+#pragma unroll
+        for (int jd = 0; jd < D / 8; jd += 2) {
+          const int mi = lane >> 3;
+          const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
+          const int d = 8 * (jd + (mi >> 1));
+          uint32_t bf[4];
+          ldmatrix_x4_trans(bf, sw_addr(vb + (d >> 6) * 8192, key, d & 63));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_bf16_16816(oacc[jd], ph, b0);
+          mma_bf16_16816(oacc[jd], pl, b0);
+          mma_bf16_16816(oacc[jd + 1], ph, b1);
+          mma_bf16_16816(oacc[jd + 1], pl, b1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+
+    // merge the 4 warps' states through shared memory (the ring is idle now)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (*(volatile int*)&s_abort) return;  // CTA-uniform
+    l0 = quad_sum(l0);
+    l1 = quad_sum(l1);
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd] = oacc[i][0];
+      sm_o[(warp * 16 + g) * D + 8 * i + 2 * qd + 1] = oacc[i][1];
+      sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd] = oacc[i][2];
+      sm_o[(warp * 16 + g + 8) * D + 8 * i + 2 * qd + 1] = oacc[i][3];
+    }
+    if (qd == 0) {
+      sm_m[warp * 16 + g] = m0;
+      sm_m[warp * 16 + g + 8] = m1;
+      sm_l[warp * 16 + g] = l0;
+      sm_l[warp * 16 + g + 8] = l1;
+    }
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
   for (int e = threadIdx.x; e < hpc * D; e += 128) {
@@ -420,14 +542,17 @@ static cudaError_t decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
                             int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max,
                             const DecodePlan& p, int* err, cudaStream_t st) {
   const size_t smem = 1024 + 3 * 2 * AttnSmem<D>::TILE_BYTES + 64;
-  static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(attn_decode_kernel<D>, smem, attr);
+  const bool narrow = p.hpc <= 8;
+  static std::atomic<unsigned long long> attr{0}, attr_n{0};
+  cudaError_t e = narrow ? ensure_smem(attn_decode_kernel<D, true>, smem, attr_n)
+                         : ensure_smem(attn_decode_kernel<D, false>, smem, attr);
   if (e != cudaSuccess) return e;
   const int n_rep = H / Hkv;
   float* part_o = part;
   float* part_ml = part + (size_t)B * H * p.max_chunks * D;
   dim3 grid(p.max_chunks, B * Hkv * (n_rep / p.hpc));
-  return launch_pdl(attn_decode_kernel<D>, grid, dim3(160), smem, st, mk, mv, reinterpret_cast<const bf16*>(q),
+  return launch_pdl(narrow ? attn_decode_kernel<D, true> : attn_decode_kernel<D, false>, grid, dim3(160), smem, st,
+                    mk, mv, reinterpret_cast<const bf16*>(q),
                     reinterpret_cast<bf16*>(o), part_o, part_ml, counters, sp, sp_scalar, H, Hkv, S_max, p.hpc, p.CK,
                     p.max_chunks, err);
 }

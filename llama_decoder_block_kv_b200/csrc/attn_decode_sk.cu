@@ -78,7 +78,21 @@ __host__ __device__ __forceinline__ SkUnit sk_locate(const int* pb, const int* n
 // floats of one partial: O [hpc][D], then (max, sum) per head, padded to 16 bytes
 __host__ __device__ __forceinline__ int sk_part_stride(int hpc, int D) { return hpc * D + ((2 * hpc + 3) & ~3); }
 
-template <int D>
+// Transpose of an 8 x 8 matrix of 16-bit values held as a warp fragment (thread
+// t holds row t / 4, columns 2 (t % 4), 2 (t % 4) + 1): afterwards thread t holds
+// row t / 4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// NARROW (a unit serves at most 8 query heads): the scores are computed as
+// S^T = K q^T with the 16 keys of a warp as the MMA rows and the heads as its
+// 8 columns, and the output as O^T = V^T P^T (head dimension as rows), so no
+// MMA row is spent on a missing head: half the MMAs and exponentials of the
+// heads-as-rows form, which the wider groups (9..16 heads) keep.
+template <int D, bool NARROW>
 __global__ void __launch_bounds__(160, 2)
     attn_decode_sk_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                           const bf16* __restrict__ q, bf16* __restrict__ o, float* __restrict__ part,
@@ -199,124 +213,234 @@ __global__ void __launch_bounds__(160, 2)
     const int sp = start_pos ? start_pos[u.b] : sp_scalar;
     const int L = max(1, min(sp + 1, S_max));
 
-    uint32_t qa[D / 16][4];
-    {
-      const bf16* r0 = q + ((size_t)u.b * H + h0 + (rv0 ? g : 0)) * D;
-      const bf16* r1 = q + ((size_t)u.b * H + h0 + (rv1 ? g + 8 : 0)) * D;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        qa[kk][0] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
-        qa[kk][1] = rv1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd) : 0u;
-        qa[kk][2] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
-        qa[kk][3] = rv1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
-      }
-    }
-    float oacc[D / 8][4];
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-    int st = 0;
-    for (int i = 0; i < seg_len; ++i, ++j) {
-      st = j % SK_STAGES;
-      const bool ok = wait_or_abort(&full[st], (j / SK_STAGES) & 1, err, abort_flag);
-      const int key0 = (u.t + i) * SKT + 16 * warp;  // first of this warp's 16 keys
-      if (__all_sync(0xffffffffu, ok) && key0 < L) {
-        const uint32_t kb = smem_u32(base + st * 2 * TB), vb = kb + TB;
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    int st = 0;  // the ring stage of the segment's last tile
+    if constexpr (NARROW) {
+      // ---- keys as MMA rows: thread (g, qd) holds heads 2qd, 2qd + 1 of keys g and g + 8
+      uint32_t qb[D / 16][2];  // B fragments of q^T: head g, d pairs 2qd (+8) of each 16-d step
+      {
+        const bf16* r0 = q + ((size_t)u.b * H + h0 + (rv0 ? g : 0)) * D;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const int mi = lane >> 3;
-          const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
-          const int d = 16 * kk + 8 * (mi & 1);
-          uint32_t bf[4];
-          ldmatrix_x4(bf, sk_sw(kb + (d >> 6) * 8192, key, d & 63));
-          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-          mma_bf16_16816(s[0], qa[kk], b0);
-          mma_bf16_16816(s[1], qa[kk], b1);
+          qb[kk][0] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
+          qb[kk][1] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+      }
+      float ot[D / 16][4];  // O^T: rows d = 16 i + g (+8), columns heads 2qd, 2qd + 1
 #pragma unroll
-        for (int jn = 0; jn < 2; ++jn)
+      for (int i = 0; i < D / 16; ++i) ot[i][0] = ot[i][1] = ot[i][2] = ot[i][3] = 0.f;
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2qd, 2qd + 1
+      for (int i = 0; i < seg_len; ++i, ++j) {
+        st = j % SK_STAGES;
+        const bool ok = wait_or_abort(&full[st], (j / SK_STAGES) & 1, err, abort_flag);
+        const int key0 = (u.t + i) * SKT + 16 * warp;  // first of this warp's 16 keys
+        if (__all_sync(0xffffffffu, ok) && key0 < L) {
+          const uint32_t kb = smem_u32(base + st * 2 * TB), vb = kb + TB;
+          float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float v = s[jn][e] * sl2;
-            if (key0 + 8 * jn + 2 * qd + (e & 1) >= L) v = -INFINITY;
-            s[jn][e] = v;
-            if (e < 2)
-              mx0 = fmaxf(mx0, v);
-            else
-              mx1 = fmaxf(mx1, v);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int key = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
+            const int d = 16 * kk + 8 * (lane >> 4);
+            uint32_t a[4];
+            ldmatrix_x4(a, sk_sw(kb + (d >> 6) * 8192, key, d & 63));
+            mma_bf16_16816(s, a, qb[kk]);
           }
-        // key0 < L: the maxima are finite
-        const float mn0 = fmaxf(m0, sk_quad_max(mx0)), mn1 = fmaxf(m1, sk_quad_max(mx1));
-        const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
-        m0 = mn0;
-        m1 = mn1;
-        l0 *= sc0;
-        l1 *= sc1;
+          // scale; keys at or past the history's end are masked
+          s[0] = key0 + g >= L ? -INFINITY : s[0] * sl2;
+          s[1] = key0 + g >= L ? -INFINITY : s[1] * sl2;
+          s[2] = key0 + g + 8 >= L ? -INFINITY : s[2] * sl2;
+          s[3] = key0 + g + 8 >= L ? -INFINITY : s[3] * sl2;
+          float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          oacc[c][0] *= sc0;
-          oacc[c][1] *= sc0;
-          oacc[c][2] *= sc1;
-          oacc[c][3] *= sc1;
+          for (int o = 4; o < 32; o <<= 1) {  // over the 8 key rows g
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          // key0 < L: key0 itself is valid, so the maxima are finite
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+          m0 = mn0;
+          m1 = mn1;
+          l0 *= sc0;
+          l1 *= sc1;
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            ot[c][0] *= sc0;
+            ot[c][1] *= sc1;
+            ot[c][2] *= sc0;
+            ot[c][3] *= sc1;
+          }
+          s[0] = exp2f(s[0] - mn0);
+          s[1] = exp2f(s[1] - mn1);
+          s[2] = exp2f(s[2] - mn0);
+          s[3] = exp2f(s[3] - mn1);
+          l0 += s[0] + s[2];
+          l1 += s[1] + s[3];
+          // P^T as B fragments (key pairs 2qd (+8), head g), hi + lo bf16 parts:
+          // transpose the [key][head] fragments of keys 0-7 and 8-15
+          uint32_t h01, l01, h23, l23;
+          split_bf16x2(s[0], s[1], h01, l01);
+          split_bf16x2(s[2], s[3], h23, l23);
+          const uint32_t bh[2] = {movmatrix_trans(h01), movmatrix_trans(h23)};
+          const uint32_t bl[2] = {movmatrix_trans(l01), movmatrix_trans(l23)};
+          // O^T += V^T P^T over this warp's 16 keys; V^T fragments by transposed loads of V
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            const int mi = lane >> 3;
+            const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+            const int d = 16 * c + 8 * (mi & 1);
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, sk_sw(vb + (d >> 6) * 8192, key, d & 63));
+            mma_bf16_16816(ot[c], a, bh);
+            mma_bf16_16816(ot[c], a, bl);
+          }
         }
-#pragma unroll
-        for (int jn = 0; jn < 2; ++jn) {
-          s[jn][0] = exp2f(s[jn][0] - mn0);
-          s[jn][1] = exp2f(s[jn][1] - mn0);
-          s[jn][2] = exp2f(s[jn][2] - mn1);
-          s[jn][3] = exp2f(s[jn][3] - mn1);
-          l0 += s[jn][0] + s[jn][1];
-          l1 += s[jn][2] + s[jn][3];
-        }
-        // O += P V over this warp's 16 keys, P as hi + lo bf16 parts
-        uint32_t ph[4], pl[4];
-        split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
-        split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
-        split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
-        split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
-#pragma unroll
-        for (int jd = 0; jd < D / 8; jd += 2) {
-          const int mi = lane >> 3;
-          const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
-          const int d = 8 * (jd + (mi >> 1));
-          uint32_t bf[4];
-          ldmatrix_x4_trans(bf, sk_sw(vb + (d >> 6) * 8192, key, d & 63));
-          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-          mma_bf16_16816(oacc[jd], ph, b0);
-          mma_bf16_16816(oacc[jd], pl, b0);
-          mma_bf16_16816(oacc[jd + 1], ph, b1);
-          mma_bf16_16816(oacc[jd + 1], pl, b1);
+        if (i + 1 < seg_len) {  // the segment's last stage is released after the merge below
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[st]);
         }
       }
-      if (i + 1 < seg_len) {  // the segment's last stage is released after the merge below
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
       }
-    }
-    l0 = sk_quad_sum(l0);
-    l1 = sk_quad_sum(l1);
+      // this warp's state -> [warp][head][D] in the stage of the segment's last tile
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      float* so = reinterpret_cast<float*>(base + st * 2 * TB);
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        so[(warp * 16 + 2 * qd) * D + 16 * c + g] = ot[c][0];
+        so[(warp * 16 + 2 * qd + 1) * D + 16 * c + g] = ot[c][1];
+        so[(warp * 16 + 2 * qd) * D + 16 * c + g + 8] = ot[c][2];
+        so[(warp * 16 + 2 * qd + 1) * D + 16 * c + g + 8] = ot[c][3];
+      }
+      if (g == 0) {
+        s_m[warp * 16 + 2 * qd] = m0;
+        s_m[warp * 16 + 2 * qd + 1] = m1;
+        s_l[warp * 16 + 2 * qd] = l0;
+        s_l[warp * 16 + 2 * qd + 1] = l1;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    } else {
+      uint32_t qa[D / 16][4];
+      {
+        const bf16* r0 = q + ((size_t)u.b * H + h0 + (rv0 ? g : 0)) * D;
+        const bf16* r1 = q + ((size_t)u.b * H + h0 + (rv1 ? g + 8 : 0)) * D;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          qa[kk][0] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 2 * qd) : 0u;
+          qa[kk][1] = rv1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 2 * qd) : 0u;
+          qa[kk][2] = rv0 ? *reinterpret_cast<const uint32_t*>(r0 + 16 * kk + 8 + 2 * qd) : 0u;
+          qa[kk][3] = rv1 ? *reinterpret_cast<const uint32_t*>(r1 + 16 * kk + 8 + 2 * qd) : 0u;
+        }
+      }
+      float oacc[D / 8][4];
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    // Merge the four warps' states in the stage of the segment's last tile, which
-    // every warp has finished reading: [4 warps][16 rows][D] floats fill its
-    // 2 x 64 x D bf16 exactly; the (max, sum) pairs go to s_m, s_l.
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    float* sm_o = reinterpret_cast<float*>(base + st * 2 * TB);
+      for (int i = 0; i < seg_len; ++i, ++j) {
+        st = j % SK_STAGES;
+        const bool ok = wait_or_abort(&full[st], (j / SK_STAGES) & 1, err, abort_flag);
+        const int key0 = (u.t + i) * SKT + 16 * warp;  // first of this warp's 16 keys
+        if (__all_sync(0xffffffffu, ok) && key0 < L) {
+          const uint32_t kb = smem_u32(base + st * 2 * TB), vb = kb + TB;
+          float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      *reinterpret_cast<float2*>(sm_o + (warp * 16 + g) * D + 8 * c + 2 * qd) = make_float2(oacc[c][0], oacc[c][1]);
-      *reinterpret_cast<float2*>(sm_o + (warp * 16 + g + 8) * D + 8 * c + 2 * qd) =
-          make_float2(oacc[c][2], oacc[c][3]);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int mi = lane >> 3;
+            const int key = 16 * warp + 8 * (mi >> 1) + (lane & 7);
+            const int d = 16 * kk + 8 * (mi & 1);
+            uint32_t bf[4];
+            ldmatrix_x4(bf, sk_sw(kb + (d >> 6) * 8192, key, d & 63));
+            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+            mma_bf16_16816(s[0], qa[kk], b0);
+            mma_bf16_16816(s[1], qa[kk], b1);
+          }
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int jn = 0; jn < 2; ++jn)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float v = s[jn][e] * sl2;
+              if (key0 + 8 * jn + 2 * qd + (e & 1) >= L) v = -INFINITY;
+              s[jn][e] = v;
+              if (e < 2)
+                mx0 = fmaxf(mx0, v);
+              else
+                mx1 = fmaxf(mx1, v);
+            }
+          // key0 < L: the maxima are finite
+          const float mn0 = fmaxf(m0, sk_quad_max(mx0)), mn1 = fmaxf(m1, sk_quad_max(mx1));
+          const float sc0 = exp2f(m0 - mn0), sc1 = exp2f(m1 - mn1);
+          m0 = mn0;
+          m1 = mn1;
+          l0 *= sc0;
+          l1 *= sc1;
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            oacc[c][0] *= sc0;
+            oacc[c][1] *= sc0;
+            oacc[c][2] *= sc1;
+            oacc[c][3] *= sc1;
+          }
+#pragma unroll
+          for (int jn = 0; jn < 2; ++jn) {
+            s[jn][0] = exp2f(s[jn][0] - mn0);
+            s[jn][1] = exp2f(s[jn][1] - mn0);
+            s[jn][2] = exp2f(s[jn][2] - mn1);
+            s[jn][3] = exp2f(s[jn][3] - mn1);
+            l0 += s[jn][0] + s[jn][1];
+            l1 += s[jn][2] + s[jn][3];
+          }
+          // O += P V over this warp's 16 keys, P as hi + lo bf16 parts
+          uint32_t ph[4], pl[4];
+          split_bf16x2(s[0][0], s[0][1], ph[0], pl[0]);
+          split_bf16x2(s[0][2], s[0][3], ph[1], pl[1]);
+          split_bf16x2(s[1][0], s[1][1], ph[2], pl[2]);
+          split_bf16x2(s[1][2], s[1][3], ph[3], pl[3]);
+#pragma unroll
+          for (int jd = 0; jd < D / 8; jd += 2) {
+            const int mi = lane >> 3;
+            const int key = 16 * warp + 8 * (mi & 1) + (lane & 7);
+            const int d = 8 * (jd + (mi >> 1));
+            uint32_t bf[4];
+            ldmatrix_x4_trans(bf, sk_sw(vb + (d >> 6) * 8192, key, d & 63));
+            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+            mma_bf16_16816(oacc[jd], ph, b0);
+            mma_bf16_16816(oacc[jd], pl, b0);
+            mma_bf16_16816(oacc[jd + 1], ph, b1);
+            mma_bf16_16816(oacc[jd + 1], pl, b1);
+          }
+        }
+        if (i + 1 < seg_len) {  // the segment's last stage is released after the merge below
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[st]);
+        }
+      }
+      l0 = sk_quad_sum(l0);
+      l1 = sk_quad_sum(l1);
+      // this warp's state -> [warp][head][D] in the stage of the segment's last tile
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      float* so = reinterpret_cast<float*>(base + st * 2 * TB);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        *reinterpret_cast<float2*>(so + (warp * 16 + g) * D + 8 * c + 2 * qd) = make_float2(oacc[c][0], oacc[c][1]);
+        *reinterpret_cast<float2*>(so + (warp * 16 + g + 8) * D + 8 * c + 2 * qd) =
+            make_float2(oacc[c][2], oacc[c][3]);
+      }
+      if (qd == 0) {
+        s_m[warp * 16 + g] = m0;
+        s_m[warp * 16 + g + 8] = m1;
+        s_l[warp * 16 + g] = l0;
+        s_l[warp * 16 + g + 8] = l1;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
-    if (qd == 0) {
-      s_m[warp * 16 + g] = m0;
-      s_m[warp * 16 + g + 8] = m1;
-      s_l[warp * 16 + g] = l0;
-      s_l[warp * 16 + g + 8] = l1;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // Merge the four warps' states, held in the stage of the segment's last
+    // tile, which every warp has finished reading: [4 warps][16 rows][D] floats
+    // fill its 2 x 64 x D bf16 exactly; the (max, sum) pairs are in s_m, s_l.
+    float* sm_o = reinterpret_cast<float*>(base + st * 2 * TB);
     const uint32_t P = (uint32_t)pb[u.b] * (uint32_t)HG + (uint32_t)u.zl * (uint32_t)n_u;  // the unit's first tile
     const bool whole = u.t == 0 && seg_len == n_u;
     // Partial state of this CTA for a split unit: slot 2 cta when the unit began
@@ -412,14 +536,14 @@ static size_t sk_smem(int D, int B) {
   return 1024 + (size_t)SK_STAGES * 2 * SKT * D * 2 + 2 * SK_STAGES * 8 + (size_t)(2 * B + 1) * 4;
 }
 
-template <int D>
+template <int D, bool NARROW>
 static cudaError_t decode_sk_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int S_max,
                                const DecodeSkPlan& p, int* err, cudaStream_t st) {
   static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(attn_decode_sk_kernel<D>, sk_smem(D, 1024), attr);
+  cudaError_t e = ensure_smem(attn_decode_sk_kernel<D, NARROW>, sk_smem(D, 1024), attr);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_decode_sk_kernel<D>, dim3(p.grid), dim3(160), sk_smem(D, B), st, mk, mv,
+  return launch_pdl(attn_decode_sk_kernel<D, NARROW>, dim3(p.grid), dim3(160), sk_smem(D, B), st, mk, mv,
                     reinterpret_cast<const bf16*>(q), reinterpret_cast<bf16*>(o), part, counters, sp, sp_scalar, B,
                     H, Hkv, S_max, p.hpc, err);
 }
@@ -428,8 +552,12 @@ cudaError_t launch_attn_decode_sk(const CUtensorMap& mk, const CUtensorMap& mv, 
                                   int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                   const DecodeSkPlan& p, int* err, cudaStream_t st) {
   if (!p.ok) return cudaErrorInvalidValue;
-  if (D == 128) return decode_sk_d<128>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
-  return decode_sk_d<64>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  if (p.hpc <= 8) {
+    if (D == 128) return decode_sk_d<128, true>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+    return decode_sk_d<64, true>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  }
+  if (D == 128) return decode_sk_d<128, false>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
+  return decode_sk_d<64, false>(mk, mv, q, o, part, counters, sp, sp_scalar, B, H, Hkv, S_max, p, err, st);
 }
 
 // Host walk of the split for the given positions, with the kernel's own
