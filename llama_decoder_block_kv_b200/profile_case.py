@@ -3,7 +3,8 @@
   python -m llama_decoder_block_kv_b200.profile_case gemv M N K [--reps R] [--graph]
   python -m llama_decoder_block_kv_b200.profile_case tc   M N K [--reps R]
   python -m llama_decoder_block_kv_b200.profile_case simt M N K [--reps R]
-  python -m llama_decoder_block_kv_b200.profile_case prefill-attn T   (LLaMA-7B layer shape, one block call)
+  python -m llama_decoder_block_kv_b200.profile_case prefill-attn T [--batch B] [--shape 7b|8b]
+                                                     (LLaMA-7B or LLaMA-3-8B layer shape, one block call)
   python -m llama_decoder_block_kv_b200.profile_case decode-attn B L [--decode-attention chunked|streamk|auto]
                                                      (LLaMA-2-70B layer shape, one block call)
 
@@ -28,6 +29,9 @@ def main():
     ap.add_argument("--graph", action="store_true", help="time the launches inside one CUDA graph")
     ap.add_argument("--decode-attention", default="auto", choices=["auto", "chunked", "streamk"],
                     help="decode-attn: the attention kernel of the call (llama_set_decode_attention)")
+    ap.add_argument("--shape", default="7b", choices=["7b", "8b"],
+                    help="prefill-attn: the LLaMA-7B layer (MHA) or the LLaMA-3-8B layer (GQA 32/8)")
+    ap.add_argument("--batch", type=int, default=1, help="prefill-attn: sequences of T tokens")
     ap.add_argument("--row-major", action="store_true",
                     help="gemv / tc: pass the weights row-major instead of in the library's tile layout")
     a = ap.parse_args()
@@ -72,11 +76,15 @@ def main():
               f"{byts / ms / 1e6:.1f} GB/s")
         return
     if a.kind == "prefill-attn":
-        w = synth.LLAMA7B_LAYER
         T = a.sizes[0]
+        if a.shape == "7b":
+            w = synth.LLAMA7B_LAYER.with_(max_batch_size=a.batch, max_seq_len=max(T, 2048))
+        else:
+            w = synth.LLAMA3_8B_PREFILL.with_(n_layers=1, vocab_size=0, max_batch_size=a.batch,
+                                              max_seq_len=max(T, 2048))
         m = B.Llama(B.ModelArgs.from_workload(w))
         B.llama_set_layer(m.ctx, 0, synth.layer_weights(w, 0, device="cuda"))
-        h0 = synth.hidden(w, (1, T, w.dim), 0, "cuda")
+        h0 = synth.hidden(w, (a.batch, T, w.dim), 0, "cuda")
         pos = 0
     else:
         w = synth.LLAMA70B_LAYER

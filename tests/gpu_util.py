@@ -129,9 +129,13 @@ def assert_cache_matches(pair: Pair, layer: int, written: np.ndarray, tol: float
 # same rounding points and fp32 sums on the CPU, and the GPU result must be
 # within the flat bound, or within EMU_FACTOR x the emulation's own distance
 # from the oracle on the same inputs, for the maximum and for the 99th
-# percentile of |error| separately.
+# percentile of |error| separately. The factor is 2: the tensor cores' fp32
+# accumulation of bf16 products is measurably coarser than an IEEE fp32 sum
+# (test_gpu_linear.py prints both against float64: the tcgen05 GEMM's rms
+# error is 15-26 x that of sequential fp32 at K = 4096 .. 11008), so each
+# linear feeds the bf16 rounding points a few more flips than the emulation's.
 
-EMU_FACTOR = 1.5
+EMU_FACTOR = 2.0
 
 
 def assert_close_emulated(got: np.ndarray, ref: np.ndarray, emu: np.ndarray, flat: float, what: str = ""):

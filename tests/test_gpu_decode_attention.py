@@ -229,7 +229,7 @@ def test_24_query_heads_per_kv_head_at_head_dim_128():
     """dim 3072, 24 query heads on one kv head, head_dim 128 (three decode groups
     of 8, prefill groups of 8): a 70-token prefill and three decode steps through
     both kernels. At ffn 8192 the fp32 accumulation alone comes near the flat
-    2e-2, so the bound is the one of the full-size tests: the flat one, or 1.5 x
+    2e-2, so the bound is the one of the full-size tests: the flat one, or 2 x
     the fp32 emulation's distance from the oracle on the same inputs."""
     from tests import emulation as E
     from tests.gpu_util import assert_close_emulated

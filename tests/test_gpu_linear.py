@@ -79,3 +79,27 @@ def test_tiled_weights_give_identical_results(path, M, N, K):
     torch.cuda.synchronize()
     assert torch.equal(y0, y1)
     _check(x, w, y1)
+
+
+@pytest.mark.parametrize("M,N,K,path", [(512, 4096, 4096, B.LLAMA_PATH_TCGEN05), (512, 4096, 11008, B.LLAMA_PATH_TCGEN05),
+                                        (16, 4096, 4096, B.LLAMA_PATH_GEMV), (1, 4096, 11008, B.LLAMA_PATH_GEMV)])
+def test_accumulation_error_against_fp32_orders(M, N, K, path):
+    """How far the tensor-core accumulation is from float64, next to an fp32 CPU
+    sum taken in the same 16-term blocks: printed (the full-size parity bound
+    is sized from it) and held to the GEMM-core tolerance."""
+    x, w = _inputs(M, N, K, torch.bfloat16, 51)
+    y = torch.empty((M, N), device="cuda")
+    B.llama_linear(x, w, y, path)
+    torch.cuda.synchronize()
+    xd, wd = x.double().cpu(), w.double().cpu()
+    ref = (xd @ wd.T).numpy()
+    xf, wf = x.float().cpu(), w.float().cpu()
+    seq = torch.zeros(M, N)
+    for k0 in range(0, K, 16):
+        seq += xf[:, k0:k0 + 16] @ wf[:, k0:k0 + 16].T
+    eg = y.double().cpu().numpy() - ref
+    es = seq.double().numpy() - ref
+    rg, rs = float(np.sqrt(np.mean(eg ** 2))), float(np.sqrt(np.mean(es ** 2)))
+    print(f"[accumulation] M={M} N={N} K={K} path={path}: GPU rms {rg:.3e} max {np.abs(eg).max():.3e}; "
+          f"fp32 16-term blocks rms {rs:.3e} max {np.abs(es).max():.3e}; ratio {rg / rs:.1f}")
+    assert np.abs(eg).max() <= 2e-5 * np.abs(ref).max() + 1e-6

@@ -1,7 +1,7 @@
 """Parity at the workloads' full sizes, in the launch configuration the bench
 times (llama_block_forward, batch and positions of the workload), against
 the oracle run on the same seeded inputs. The bound is the flat one (2e-2 on
-hidden states, 5e-2 on logits), or 1.5 x the distance from the oracle of an
+hidden states, 5e-2 on logits), or 2 x the distance from the oracle of an
 fp32 CPU emulation with the same rounding points (tests/emulation.py) where
 fp32 accumulation alone exceeds the flat bound; both numbers are printed."""
 import numpy as np
