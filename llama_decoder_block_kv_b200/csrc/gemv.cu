@@ -65,14 +65,11 @@ __host__ __device__ __forceinline__ int sk_owner(int x, int total, int grid) {
   return c;
 }
 
-constexpr int NEXT_PREFETCH = 6;  // weight tiles of the next linear brought into L2 per CTA
-
 template <int MB>
 __global__ void __launch_bounds__(160, 1)
     llama_decode_linear_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
                      int N, int nk, int total, int tiled, float* __restrict__ part, int* __restrict__ counters,
-                     EpiParams ep, const __grid_constant__ CUtensorMap map_next, int next_nk, int next_total,
-                     int next_grid) {
+                     EpiParams ep) {
   constexpr int STAGES = stages(MB);
   constexpr uint32_t SB = stage_bytes(MB);
   extern __shared__ uint8_t smem_raw[];
@@ -127,16 +124,6 @@ __global__ void __launch_bounds__(160, 1)
         mbar_arrive_expect_tx(&full[st], SB);
         tma_load_2d(dst, &map_w, &full[st], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
         tma_load_2d(dst + W_BYTES, &map_x, &full[st], ks * KB, 0);
-      }
-      // The next linear's CTA of the same number starts its range with these
-      // tiles: bring them into L2 while this kernel's last stages drain, so its
-      // ring fills from L2 instead of waiting on HBM.
-      if (next_grid > 0 && cta < next_grid && !*abort_flag) {
-        const int nb = sk_begin(cta, next_total, next_grid), ne = sk_begin(cta + 1, next_total, next_grid);
-        for (int y = nb; y < ne && y < nb + NEXT_PREFETCH; ++y) {
-          const int rb = y / next_nk, ks = y - rb * next_nk;
-          tma_prefetch_l2_2d(&map_next, 0, (rb * next_nk + ks) * RPC);
-        }
       }
       // the CTA must not retire while a copy into its shared memory is in flight
       for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, ep.err);
@@ -337,19 +324,18 @@ bool check_gemv_plan(int M, int N, int K, int num_sms) {
 
 template <int MB>
 static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
-                             int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st,
-                             const GemvNext& nx) {
+                             int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
   constexpr size_t smem = gemv_smem(MB);
   static std::atomic<unsigned long long> attr{0};
   cudaError_t e = ensure_smem(llama_decode_linear_kernel<MB>, smem, attr);
   if (e != cudaSuccess) return e;
-  return launch_pdl(llama_decode_linear_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total,
-                    tiled, part, counters, ep, nx.map, nx.nk, nx.total, nx.grid);
+  return launch_pdl(llama_decode_linear_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
+                    counters, ep);
 }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
                              float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
-                             const CUtensorMap* wmap, const GemvNext* next) {
+                             const CUtensorMap* wmap) {
   (void)num_sms;
   const int MB = (M + 7) / 8;
   CUtensorMap mw, mx;
@@ -358,18 +344,11 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int
   else if (!make_tmap_weights(&mw, W, tiled, N, K, RPC))
     return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
-  GemvNext nx;
-  if (next && next->grid > 0) {
-    nx = *next;
-  } else {
-    nx.map = mw;  // a valid map; grid 0 means nothing is prefetched
-    nx.grid = 0;
-  }
   switch (MB) {
-    case 1: return launch_mb<1>(mw, mx, M, N, p, tiled, part, counters, ep, st, nx);
-    case 2: return launch_mb<2>(mw, mx, M, N, p, tiled, part, counters, ep, st, nx);
-    case 3: return launch_mb<3>(mw, mx, M, N, p, tiled, part, counters, ep, st, nx);
-    default: return launch_mb<4>(mw, mx, M, N, p, tiled, part, counters, ep, st, nx);
+    case 1: return launch_mb<1>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    case 2: return launch_mb<2>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    case 3: return launch_mb<3>(mw, mx, M, N, p, tiled, part, counters, ep, st);
+    default: return launch_mb<4>(mw, mx, M, N, p, tiled, part, counters, ep, st);
   }
 }
 

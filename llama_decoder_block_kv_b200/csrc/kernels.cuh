@@ -71,17 +71,10 @@ struct GemvPlan {
 GemvPlan plan_gemv(int M, int N, int K, int num_sms);
 bool check_gemv_plan(int M, int N, int K, int num_sms);  // host walk of a plan (see gemv.cu)
 // W: [N][K] row-major (tiled = 0) or the library's weight tiles (tiled = 1, tile_weights)
-// The linear the stream runs next (tiled weights): its map and split. Each CTA
-// prefetches into L2 the first weight tiles of the same-numbered CTA's range of
-// that linear once it has issued its own last tile.
-struct GemvNext {
-  CUtensorMap map;
-  int nk = 0, total = 0, grid = 0;  // grid == 0: none
-};
 // wmap (optional): a tensor map of W encoded once by the caller (tiled layout, 128-row boxes); else encoded here
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
                              float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
-                             const CUtensorMap* wmap = nullptr, const GemvNext* next = nullptr);
+                             const CUtensorMap* wmap = nullptr);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -201,7 +201,7 @@ EpiParams epi_base(llama_ctx* c, int kind, int M, int N) {
 // 128 x 64 bf16 tiles (tile_weights) in bf16 mode.
 // wmap: W's tensor map (tiled layout, 128-row boxes), encoded when the weights were set.
 int gemm(llama_ctx* c, const void* A, const void* W, const CUtensorMap* wmap, int M, int N, int K, const EpiParams& ep,
-         cudaStream_t st, const GemvNext* next = nullptr) {
+         cudaStream_t st) {
   if (!c->bf16) {
     launch_gemm_simt<float>(A, W, M, N, K, ep, st);
     return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -209,7 +209,7 @@ int gemm(llama_ctx* c, const void* A, const void* W, const CUtensorMap* wmap, in
   if (M <= 32 && K % 64 == 0) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st, wmap, next) == cudaSuccess
+    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st, wmap) == cudaSuccess
                ? LLAMA_OK
                : LLAMA_ERR_CUDA;
   }
@@ -277,35 +277,11 @@ bool use_stream_k(int mode, const DecodeSkPlan& sk, int max_len, int num_sms) {
   return sk.hpc <= 8 && w_max >= 8LL * num_sms;
 }
 
-// The decode linear the stream runs after this one (for the GEMV's L2 hand-off):
-// weight map `w` of layer `ly`, [N][K].
-GemvNext gemv_next(const llama_ctx* c, const Layer& ly, int w, int M, int N, int K) {
-  GemvNext nx;
-  const GemvPlan p = plan_gemv(M, N, K, c->num_sms);
-  nx.map = ly.map_w[w];
-  nx.nk = p.nk;
-  nx.total = p.total;
-  nx.grid = p.grid;
-  return nx;
-}
-
 int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev, int sp_host, cudaStream_t st) {
   Layer& Ly = c->layers[layer];
   const int M = B * T;
   const int HD = c->H * c->D;
   int r;
-  // decode calls: each GEMV hands the next one's first weight tiles to L2
-  const bool gemv = c->bf16 && M <= 32;
-  GemvNext nx[4];
-  if (gemv) {
-    nx[0] = gemv_next(c, Ly, 1, M, c->dim, HD);           // after wqkv: wo
-    nx[1] = gemv_next(c, Ly, 2, M, 2 * c->F, c->dim);     // after wo: w1|w3
-    nx[2] = gemv_next(c, Ly, 3, M, c->dim, c->F);         // after w1|w3: w2
-    if (layer + 1 < c->L)                                 // after w2: the next block's wqkv
-      nx[3] = gemv_next(c, c->layers[layer + 1], 0, M, c->n_qkv, c->dim);
-    else if (c->L == 1)                                   // a single block: the next step's wqkv
-      nx[3] = gemv_next(c, Ly, 0, M, c->n_qkv, c->dim);
-  }
   if (T == 1 && c->decode_mode == LLAMA_DECODE_PERSISTENT) {
     if (!c->bf16 || !c->gbar) return LLAMA_ERR_INVALID_ARGS;
     r = run_block_persistent(c, layer, h, B, sp_dev, sp_host, st);
@@ -327,7 +303,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.Hkv = c->Hkv;
   e.D = c->D;
   e.S_max = c->S;
-  if ((r = gemm(c, c->xn, Ly.wqkv, &Ly.map_w[0], M, c->n_qkv, c->dim, e, st, gemv ? &nx[0] : nullptr))) return r;
+  if ((r = gemm(c, c->xn, Ly.wqkv, &Ly.map_w[0], M, c->n_qkv, c->dim, e, st))) return r;
 
   cudaError_t ce;
   if (!c->bf16) {
@@ -357,7 +333,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;
   e.ld_out = c->dim;
-  if ((r = gemm(c, c->o, Ly.wo, &Ly.map_w[1], M, c->dim, HD, e, st, gemv ? &nx[1] : nullptr))) return r;
+  if ((r = gemm(c, c->o, Ly.wo, &Ly.map_w[1], M, c->dim, HD, e, st))) return r;
 
   if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
                : launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
@@ -365,12 +341,12 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
 
   e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
   e.g_out = c->g;
-  if ((r = gemm(c, c->xn, Ly.w13, &Ly.map_w[2], M, 2 * c->F, c->dim, e, st, gemv ? &nx[2] : nullptr))) return r;
+  if ((r = gemm(c, c->xn, Ly.w13, &Ly.map_w[2], M, 2 * c->F, c->dim, e, st))) return r;
 
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;
   e.ld_out = c->dim;
-  return gemm(c, c->g, Ly.w2, &Ly.map_w[3], M, c->dim, c->F, e, st, gemv ? &nx[3] : nullptr);
+  return gemm(c, c->g, Ly.w2, &Ly.map_w[3], M, c->dim, c->F, e, st);
 }
 
 // embedding -> blocks -> final norm -> LM head
