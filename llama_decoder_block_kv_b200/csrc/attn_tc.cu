@@ -16,11 +16,19 @@
 //   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of two
 //               64-column TMEM buffers, and O += P(j-1) V(j-1) into a D-column
 //               TMEM accumulator (P from shared memory, V read N-major);
-//   warps 2..5  softmax, one thread per query row (its TMEM lane): read the
-//               row of S, mask, exponentiate against a running maximum that is
-//               raised only when a new score exceeds it by more than 2^8 (then
-//               O and the sum are rescaled in TMEM), write P as bf16 into shared
-//               memory; at the end O / sum -> bf16 output.
+//   warps 2..9  softmax, two threads per query row: a warp may only reach
+//               the TMEM lanes of its quarter (warp id mod 4), so warps w and
+//               w + 4 share the 32 rows of one quarter and each takes 32 of the
+//               tile's 64 keys (and half of O's columns). Each thread reads its
+//               half row of S, masks it, and the pair exchanges its row maxima
+//               through shared memory (a 64-thread named barrier per quarter),
+//               so both halves exponentiate against the same running maximum,
+//               which is raised only when a new score exceeds it by more than
+//               2^8 (then O and the sums are rescaled in TMEM); P goes to shared
+//               memory as two bf16 parts (P = P_hi + P_lo, the second the
+//               rounding of the remainder), so O += P_hi V + P_lo V keeps about
+//               16 bits of each probability; at the end O / (sum of both
+//               halves) -> bf16.
 // S(j+1) is computed while the softmax of tile j runs. Key tiles beyond the
 // block's last position are never loaded; the causal predicate masks the rest.
 #include "kernels.cuh"
@@ -29,19 +37,24 @@ namespace llama {
 
 namespace {
 constexpr int KT = 64;       // keys per tile
-constexpr int RING = 3;      // K/V stages
+constexpr int KRING = 4;     // K stages (a K tile is free once S(j) is computed)
+constexpr int VRING = 3;     // V stages (a V tile is free once P(j) V(j) is computed)
 constexpr float LOG2E_TC = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;  // raise the running max only past 2^8
 }  // namespace
 
-template <int D>
+template <int D, bool SPLIT_P>
 struct AttnTcCfg {
   static constexpr int HALVES = D / 64;
   static constexpr uint32_t Q_BYTES = 128 * D * 2;   // two (or one) 128 x 64 boxes
   static constexpr uint32_t KV_BYTES = KT * D * 2;   // one K or one V tile
-  static constexpr uint32_t P_BYTES = 128 * KT * 2;  // 128 rows x 64 keys (two buffers)
-  static constexpr size_t SMEM = 1024 + Q_BYTES + RING * 2 * KV_BYTES + 2 * P_BYTES + 256;
-  static constexpr uint32_t TMEM_COLS = 256;  // S0, S1 (64 columns each), O (D columns)
+  static constexpr uint32_t P_BYTES = 128 * KT * 2;  // 128 rows x 64 keys of bf16
+  // P(j) in bf16, or as P_hi + P_lo, each in bf16 (P_lo = the bf16 rounding of P - P_hi); two buffers
+  static constexpr uint32_t PBUF_BYTES = (SPLIT_P ? 2 : 1) * P_BYTES;
+  // the final (max, sum) of each row in each softmax group: [2 groups][2][128 rows]
+  static constexpr uint32_t RED_BYTES = 2 * 2 * 128 * 4;
+  static constexpr size_t SMEM = 1024 + Q_BYTES + (KRING + VRING) * KV_BYTES + 2 * PBUF_BYTES + RED_BYTES + 512;
+  static constexpr uint32_t TMEM_COLS = 512;  // four 64-column S buffers, then O of each softmax group (D each)
 };
 
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
@@ -89,35 +102,77 @@ __device__ __forceinline__ void tmem_st_32cols(uint32_t taddr, const float* v) {
       : "memory");
 }
 
-template <int D>
-__global__ void __launch_bounds__(192, 1)
+// sm_100 packed fp32 arithmetic: two lanes of a 64-bit register per instruction
+// (halves the FMA-pipe instructions of the softmax), and the 3-input maximum.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub_f2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+constexpr int SOFTMAX_THREADS = 256;  // 8 warps: two groups of four, one thread per query row in each
+constexpr int ATTN_TC_THREADS = 64 + SOFTMAX_THREADS;
+
+template <int D, bool SPLIT_P>
+__global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                            const __grid_constant__ CUtensorMap map_v, bf16* __restrict__ o,
                            const int* __restrict__ start_pos, int sp_scalar, int T, int H, int Hkv, int S_max,
                            int hpc, int* err) {
-  using Cfg = AttnTcCfg<D>;
+  using Cfg = AttnTcCfg<D, SPLIT_P>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sKV = sQ + Cfg::Q_BYTES;                 // RING x (K, V)
-  uint8_t* sP = sKV + RING * 2 * Cfg::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * Cfg::P_BYTES);
+  uint8_t* sK = sQ + Cfg::Q_BYTES;                  // KRING K tiles
+  uint8_t* sV = sK + KRING * Cfg::KV_BYTES;         // VRING V tiles
+  uint8_t* sP = sV + VRING * Cfg::KV_BYTES;         // [group] P buffers (hi, then lo)
+  float* red = reinterpret_cast<float*>(sP + 2 * Cfg::PBUF_BYTES);  // [group][m, l][128 rows]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * Cfg::PBUF_BYTES + Cfg::RED_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;          // [RING]
-  uint64_t* kv_empty = kv_full + RING;   // [RING]
-  uint64_t* s_full = kv_empty + RING;    // [2]
-  uint64_t* s_free = s_full + 2;         // [2]
-  uint64_t* p_full = s_free + 2;         // [2] per P buffer
-  uint64_t* o_done = p_full + 2;         // [2] PV(j) completes o_done[j & 1]
+  uint64_t* k_full = bars + 1;           // [KRING]
+  uint64_t* k_empty = k_full + KRING;    // [KRING]
+  uint64_t* v_full = k_empty + KRING;    // [VRING]
+  uint64_t* v_empty = v_full + VRING;    // [VRING]
+  uint64_t* s_full = v_empty + VRING;    // [4] S buffer (group, slot)
+  uint64_t* s_free = s_full + 4;         // [4]
+  uint64_t* p_full = s_free + 4;         // [2] per group
+  uint64_t* o_done = p_full + 2;         // [2] per group: its latest PV has finished
   uint64_t* drained = o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  uint64_t* fin = drained + 1;           // [4]: the two warps of a lane quarter exchange (m, l)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_rep = H / Hkv, groups = n_rep / hpc;
   const int BQ = 128 / hpc;
-  const int qblk = gridDim.x - 1 - blockIdx.x;  // longest (latest) query blocks first
-  const int z = blockIdx.y;
+  // blocks are dispatched in linear order (x fastest): the query-block index is
+  // the slow dimension, counted down, so the longest (latest) query blocks of
+  // every head start first and the short ones fill the tail
+  const int qblk = gridDim.y - 1 - blockIdx.y;
+  const int z = blockIdx.x;
   const int b = z / (Hkv * groups);
   const int kvh = (z / groups) % Hkv;
   const int grp = z % groups;
@@ -126,19 +181,24 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < RING; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < KRING; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < VRING; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], SOFTMAX_THREADS / 2);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], SOFTMAX_THREADS / 2);
       mbar_init(&o_done[i], 1);
     }
     mbar_init(drained, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&fin[i], 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -158,6 +218,9 @@ __global__ void __launch_bounds__(192, 1)
   const int kv_len = min(sp + q_last + 1, S_max);
   const int n = (kv_len + KT - 1) / KT;
   const int row0 = (b * Hkv + kvh) * S_max;
+  // Key tile j goes to softmax group j & 1 as the group's tile k = j >> 1; its
+  // S lands in TMEM buffer 2 (j & 1) + (k & 1) (64 columns each, columns 0..255),
+  // and P(j) V(j) accumulates into the group's O (columns 256 + 128 (j & 1)).
 
   if (warp == 0) {
     if (lane == 0) {
@@ -169,22 +232,36 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int hf = 0; hf < Cfg::HALVES; ++hf)
         tma_load_3d(sQ + hf * 16384, &map_q, q_full, hf * 64, h0, b * T + q0);
-      int j = 0;
-      for (; j < n; ++j) {
-        const int st = j % RING;
-        if (!wait_or_abort(&kv_empty[st], ((j / RING) & 1) ^ 1, err, abort_flag)) break;
-        uint8_t* k_dst = sKV + st * 2 * Cfg::KV_BYTES;
-        uint8_t* v_dst = k_dst + Cfg::KV_BYTES;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * Cfg::KV_BYTES);
+      // K runs KRING tiles ahead of V: V(j) waits for P(j - VRING) V(j - VRING), and
+      // K(j + KRING) for S(j), which the MMA thread computes tiles ahead of P V
+      auto load_k = [&](int t) -> bool {
+        const int st = t % KRING;
+        if (!wait_or_abort(&k_empty[st], ((t / KRING) & 1) ^ 1, err, abort_flag)) return false;
+        mbar_arrive_expect_tx(&k_full[st], Cfg::KV_BYTES);
 #pragma unroll
-        for (int hf = 0; hf < Cfg::HALVES; ++hf) {
-          tma_load_2d(k_dst + hf * 8192, &map_k, &kv_full[st], hf * 64, row0 + j * KT);
-          tma_load_2d(v_dst + hf * 8192, &map_v, &kv_full[st], hf * 64, row0 + j * KT);
-        }
+        for (int hf = 0; hf < Cfg::HALVES; ++hf)
+          tma_load_2d(sK + st * Cfg::KV_BYTES + hf * 8192, &map_k, &k_full[st], hf * 64, row0 + t * KT);
+        return true;
+      };
+      int nk_issued = 0, nv_issued = 0;
+      bool ok = true;
+      for (; ok && nk_issued < min(n, KRING); ++nk_issued) ok = load_k(nk_issued);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % VRING;
+        if (!(ok = wait_or_abort(&v_empty[st], ((j / VRING) & 1) ^ 1, err, abort_flag))) break;
+        mbar_arrive_expect_tx(&v_full[st], Cfg::KV_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < Cfg::HALVES; ++hf)
+          tma_load_2d(sV + st * Cfg::KV_BYTES + hf * 8192, &map_v, &v_full[st], hf * 64, row0 + j * KT);
+        ++nv_issued;
+        if (nk_issued < n && (ok = load_k(nk_issued))) ++nk_issued;
       }
       // every copy into this CTA's shared memory lands before the CTA can retire
       mbar_wait(q_full, 0, err);
-      for (int i = (j > RING ? j - RING : 0); i < j; ++i) mbar_wait(&kv_full[i % RING], (i / RING) & 1, err);
+      for (int i = (nk_issued > KRING ? nk_issued - KRING : 0); i < nk_issued; ++i)
+        mbar_wait(&k_full[i % KRING], (i / KRING) & 1, err);
+      for (int i = (nv_issued > VRING ? nv_issued - VRING : 0); i < nv_issued; ++i)
+        mbar_wait(&v_full[i % VRING], (i / VRING) & 1, err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -193,37 +270,48 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D) | (1u << 16);  // B (= V) N-major
       const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
       bool ok = wait_or_abort(q_full, 0, err, abort_flag);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int st = j % RING;
-          if (!wait_or_abort(&kv_full[st], (j / RING) & 1, err, abort_flag)) break;
-          if (!wait_or_abort(&s_free[j & 1], ((j >> 1) & 1) ^ 1, err, abort_flag)) break;
+      // S(j) = Q K(j)^T into its buffer once K(j) is in and the group has read that
+      // buffer's previous tile (j - 4); O_g += P(j) V(j) once group j & 1 has written
+      // P(j), which also releases K/V stage j. Order: S(0), S(1), then S(j + 2), PV(j).
+      int js = 0;  // next S to issue
+      for (int j = 0; ok && j < n; ++j) {
+        for (; ok && js < n && js <= j + 2; ++js) {
+          const int st = js % KRING;
+          ok = wait_or_abort(&k_full[st], (js / KRING) & 1, err, abort_flag);
+          const int sb = 2 * (js & 1) + ((js >> 1) & 1);
+          ok = ok && wait_or_abort(&s_free[sb], ((js >> 2) & 1) ^ 1, err, abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sKV + st * 2 * Cfg::KV_BYTES);
+          const uint32_t k_addr = smem_u32(sK + st * Cfg::KV_BYTES);
+          const uint32_t sd = tmem + (uint32_t)(sb * KT);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;   // Q: 16 KB per 64-wide half
             const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;   // K: 8 KB per half
-            tc_mma_bf16(tmem + (j & 1) * KT, make_sw128_desc(q_addr + off), make_sw128_desc(k_addr + koff), idesc_s,
-                        kk > 0 ? 1u : 0u);
+            tc_mma_bf16(sd, make_sw128_desc(q_addr + off), make_sw128_desc(k_addr + koff), idesc_s, kk > 0 ? 1u : 0u);
           }
-          tc_commit(&s_full[j & 1]);
+          tc_commit(&s_full[sb]);
+          tc_commit(&k_empty[st]);
         }
-        if (j >= 1) {
-          const int jp = j - 1, stp = jp % RING;
-          if (!wait_or_abort(&p_full[jp & 1], (jp >> 1) & 1, err, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sKV + stp * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES);
+        if (!ok) break;
+        const int g2 = j & 1, k = j >> 1, st = j % VRING;
+        if (!(ok = wait_or_abort(&v_full[st], (j / VRING) & 1, err, abort_flag))) break;
+        if (!(ok = wait_or_abort(&p_full[g2], k & 1, err, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV + st * Cfg::KV_BYTES);
+        const uint32_t od = tmem + 4 * KT + g2 * D;
 #pragma unroll
-          for (int kk = 0; kk < KT / 16; ++kk) {
-            // A = P (K-major: 128 rows x 64 keys); B = V N-major: 16 keys (2048 B) per step,
-            // 64-wide d blocks 8 KB apart (leading byte offset), 8-key groups 1 KB apart
-            tc_mma_bf16(tmem + 2 * KT, make_sw128_desc(p_addr + (jp & 1) * Cfg::P_BYTES + kk * 32),
-                        make_sw128_desc_lbo(v_addr + kk * 2048, 8192, 1024), idesc_pv, (jp | kk) != 0 ? 1u : 0u);
-          }
-          tc_commit(&o_done[jp & 1]);
-          tc_commit(&kv_empty[stp]);
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          // A = P (K-major: 128 rows x 64 keys); B = V N-major: 16 keys (2048 B) per step,
+          // 64-wide d blocks 8 KB apart (leading byte offset), 8-key groups 1 KB apart.
+          // O += P_hi V + P_lo V: P carries ~16 significant bits into the sum.
+          const uint64_t vdesc = make_sw128_desc_lbo(v_addr + kk * 2048, 8192, 1024);
+          const uint32_t pa = p_addr + g2 * Cfg::PBUF_BYTES + kk * 32;
+          tc_mma_bf16(od, make_sw128_desc(pa), vdesc, idesc_pv, (k | kk) != 0 ? 1u : 0u);
+          if constexpr (SPLIT_P) tc_mma_bf16(od, make_sw128_desc(pa + Cfg::P_BYTES), vdesc, idesc_pv, 1u);
         }
+        tc_commit(&o_done[g2]);
+        tc_commit(&v_empty[st]);
       }
       tc_commit(drained);
       const uint64_t t0 = global_timer_ns();
@@ -233,117 +321,164 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // -------------------------------------------------------------------- softmax
     const int quarter = warp & 3;
+    const int sg = (warp - 2) >> 2;             // softmax group: key tiles j with j & 1 == sg
     const int r = quarter * 32 + lane;          // query row = TMEM lane
     const int pos_l = r / hpc, hl = r - pos_l * hpc;
     const int p_row = sp + min(q0 + pos_l, T - 1);
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t o_cols = lane_base + 4 * KT + sg * D;
     const float sl2 = rsqrtf((float)D) * LOG2E_TC;
+    const uint64_t scale2 = f2(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = wait_or_abort(&s_full[j & 1], (j >> 1) & 1, err, abort_flag);
+    int k = 0;
+    for (int j = sg; j < n; j += 2, ++k) {
+      const int sb = 2 * sg + (k & 1);
+      ok = wait_or_abort(&s_full[sb], (k >> 1) & 1, err, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       float s[KT];
-      tmem_ld_32cols(lane_base + (j & 1) * KT, s);
-      tmem_ld_32cols(lane_base + (j & 1) * KT + 32, s + 32);
+      tmem_ld_32cols(lane_base + sb * KT, s);
+      tmem_ld_32cols(lane_base + sb * KT + 32, s + 32);
       tc_fence_before();
-      mbar_arrive(&s_free[j & 1]);
-      // row maximum of the raw scores (masked keys -inf), four independent chains
+      mbar_arrive(&s_free[sb]);
+      // row maximum of the raw scores (masked keys -inf): two chains of 3-input maxima
       const int key0 = j * KT;
       if (__any_sync(0xffffffffu, key0 + KT - 1 > p_row)) {
 #pragma unroll
         for (int c = 0; c < KT; ++c)
           if (key0 + c > p_row) s[c] = -INFINITY;
       }
-      float mx[4] = {s[0], s[1], s[2], s[3]};
+      float ma = max3f(s[0], s[1], s[2]), mb = max3f(s[3], s[4], s[5]);
 #pragma unroll
-      for (int c = 4; c < KT; c += 4) {
-        mx[0] = fmaxf(mx[0], s[c]);
-        mx[1] = fmaxf(mx[1], s[c + 1]);
-        mx[2] = fmaxf(mx[2], s[c + 2]);
-        mx[3] = fmaxf(mx[3], s[c + 3]);
+      for (int c = 6; c < 62; c += 4) {
+        ma = max3f(ma, s[c], s[c + 1]);
+        mb = max3f(mb, s[c + 2], s[c + 3]);
       }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;  // log2 units
-      // P(j) goes to buffer j & 1, last read by PV(j-2)
-      if (j >= 2) {
-        ok = wait_or_abort(&o_done[j & 1], ((j - 2) >> 1) & 1, err, abort_flag);
+      const float mt = max3f(ma, mb, fmaxf(s[62], s[63])) * sl2;  // log2 units
+      // the group's P buffer was last read by its previous tile's PV
+      if (k >= 1) {
+        ok = wait_or_abort(&o_done[sg], (k - 1) & 1, err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      if (j == 0) {
+      if (k == 0) {
         m_used = mt;
       } else if (__any_sync(0xffffffffu, mt > m_used + RESCALE_LOG2)) {
-        // O is rescaled in TMEM only once PV(j-1) has finished accumulating into it
-        ok = wait_or_abort(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // the group's O has finished accumulating (the wait above): rescale it in TMEM
         const float m_new = fmaxf(m_used, mt);
         const float alpha = exp2f(m_used - m_new);
         l *= alpha;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           float ov[32];
-          tmem_ld_32cols(lane_base + 2 * KT + c, ov);
+          tmem_ld_32cols(o_cols + c, ov);
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tmem_st_32cols(lane_base + 2 * KT + c, ov);
+          tmem_st_32cols(o_cols + c, ov);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         m_used = m_new;
       }
       // P row -> bf16 in the 128-byte-swizzled K-major layout the MMA reads;
-      // p = 2^(s * log2(e)/sqrt(D) - m) is one FMA and one ex2
-      uint8_t* prow = sP + (j & 1) * Cfg::P_BYTES + r * 128;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(s * log2(e)/sqrt(D) - m): one packed FMA per pair and one ex2 each
+      uint8_t* prow = sP + sg * Cfg::PBUF_BYTES + r * 128;
+      // a row may have no visible key yet in this group's tiles (its first tile
+      // lies past the row's position): m_used is then -inf and every score is
+      // -inf, so p = 2^(-inf - 0) = 0 instead of 2^(-inf + inf)
+      const float m_ref = m_used == -INFINITY ? 0.f : m_used;
+      const uint64_t negm2 = f2(-m_ref, -m_ref);
+      uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
       for (int c8 = 0; c8 < KT / 8; ++c8) {
         float pv[8];
+        uint64_t p2[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = ex2_approx(fmaf(s[c8 * 8 + e], sl2, -m_used));
-          ls[e & 3] += pv[e];
+        for (int e = 0; e < 4; ++e) {
+          float t0, t1;
+          f2_split(fma_f2(f2(s[c8 * 8 + 2 * e], s[c8 * 8 + 2 * e + 1]), scale2, negm2), t0, t1);
+          pv[2 * e] = ex2_approx(t0);
+          pv[2 * e + 1] = ex2_approx(t1);
+          p2[e] = f2(pv[2 * e], pv[2 * e + 1]);
+          lsum[e & 1] = add_f2(lsum[e & 1], p2[e]);
         }
-        uint4 u;
-        u.x = pack_bf16x2(pv[0], pv[1]);
-        u.y = pack_bf16x2(pv[2], pv[3]);
-        u.z = pack_bf16x2(pv[4], pv[5]);
-        u.w = pack_bf16x2(pv[6], pv[7]);
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = u;
+        const uint32_t off = (c8 ^ (r & 7)) << 4;
+        if constexpr (SPLIT_P) {
+          // hi = bf16(p) per pair; lo = bf16(p - hi), the remainder taken as one packed subtraction
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hi[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+            float r0, r1;
+            f2_split(sub_f2(p2[e], f2(__uint_as_float(hi[e] << 16), __uint_as_float(hi[e] & 0xFFFF0000u))), r0, r1);
+            lo[e] = pack_bf16x2(r0, r1);
+          }
+          *reinterpret_cast<uint4*>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(prow + Cfg::P_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        } else {
+          *reinterpret_cast<uint4*>(prow + off) =
+              make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
+                         pack_bf16x2(pv[6], pv[7]));
+        }
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      {
+        float a0, a1, b0, b1;
+        f2_split(lsum[0], a0, a1);
+        f2_split(lsum[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[sg]);
     }
-    if (ok) {
-      ok = wait_or_abort(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, err, abort_flag);
+    // the group's last PV has finished (k tiles processed)
+    if (ok && k > 0) {
+      ok = wait_or_abort(&o_done[sg], (k - 1) & 1, err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
+    // (m, l) of both groups for this row (every softmax thread arrives once,
+    // also after a timeout; the wait is bounded all the same)
+    red[(sg * 2) * 128 + r] = m_used;
+    red[(sg * 2 + 1) * 128 + r] = l;
+    mbar_arrive(&fin[quarter]);
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&fin[quarter], 0, err, abort_flag));
     if (ok) {
+      // O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)); group sg
+      // writes columns sg * D/2 .. of the row. A group without tiles has m = -inf and
+      // an O that was never written: its weight is 0 and its columns are not read.
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float m0 = red[0 * 128 + r], l0 = red[1 * 128 + r], m1 = red[2 * 128 + r], l1 = red[3 * 128 + r];
+      const float mm = fmaxf(m0, m1);
+      const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - mm), f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mm);
+      const float inv = 1.f / (l0 * f0 + l1 * f1);
+      const bool has1 = n > 1;  // group 1 had at least one tile
       const bool store = q0 + pos_l < T;
-      bf16* dst = o + ((size_t)(b * T + q0 + pos_l) * H + h0 + hl) * D;
+      bf16* dst = o + ((size_t)(b * T + q0 + pos_l) * H + h0 + hl) * D + sg * (D / 2);
+      const uint32_t oc0 = lane_base + 4 * KT + sg * (D / 2), oc1 = oc0 + D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        float ov[32];
-        tmem_ld_32cols(lane_base + 2 * KT + c, ov);
+      for (int c = 0; c < D / 2; c += 32) {
+        float o0[32];
+        tmem_ld_32cols(oc0 + c, o0);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o0[e] *= f0;
+        if (has1) {
+          float o1[32];
+          tmem_ld_32cols(oc1 + c, o1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o0[e] = fmaf(o1[e], f1, o0[e]);
+        }
         if (store) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             float v8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v8[i] = ov[e + i] * inv;
+            for (int i = 0; i < 8; ++i) v8[i] = o0[e + i] * inv;
             store8(dst + c + e, v8);
           }
         }
@@ -365,19 +500,25 @@ __global__ void __launch_bounds__(192, 1)
 // ordered (token, head), the canonical K-major tile of the MMA.
 static bool make_q_map(CUtensorMap* map, const void* q, int tokens, int H, int D, int hpc);
 
+// P enters the PV product as two bf16 parts (hi + lo): about 16 bits of each
+// probability instead of 8, for one more MMA per 16 keys.
+constexpr bool kSplitP = true;
+
 template <int D>
 static cudaError_t prefill_tc_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
                                 int sp_scalar, int B, int T, int H, int Hkv, int S_max, int* err, cudaStream_t st) {
+  using Cfg = AttnTcCfg<D, kSplitP>;
   const int n_rep = H / Hkv;
   const int hpc = prefill_heads_per_cta(n_rep);
   const int BQ = 128 / hpc;
   CUtensorMap mq;
   if (!make_q_map(&mq, q, B * T, H, D, hpc)) return cudaErrorInvalidValue;
   static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(attn_prefill_tc_kernel<D>, AttnTcCfg<D>::SMEM, attr);
+  cudaError_t e = ensure_smem(attn_prefill_tc_kernel<D, kSplitP>, Cfg::SMEM, attr);
   if (e != cudaSuccess) return e;
-  dim3 grid((T + BQ - 1) / BQ, B * Hkv * (n_rep / hpc));
-  return launch_pdl(attn_prefill_tc_kernel<D>, grid, dim3(192), AttnTcCfg<D>::SMEM, st, mq, mk, mv,
+  dim3 grid(B * Hkv * (n_rep / hpc), (T + BQ - 1) / BQ);
+  if (grid.y > 65535) return cudaErrorInvalidValue;
+  return launch_pdl(attn_prefill_tc_kernel<D, kSplitP>, grid, dim3(ATTN_TC_THREADS), Cfg::SMEM, st, mq, mk, mv,
                     reinterpret_cast<bf16*>(o), sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
 }
 
