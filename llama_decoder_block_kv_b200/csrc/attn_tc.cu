@@ -12,25 +12,30 @@
 // largest power of two (at most 8) dividing n_rep, so the rows hold whole
 // positions and a kv head's n_rep query heads take n_rep / hpc CTAs.
 //   warp 0      TMA: the Q tile once (a 3-D box over [token][head][d]), then
-//               64-key K and V tiles of the cache into a 3-stage ring;
-//   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of two
-//               64-column TMEM buffers, and O += P(j-1) V(j-1) into a D-column
-//               TMEM accumulator (P from shared memory, V read N-major);
-//   warps 2..9  softmax, two threads per query row: a warp may only reach
-//               the TMEM lanes of its quarter (warp id mod 4), so warps w and
-//               w + 4 share the 32 rows of one quarter and each takes 32 of the
-//               tile's 64 keys (and half of O's columns). Each thread reads its
-//               half row of S, masks it, and the pair exchanges its row maxima
-//               through shared memory (a 64-thread named barrier per quarter),
-//               so both halves exponentiate against the same running maximum,
-//               which is raised only when a new score exceeds it by more than
-//               2^8 (then O and the sums are rescaled in TMEM); P goes to shared
-//               memory as two bf16 parts (P = P_hi + P_lo, the second the
-//               rounding of the remainder), so O += P_hi V + P_lo V keeps about
-//               16 bits of each probability; at the end O / (sum of both
-//               halves) -> bf16.
-// S(j+1) is computed while the softmax of tile j runs. Key tiles beyond the
-// block's last position are never loaded; the causal predicate masks the rest.
+//               64-key K tiles into a 4-stage ring and V tiles into a 3-stage
+//               ring (a K tile is free once its S is computed, a V tile once its
+//               P V is, so the two rings run at their own pace);
+//   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of four
+//               64-column TMEM buffers (two per softmax group), and
+//               O_g += P(j) V(j) into group g's D-column TMEM accumulator
+//               (P from shared memory, V read N-major), issuing S two tiles
+//               ahead of P V;
+//   warps 2..9  softmax, two groups of four warps, one thread per query row in
+//               each (a warp reaches only the TMEM lanes of its quarter, warp id
+//               mod 4). Group g takes the key tiles j with j mod 2 = g, keeping
+//               its own running maximum, sum and O, so while one group
+//               exponentiates its tile the other reads or waits for the next S.
+//               A thread reads its row of S, masks it, raises its running
+//               maximum only when a score exceeds it by more than 2^8 (O and the
+//               sum are then rescaled in TMEM), and writes P to shared memory as
+//               two bf16 parts (P = P_hi + P_lo, the second the rounding of the
+//               remainder), so O += P_hi V + P_lo V keeps about 16 bits of each
+//               probability. At the end the two groups exchange (max, sum) per
+//               row through shared memory and each writes half of the row's
+//               O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m))
+//               as bf16.
+// Key tiles beyond the block's last position are never loaded; the causal
+// predicate masks the rest.
 #include "kernels.cuh"
 
 namespace llama {
