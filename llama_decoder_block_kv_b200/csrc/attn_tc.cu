@@ -12,14 +12,17 @@
 // largest power of two (at most 8) dividing n_rep, so the rows hold whole
 // positions and a kv head's n_rep query heads take n_rep / hpc CTAs.
 //   warp 0      TMA: the Q tile once (a 3-D box over [token][head][d]), then
-//               64-key K tiles into a 4-stage ring and V tiles into a 3-stage
-//               ring (a K tile is free once its S is computed, a V tile once its
-//               P V is, so the two rings run at their own pace);
+//               64-key K tiles and V tiles into two 4-stage rings (a K tile is
+//               free once its S is computed, a V tile once its P V is, so the
+//               two rings run at their own pace);
 //   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of four
 //               64-column TMEM buffers (two per softmax group), and
-//               O_g += P(j) V(j) into group g's D-column TMEM accumulator
-//               (P from shared memory, V read N-major), issuing S two tiles
-//               ahead of P V;
+//               O_g += P(j) V(j) into group g's D-column TMEM accumulator with
+//               P(j) read from TMEM, where the softmax wrote it over S(j), and V
+//               read N-major from shared memory; S is issued two tiles ahead.
+//               Only the B operands (K, V) then come from shared memory: with
+//               both operands there, operand reads, not the MMA math, set
+//               the pace;
 //   warps 2..9  softmax, two groups of four warps, one thread per query row in
 //               each (a warp reaches only the TMEM lanes of its quarter, warp id
 //               mod 4). Group g takes the key tiles j with j mod 2 = g, keeping
@@ -27,13 +30,16 @@
 //               exponentiates its tile the other reads or waits for the next S.
 //               A thread reads its row of S, masks it, raises its running
 //               maximum only when a score exceeds it by more than 2^8 (O and the
-//               sum are then rescaled in TMEM), and writes P to shared memory as
-//               two bf16 parts (P = P_hi + P_lo, the second the rounding of the
+//               sum are then rescaled in TMEM), and writes P over S as two bf16
+//               parts (P = P_hi + P_lo, the second the rounding of the
 //               remainder), so O += P_hi V + P_lo V keeps about 16 bits of each
 //               probability. At the end the two groups exchange (max, sum) per
 //               row through shared memory and each writes half of the row's
 //               O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m))
 //               as bf16.
+// A buffer holds S(j), then P(j), until P(j) V(j) has finished; S(j + 4) waits
+// for that (s_free). P has one barrier per buffer, since a group can write
+// P(j + 2) into its other buffer before P(j) V(j) is issued.
 // Key tiles beyond the block's last position are never loaded; the causal
 // predicate masks the rest.
 #include "kernels.cuh"
@@ -43,7 +49,7 @@ namespace llama {
 namespace {
 constexpr int KT = 64;       // keys per tile
 constexpr int KRING = 4;     // K stages (a K tile is free once S(j) is computed)
-constexpr int VRING = 3;     // V stages (a V tile is free once P(j) V(j) is computed)
+constexpr int VRING = 4;     // V stages (a V tile is free once P(j) V(j) is computed)
 constexpr float LOG2E_TC = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;  // raise the running max only past 2^8
 }  // namespace
@@ -53,14 +59,50 @@ struct AttnTcCfg {
   static constexpr int HALVES = D / 64;
   static constexpr uint32_t Q_BYTES = 128 * D * 2;   // two (or one) 128 x 64 boxes
   static constexpr uint32_t KV_BYTES = KT * D * 2;   // one K or one V tile
-  static constexpr uint32_t P_BYTES = 128 * KT * 2;  // 128 rows x 64 keys of bf16
-  // P(j) in bf16, or as P_hi + P_lo, each in bf16 (P_lo = the bf16 rounding of P - P_hi); two buffers
-  static constexpr uint32_t PBUF_BYTES = (SPLIT_P ? 2 : 1) * P_BYTES;
   // the final (max, sum) of each row in each softmax group: [2 groups][2][128 rows]
   static constexpr uint32_t RED_BYTES = 2 * 2 * 128 * 4;
-  static constexpr size_t SMEM = 1024 + Q_BYTES + (KRING + VRING) * KV_BYTES + 2 * PBUF_BYTES + RED_BYTES + 512;
-  static constexpr uint32_t TMEM_COLS = 512;  // four 64-column S buffers, then O of each softmax group (D each)
+  static constexpr size_t SMEM = 1024 + Q_BYTES + (KRING + VRING) * KV_BYTES + RED_BYTES + 512;
+  // four 64-column S buffers (P(j) is written over S(j): 32 columns of bf16 pairs
+  // for P_hi, then 32 for P_lo), then O of each softmax group (D columns each)
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t P_LO_COL = 32;
 };
+
+// D[tmem] (+)= A[tmem] * B[smem]: A = 128 rows (TMEM lanes) x 16 bf16 (8 columns of
+// bf16 pairs, K-major), B by shared-memory descriptor, fp32 accumulation.
+__device__ __forceinline__ void tc_mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 64 consecutive TMEM columns of this thread's lane: two loads, one wait
+__device__ __forceinline__ void tmem_ld_64cols(uint32_t taddr, float* v) {
+  uint32_t r[64];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[32 * h + 0]), "=r"(r[32 * h + 1]), "=r"(r[32 * h + 2]), "=r"(r[32 * h + 3]),
+          "=r"(r[32 * h + 4]), "=r"(r[32 * h + 5]), "=r"(r[32 * h + 6]), "=r"(r[32 * h + 7]),
+          "=r"(r[32 * h + 8]), "=r"(r[32 * h + 9]), "=r"(r[32 * h + 10]), "=r"(r[32 * h + 11]),
+          "=r"(r[32 * h + 12]), "=r"(r[32 * h + 13]), "=r"(r[32 * h + 14]), "=r"(r[32 * h + 15]),
+          "=r"(r[32 * h + 16]), "=r"(r[32 * h + 17]), "=r"(r[32 * h + 18]), "=r"(r[32 * h + 19]),
+          "=r"(r[32 * h + 20]), "=r"(r[32 * h + 21]), "=r"(r[32 * h + 22]), "=r"(r[32 * h + 23]),
+          "=r"(r[32 * h + 24]), "=r"(r[32 * h + 25]), "=r"(r[32 * h + 26]), "=r"(r[32 * h + 27]),
+          "=r"(r[32 * h + 28]), "=r"(r[32 * h + 29]), "=r"(r[32 * h + 30]), "=r"(r[32 * h + 31])
+        : "r"(taddr + 32 * h)
+        : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {
@@ -153,18 +195,19 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
   uint8_t* sQ = base;
   uint8_t* sK = sQ + Cfg::Q_BYTES;                  // KRING K tiles
   uint8_t* sV = sK + KRING * Cfg::KV_BYTES;         // VRING V tiles
-  uint8_t* sP = sV + VRING * Cfg::KV_BYTES;         // [group] P buffers (hi, then lo)
-  float* red = reinterpret_cast<float*>(sP + 2 * Cfg::PBUF_BYTES);  // [group][m, l][128 rows]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * Cfg::PBUF_BYTES + Cfg::RED_BYTES);
+  float* red = reinterpret_cast<float*>(sV + VRING * Cfg::KV_BYTES);  // [group][m, l][128 rows]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VRING * Cfg::KV_BYTES + Cfg::RED_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;           // [KRING]
   uint64_t* k_empty = k_full + KRING;    // [KRING]
   uint64_t* v_full = k_empty + KRING;    // [VRING]
   uint64_t* v_empty = v_full + VRING;    // [VRING]
-  uint64_t* s_full = v_empty + VRING;    // [4] S buffer (group, slot)
-  uint64_t* s_free = s_full + 4;         // [4]
-  uint64_t* p_full = s_free + 4;         // [2] per group
-  uint64_t* o_done = p_full + 2;         // [2] per group: its latest PV has finished
+  uint64_t* s_full = v_empty + VRING;    // [4] S buffer (group, slot) holds S(j)
+  uint64_t* s_free = s_full + 4;         // [4] ... and P(j) V(j), which read P(j) there, has finished
+  // [4] per S buffer: P written over its S (one barrier per buffer: a group may
+  // write P(j + 2) into its other buffer before the MMA thread has taken P(j))
+  uint64_t* p_full = s_free + 4;
+  uint64_t* o_done = p_full + 4;         // [2] per group: its latest PV has finished
   uint64_t* drained = o_done + 2;
   uint64_t* fin = drained + 1;           // [4]: the two warps of a lane quarter exchange (m, l)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 4);
@@ -196,12 +239,10 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], SOFTMAX_THREADS / 2);
-    }
-    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_free[i], 1);
       mbar_init(&p_full[i], SOFTMAX_THREADS / 2);
-      mbar_init(&o_done[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(drained, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&fin[i], 64);
     *abort_flag = 0;
@@ -273,11 +314,12 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       // ------------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = make_idesc_bf16(128, KT);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D) | (1u << 16);  // B (= V) N-major
-      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+      const uint32_t q_addr = smem_u32(sQ);
       bool ok = wait_or_abort(q_full, 0, err, abort_flag);
-      // S(j) = Q K(j)^T into its buffer once K(j) is in and the group has read that
-      // buffer's previous tile (j - 4); O_g += P(j) V(j) once group j & 1 has written
-      // P(j), which also releases K/V stage j. Order: S(0), S(1), then S(j + 2), PV(j).
+      // S(j) = Q K(j)^T into buffer 2 (j & 1) + ((j >> 1) & 1) once K(j) is in and
+      // P(j - 4) V(j - 4), which read that buffer last, has finished; O_g += P(j) V(j)
+      // once group j & 1 has written P(j) over S(j). Order: S(0), S(1), then S(j + 2),
+      // PV(j) for each j, so S(j + 2) waits for PV(j - 2), issued two steps earlier.
       int js = 0;  // next S to issue
       for (int j = 0; ok && j < n; ++j) {
         for (; ok && js < n && js <= j + 2; ++js) {
@@ -300,22 +342,25 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
         }
         if (!ok) break;
         const int g2 = j & 1, k = j >> 1, st = j % VRING;
+        const int sb = 2 * g2 + (k & 1);
         if (!(ok = wait_or_abort(&v_full[st], (j / VRING) & 1, err, abort_flag))) break;
-        if (!(ok = wait_or_abort(&p_full[g2], k & 1, err, abort_flag))) break;
+        if (!(ok = wait_or_abort(&p_full[sb], (k >> 1) & 1, err, abort_flag))) break;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * Cfg::KV_BYTES);
         const uint32_t od = tmem + 4 * KT + g2 * D;
+        const uint32_t pa = tmem + (uint32_t)(sb * KT);
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
-          // A = P (K-major: 128 rows x 64 keys); B = V N-major: 16 keys (2048 B) per step,
-          // 64-wide d blocks 8 KB apart (leading byte offset), 8-key groups 1 KB apart.
+          // A = P from TMEM (128 lanes x 16 keys = 8 columns of bf16 pairs per step);
+          // B = V N-major: 16 keys (2048 B) per step, 64-wide d blocks 8 KB apart
+          // (leading byte offset), 8-key groups 1 KB apart.
           // O += P_hi V + P_lo V: P carries ~16 significant bits into the sum.
           const uint64_t vdesc = make_sw128_desc_lbo(v_addr + kk * 2048, 8192, 1024);
-          const uint32_t pa = p_addr + g2 * Cfg::PBUF_BYTES + kk * 32;
-          tc_mma_bf16(od, make_sw128_desc(pa), vdesc, idesc_pv, (k | kk) != 0 ? 1u : 0u);
-          if constexpr (SPLIT_P) tc_mma_bf16(od, make_sw128_desc(pa + Cfg::P_BYTES), vdesc, idesc_pv, 1u);
+          tc_mma_bf16_tmem_a(od, pa + kk * 8, vdesc, idesc_pv, (k | kk) != 0 ? 1u : 0u);
+          if constexpr (SPLIT_P) tc_mma_bf16_tmem_a(od, pa + Cfg::P_LO_COL + kk * 8, vdesc, idesc_pv, 1u);
         }
         tc_commit(&o_done[g2]);
+        tc_commit(&s_free[sb]);
         tc_commit(&v_empty[st]);
       }
       tc_commit(drained);
@@ -346,10 +391,7 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       }
       tc_fence_after();
       float s[KT];
-      tmem_ld_32cols(lane_base + sb * KT, s);
-      tmem_ld_32cols(lane_base + sb * KT + 32, s + 32);
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
+      tmem_ld_64cols(lane_base + sb * KT, s);
       // row maximum of the raw scores (masked keys -inf): two chains of 3-input maxima
       const int key0 = j * KT;
       if (__any_sync(0xffffffffu, key0 + KT - 1 > p_row)) {
@@ -364,19 +406,18 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
         mb = max3f(mb, s[c + 2], s[c + 3]);
       }
       const float mt = max3f(ma, mb, fmaxf(s[62], s[63])) * sl2;  // log2 units
-      // the group's P buffer was last read by its previous tile's PV
-      if (k >= 1) {
+      if (k == 0) {
+        m_used = mt;
+      } else if (__any_sync(0xffffffffu, mt > m_used + RESCALE_LOG2)) {
+        // rescale the group's O in TMEM once its previous PV has finished (S(j) being
+        // here means PV(j - 4), the group's tile before last, has finished, so the
+        // phase waited for is the latest one or the next)
         ok = wait_or_abort(&o_done[sg], (k - 1) & 1, err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-      if (k == 0) {
-        m_used = mt;
-      } else if (__any_sync(0xffffffffu, mt > m_used + RESCALE_LOG2)) {
-        // the group's O has finished accumulating (the wait above): rescale it in TMEM
         const float m_new = fmaxf(m_used, mt);
         const float alpha = exp2f(m_used - m_new);
         l *= alpha;
@@ -391,62 +432,49 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         m_used = m_new;
       }
-      // P row -> bf16 in the 128-byte-swizzled K-major layout the MMA reads;
-      // p = 2^(s * log2(e)/sqrt(D) - m): one packed FMA per pair and one ex2 each
-      uint8_t* prow = sP + sg * Cfg::PBUF_BYTES + r * 128;
-      // a row may have no visible key yet in this group's tiles (its first tile
+      // P row -> bf16 pairs written over this row's S in TMEM (column c holds keys
+      // 2c, 2c + 1, the K-major A layout of the PV MMA); P_lo 32 columns further on.
+      // p = 2^(s * log2(e)/sqrt(D) - m): one packed FMA per pair and one ex2 each.
+      // A row may have no visible key yet in this group's tiles (its first tile
       // lies past the row's position): m_used is then -inf and every score is
       // -inf, so p = 2^(-inf - 0) = 0 instead of 2^(-inf + inf)
       const float m_ref = m_used == -INFINITY ? 0.f : m_used;
       const uint64_t negm2 = f2(-m_ref, -m_ref);
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+      float ph[KT / 2], plo[SPLIT_P ? KT / 2 : 1];
 #pragma unroll
-      for (int c8 = 0; c8 < KT / 8; ++c8) {
-        float pv[8];
-        uint64_t p2[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float t0, t1;
-          f2_split(fma_f2(f2(s[c8 * 8 + 2 * e], s[c8 * 8 + 2 * e + 1]), scale2, negm2), t0, t1);
-          pv[2 * e] = ex2_approx(t0);
-          pv[2 * e + 1] = ex2_approx(t1);
-          p2[e] = f2(pv[2 * e], pv[2 * e + 1]);
-          lsum[e & 1] = add_f2(lsum[e & 1], p2[e]);
-        }
-        const uint32_t off = (c8 ^ (r & 7)) << 4;
+      for (int e = 0; e < KT / 2; ++e) {
+        float t0, t1;
+        f2_split(fma_f2(f2(s[2 * e], s[2 * e + 1]), scale2, negm2), t0, t1);
+        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+        const uint64_t p2 = f2(p0, p1);
+        lsum[e & 1] = add_f2(lsum[e & 1], p2);
+        const uint32_t hi = pack_bf16x2(p0, p1);
+        ph[e] = __uint_as_float(hi);
         if constexpr (SPLIT_P) {
-          // hi = bf16(p) per pair; lo = bf16(p - hi), the remainder taken as one packed subtraction
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-            float r0, r1;
-            f2_split(sub_f2(p2[e], f2(__uint_as_float(hi[e] << 16), __uint_as_float(hi[e] & 0xFFFF0000u))), r0, r1);
-            lo[e] = pack_bf16x2(r0, r1);
-          }
-          *reinterpret_cast<uint4*>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(prow + Cfg::P_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        } else {
-          *reinterpret_cast<uint4*>(prow + off) =
-              make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
-                         pack_bf16x2(pv[6], pv[7]));
+          // lo = bf16(p - hi), the remainder taken as one packed subtraction
+          float r0, r1;
+          f2_split(sub_f2(p2, f2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u))), r0, r1);
+          plo[e] = __uint_as_float(pack_bf16x2(r0, r1));
         }
       }
+      const uint32_t p_cols = lane_base + sb * KT;
+      tmem_st_32cols(p_cols, ph);
+      if constexpr (SPLIT_P) tmem_st_32cols(p_cols + Cfg::P_LO_COL, plo);
       {
         float a0, a1, b0, b1;
         f2_split(lsum[0], a0, a1);
         f2_split(lsum[1], b0, b1);
         l += (a0 + a1) + (b0 + b1);
       }
-      fence_proxy_async_smem();
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[sg]);
+      mbar_arrive(&p_full[sb]);
     }
-    // the group's last PV has finished (k tiles processed)
-    if (ok && k > 0) {
-      ok = wait_or_abort(&o_done[sg], (k - 1) & 1, err, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-    }
+    // every MMA of the CTA has finished (the MMA thread commits `drained` once,
+    // after its last PV): both groups' O are complete. A wait on o_done could not
+    // tell here whether one or two of the group's PVs are still running.
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(drained, 0, err, abort_flag));
     // (m, l) of both groups for this row (every softmax thread arrives once,
     // also after a timeout; the wait is bounded all the same)
     red[(sg * 2) * 128 + r] = m_used;
