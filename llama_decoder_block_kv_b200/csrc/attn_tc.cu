@@ -12,60 +12,55 @@
 // largest power of two (at most 8) dividing n_rep, so the rows hold whole
 // positions and a kv head's n_rep query heads take n_rep / hpc CTAs.
 //   warp 0      TMA: the Q tile once (a 3-D box over [token][head][d]), then
-//               64-key K tiles and V tiles into two 4-stage rings (a K tile is
-//               free once its S is computed, a V tile once its P V is, so the
-//               two rings run at their own pace);
-//   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into one of four
-//               64-column TMEM buffers (two per softmax group), and
-//               O_g += P(j) V(j) into group g's D-column TMEM accumulator with
-//               P(j) read from TMEM, where the softmax wrote it over S(j), and V
-//               read N-major from shared memory; S is issued two tiles ahead.
-//               Only the B operands (K, V) then come from shared memory: with
-//               both operands there, operand reads, not the MMA math, set
-//               the pace;
-//   warps 2..9  softmax, two groups of four warps, one thread per query row in
-//               each (a warp reaches only the TMEM lanes of its quarter, warp id
-//               mod 4). Group g takes the key tiles j with j mod 2 = g, keeping
-//               its own running maximum, sum and O, so while one group
-//               exponentiates its tile the other reads or waits for the next S.
-//               A thread reads its row of S, masks it, raises its running
-//               maximum only when a score exceeds it by more than 2^8 (O and the
-//               sum are then rescaled in TMEM), and writes P over S as two bf16
-//               parts (P = P_hi + P_lo, the second the rounding of the
-//               remainder), so O += P_hi V + P_lo V keeps about 16 bits of each
-//               probability. At the end the two groups exchange (max, sum) per
-//               row through shared memory and each writes half of the row's
-//               O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m))
-//               as bf16.
-// A buffer holds S(j), then P(j), until P(j) V(j) has finished; S(j + 4) waits
-// for that (s_free). P has one barrier per buffer, since a group can write
-// P(j + 2) into its other buffer before P(j) V(j) is issued.
-// Key tiles beyond the block's last position are never loaded; the causal
-// predicate masks the rest.
+//               128-key K tiles into a 2-stage ring and V tiles into a 3-stage
+//               ring (a K tile is free once its S is computed, a V tile once its
+//               P V is);
+//   warp 1      TMEM owner and MMA issuer: S(j) = Q K(j)^T into TMEM buffer
+//               j mod 3 (128 columns), and O += P(j) V(j) into a D-column TMEM
+//               accumulator, with P(j) read from TMEM, where the softmax wrote it
+//               over S(j), and V read N-major from shared memory. S(j + 1) is
+//               issued before P(j) V(j), so the softmax of one tile runs under
+//               the P V MMAs of the one before;
+//   warps 2..5  softmax, one thread per query row (its TMEM lane; a warp
+//               reaches only the lanes of its quarter, warp id mod 4). A thread
+//               reads its row of S, masks it, raises its running maximum only
+//               when a score exceeds it by more than 2^8 (O and the sum are then
+//               rescaled in TMEM), and writes P over S as two bf16 parts
+//               (P = P_hi + P_lo, the second the rounding of the remainder), so
+//               O += P_hi V + P_lo V keeps about 16 bits of each probability. At
+//               the end O / (sum of P) -> bf16.
+// The tile shape follows the cost of a tcgen05.mma of M = 128, K = 16, which on
+// B200 takes about 125 cycles for any N up to 128 (about 135-170 at N = 256): a
+// 128-key tile costs 8 S MMAs of N = 128 where two 64-key tiles cost 16 of N = 64.
+// A buffer holds S(j), then P(j), until P(j) V(j) has finished; S(j + 3) waits
+// for that (s_free). Key tiles beyond the block's last position are never
+// loaded; the causal predicate masks the rest.
 #include "kernels.cuh"
 
 namespace llama {
 
 namespace {
-constexpr int KT = 64;       // keys per tile
-constexpr int KRING = 4;     // K stages (a K tile is free once S(j) is computed)
-constexpr int VRING = 4;     // V stages (a V tile is free once P(j) V(j) is computed)
+constexpr int KT = 128;      // keys per tile
+constexpr int NBUF = 3;      // S / P buffers in TMEM
+constexpr int KRING = 2;     // K stages (a K tile is free once S(j) is computed)
+constexpr int VRING = 3;     // V stages (a V tile is free once P(j) V(j) is computed)
 constexpr float LOG2E_TC = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;  // raise the running max only past 2^8
 }  // namespace
 
-template <int D, bool SPLIT_P>
+template <int D>
 struct AttnTcCfg {
   static constexpr int HALVES = D / 64;
-  static constexpr uint32_t Q_BYTES = 128 * D * 2;   // two (or one) 128 x 64 boxes
-  static constexpr uint32_t KV_BYTES = KT * D * 2;   // one K or one V tile
-  // the final (max, sum) of each row in each softmax group: [2 groups][2][128 rows]
-  static constexpr uint32_t RED_BYTES = 2 * 2 * 128 * 4;
-  static constexpr size_t SMEM = 1024 + Q_BYTES + (KRING + VRING) * KV_BYTES + RED_BYTES + 512;
-  // four 64-column S buffers (P(j) is written over S(j): 32 columns of bf16 pairs
-  // for P_hi, then 32 for P_lo), then O of each softmax group (D columns each)
+  static constexpr uint32_t Q_BYTES = 128 * D * 2;      // two (or one) 128 x 64 boxes
+  static constexpr uint32_t HALF_BYTES = KT * 128;      // 128 keys x 64 d of bf16 (two 64-row boxes)
+  static constexpr uint32_t KV_BYTES = HALVES * HALF_BYTES;  // one K or one V tile
+  static constexpr size_t SMEM = 1024 + Q_BYTES + (KRING + VRING) * KV_BYTES + 512;
+  // three 128-column S buffers (P(j) is written over S(j): 64 columns of bf16
+  // pairs for P_hi, then 64 for P_lo), then O (D columns)
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t P_LO_COL = 32;
+  static constexpr uint32_t P_LO_COL = KT / 2;
+  static constexpr uint32_t O_COL = NBUF * KT;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]: A = 128 rows (TMEM lanes) x 16 bf16 (8 columns of
@@ -80,11 +75,12 @@ __device__ __forceinline__ void tc_mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tme
       : "memory");
 }
 
-// 64 consecutive TMEM columns of this thread's lane: two loads, one wait
-__device__ __forceinline__ void tmem_ld_64cols(uint32_t taddr, float* v) {
-  uint32_t r[64];
+// NC consecutive TMEM columns of this thread's lane: NC / 32 loads, one wait
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  uint32_t r[NC];
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+  for (int h = 0; h < NC / 32; ++h)
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -101,7 +97,7 @@ __device__ __forceinline__ void tmem_ld_64cols(uint32_t taddr, float* v) {
         : "memory");
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
@@ -180,37 +176,32 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-constexpr int SOFTMAX_THREADS = 256;  // 8 warps: two groups of four, one thread per query row in each
+constexpr int SOFTMAX_THREADS = 128;  // 4 warps, one thread per query row (its TMEM lane)
 constexpr int ATTN_TC_THREADS = 64 + SOFTMAX_THREADS;
 
-template <int D, bool SPLIT_P>
+template <int D>
 __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                            const __grid_constant__ CUtensorMap map_v, bf16* __restrict__ o,
                            const int* __restrict__ start_pos, int sp_scalar, int T, int H, int Hkv, int S_max,
                            int hpc, int* err) {
-  using Cfg = AttnTcCfg<D, SPLIT_P>;
+  using Cfg = AttnTcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = sQ + Cfg::Q_BYTES;                  // KRING K tiles
   uint8_t* sV = sK + KRING * Cfg::KV_BYTES;         // VRING V tiles
-  float* red = reinterpret_cast<float*>(sV + VRING * Cfg::KV_BYTES);  // [group][m, l][128 rows]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VRING * Cfg::KV_BYTES + Cfg::RED_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VRING * Cfg::KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;           // [KRING]
   uint64_t* k_empty = k_full + KRING;    // [KRING]
   uint64_t* v_full = k_empty + KRING;    // [VRING]
   uint64_t* v_empty = v_full + VRING;    // [VRING]
-  uint64_t* s_full = v_empty + VRING;    // [4] S buffer (group, slot) holds S(j)
-  uint64_t* s_free = s_full + 4;         // [4] ... and P(j) V(j), which read P(j) there, has finished
-  // [4] per S buffer: P written over its S (one barrier per buffer: a group may
-  // write P(j + 2) into its other buffer before the MMA thread has taken P(j))
-  uint64_t* p_full = s_free + 4;
-  uint64_t* o_done = p_full + 4;         // [2] per group: its latest PV has finished
-  uint64_t* drained = o_done + 2;
-  uint64_t* fin = drained + 1;           // [4]: the two warps of a lane quarter exchange (m, l)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 4);
+  uint64_t* s_full = v_empty + VRING;    // [NBUF] buffer j % NBUF holds S(j)
+  uint64_t* p_full = s_full + NBUF;      // [NBUF] ... then P(j), written over it
+  uint64_t* s_free = p_full + NBUF;      // [NBUF] ... and P(j) V(j), which read it, has finished
+  uint64_t* drained = s_free + NBUF;     // every MMA of the CTA has finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,14 +228,12 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < NBUF; ++i) {
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], SOFTMAX_THREADS);
       mbar_init(&s_free[i], 1);
-      mbar_init(&p_full[i], SOFTMAX_THREADS / 2);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(drained, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&fin[i], 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -264,9 +253,6 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
   const int kv_len = min(sp + q_last + 1, S_max);
   const int n = (kv_len + KT - 1) / KT;
   const int row0 = (b * Hkv + kvh) * S_max;
-  // Key tile j goes to softmax group j & 1 as the group's tile k = j >> 1; its
-  // S lands in TMEM buffer 2 (j & 1) + (k & 1) (64 columns each, columns 0..255),
-  // and P(j) V(j) accumulates into the group's O (columns 256 + 128 (j & 1)).
 
   if (warp == 0) {
     if (lane == 0) {
@@ -278,15 +264,22 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
 #pragma unroll
       for (int hf = 0; hf < Cfg::HALVES; ++hf)
         tma_load_3d(sQ + hf * 16384, &map_q, q_full, hf * 64, h0, b * T + q0);
-      // K runs KRING tiles ahead of V: V(j) waits for P(j - VRING) V(j - VRING), and
-      // K(j + KRING) for S(j), which the MMA thread computes tiles ahead of P V
+      // a 128-key tile of one d half is two 64-row boxes, back to back: 128 rows
+      // of 128 B in the swizzled layout both MMAs read (rows past the tensor's
+      // end arrive as zeros; rows past the block's keys are masked)
+      auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int t) {
+        mbar_arrive_expect_tx(bar, Cfg::KV_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < Cfg::HALVES; ++hf)
+#pragma unroll
+          for (int kh = 0; kh < 2; ++kh)
+            tma_load_2d(dst + hf * Cfg::HALF_BYTES + kh * 8192, map, bar, hf * 64, row0 + t * KT + kh * 64);
+      };
+      // K(t) waits for S(t - KRING); V(j) for P(j - VRING) V(j - VRING)
       auto load_k = [&](int t) -> bool {
         const int st = t % KRING;
         if (!wait_or_abort(&k_empty[st], ((t / KRING) & 1) ^ 1, err, abort_flag)) return false;
-        mbar_arrive_expect_tx(&k_full[st], Cfg::KV_BYTES);
-#pragma unroll
-        for (int hf = 0; hf < Cfg::HALVES; ++hf)
-          tma_load_2d(sK + st * Cfg::KV_BYTES + hf * 8192, &map_k, &k_full[st], hf * 64, row0 + t * KT);
+        load_tile(&map_k, sK + st * Cfg::KV_BYTES, &k_full[st], t);
         return true;
       };
       int nk_issued = 0, nv_issued = 0;
@@ -295,10 +288,7 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % VRING;
         if (!(ok = wait_or_abort(&v_empty[st], ((j / VRING) & 1) ^ 1, err, abort_flag))) break;
-        mbar_arrive_expect_tx(&v_full[st], Cfg::KV_BYTES);
-#pragma unroll
-        for (int hf = 0; hf < Cfg::HALVES; ++hf)
-          tma_load_2d(sV + st * Cfg::KV_BYTES + hf * 8192, &map_v, &v_full[st], hf * 64, row0 + j * KT);
+        load_tile(&map_v, sV + st * Cfg::KV_BYTES, &v_full[st], j);
         ++nv_issued;
         if (nk_issued < n && (ok = load_k(nk_issued))) ++nk_issued;
       }
@@ -316,50 +306,47 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D) | (1u << 16);  // B (= V) N-major
       const uint32_t q_addr = smem_u32(sQ);
       bool ok = wait_or_abort(q_full, 0, err, abort_flag);
-      // S(j) = Q K(j)^T into buffer 2 (j & 1) + ((j >> 1) & 1) once K(j) is in and
-      // P(j - 4) V(j - 4), which read that buffer last, has finished; O_g += P(j) V(j)
-      // once group j & 1 has written P(j) over S(j). Order: S(0), S(1), then S(j + 2),
-      // PV(j) for each j, so S(j + 2) waits for PV(j - 2), issued two steps earlier.
-      int js = 0;  // next S to issue
-      for (int j = 0; ok && j < n; ++j) {
-        for (; ok && js < n && js <= j + 2; ++js) {
-          const int st = js % KRING;
-          ok = wait_or_abort(&k_full[st], (js / KRING) & 1, err, abort_flag);
-          const int sb = 2 * (js & 1) + ((js >> 1) & 1);
-          ok = ok && wait_or_abort(&s_free[sb], ((js >> 2) & 1) ^ 1, err, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + st * Cfg::KV_BYTES);
-          const uint32_t sd = tmem + (uint32_t)(sb * KT);
+      // S(j) = Q K(j)^T into buffer j % NBUF once K(j) is in and P(j - NBUF) V(j - NBUF),
+      // which read that buffer last, has finished
+      auto issue_s = [&](int js) -> bool {
+        const int st = js % KRING, sb = js % NBUF;
+        if (!wait_or_abort(&k_full[st], (js / KRING) & 1, err, abort_flag)) return false;
+        if (!wait_or_abort(&s_free[sb], ((js / NBUF) & 1) ^ 1, err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + st * Cfg::KV_BYTES);
+        const uint32_t sd = tmem + (uint32_t)(sb * KT);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;   // Q: 16 KB per 64-wide half
-            const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;   // K: 8 KB per half
-            tc_mma_bf16(sd, make_sw128_desc(q_addr + off), make_sw128_desc(k_addr + koff), idesc_s, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full[sb]);
-          tc_commit(&k_empty[st]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;              // Q: 16 KB per 64-wide half
+          const uint32_t koff = (kk >> 2) * Cfg::HALF_BYTES + (kk & 3) * 32;   // K: 128 rows per half
+          tc_mma_bf16(sd, make_sw128_desc(q_addr + off), make_sw128_desc(k_addr + koff), idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        const int g2 = j & 1, k = j >> 1, st = j % VRING;
-        const int sb = 2 * g2 + (k & 1);
+        tc_commit(&s_full[sb]);
+        tc_commit(&k_empty[st]);
+        return true;
+      };
+      // Order: S(0), then S(j + 1), PV(j) for each j: S(j + 1) waits for PV(j - 2),
+      // issued two steps earlier, and the softmax of tile j + 1 runs under PV(j).
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+        const int sb = j % NBUF, st = j % VRING;
         if (!(ok = wait_or_abort(&v_full[st], (j / VRING) & 1, err, abort_flag))) break;
-        if (!(ok = wait_or_abort(&p_full[sb], (k >> 1) & 1, err, abort_flag))) break;
+        if (!(ok = wait_or_abort(&p_full[sb], (j / NBUF) & 1, err, abort_flag))) break;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * Cfg::KV_BYTES);
-        const uint32_t od = tmem + 4 * KT + g2 * D;
+        const uint32_t od = tmem + Cfg::O_COL;
         const uint32_t pa = tmem + (uint32_t)(sb * KT);
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
           // A = P from TMEM (128 lanes x 16 keys = 8 columns of bf16 pairs per step);
-          // B = V N-major: 16 keys (2048 B) per step, 64-wide d blocks 8 KB apart
-          // (leading byte offset), 8-key groups 1 KB apart.
+          // B = V N-major: 16 keys (2048 B) per step, 64-wide d halves HALF_BYTES
+          // apart (leading byte offset), 8-key groups 1 KB apart.
           // O += P_hi V + P_lo V: P carries ~16 significant bits into the sum.
-          const uint64_t vdesc = make_sw128_desc_lbo(v_addr + kk * 2048, 8192, 1024);
-          tc_mma_bf16_tmem_a(od, pa + kk * 8, vdesc, idesc_pv, (k | kk) != 0 ? 1u : 0u);
-          if constexpr (SPLIT_P) tc_mma_bf16_tmem_a(od, pa + Cfg::P_LO_COL + kk * 8, vdesc, idesc_pv, 1u);
+          const uint64_t vdesc = make_sw128_desc_lbo(v_addr + kk * 2048, Cfg::HALF_BYTES, 1024);
+          tc_mma_bf16_tmem_a(od, pa + kk * 8, vdesc, idesc_pv, (j | kk) != 0 ? 1u : 0u);
+          tc_mma_bf16_tmem_a(od, pa + Cfg::P_LO_COL + kk * 8, vdesc, idesc_pv, 1u);
         }
-        tc_commit(&o_done[g2]);
         tc_commit(&s_free[sb]);
         tc_commit(&v_empty[st]);
       }
@@ -371,48 +358,47 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
   } else {
     // -------------------------------------------------------------------- softmax
     const int quarter = warp & 3;
-    const int sg = (warp - 2) >> 2;             // softmax group: key tiles j with j & 1 == sg
     const int r = quarter * 32 + lane;          // query row = TMEM lane
     const int pos_l = r / hpc, hl = r - pos_l * hpc;
     const int p_row = sp + min(q0 + pos_l, T - 1);
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t o_cols = lane_base + 4 * KT + sg * D;
+    const uint32_t o_cols = lane_base + Cfg::O_COL;
     const float sl2 = rsqrtf((float)D) * LOG2E_TC;
     const uint64_t scale2 = f2(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    int k = 0;
-    for (int j = sg; j < n; j += 2, ++k) {
-      const int sb = 2 * sg + (k & 1);
-      ok = wait_or_abort(&s_full[sb], (k >> 1) & 1, err, abort_flag);
+    for (int j = 0; j < n; ++j) {
+      const int sb = j % NBUF;
+      ok = wait_or_abort(&s_full[sb], (j / NBUF) & 1, err, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t s_cols = lane_base + sb * KT;
       float s[KT];
-      tmem_ld_64cols(lane_base + sb * KT, s);
-      // row maximum of the raw scores (masked keys -inf): two chains of 3-input maxima
+      tmem_ld_cols<KT>(s_cols, s);
+      // row maximum of the raw scores (masked keys -inf): four chains of 3-input maxima
       const int key0 = j * KT;
       if (__any_sync(0xffffffffu, key0 + KT - 1 > p_row)) {
 #pragma unroll
         for (int c = 0; c < KT; ++c)
           if (key0 + c > p_row) s[c] = -INFINITY;
       }
-      float ma = max3f(s[0], s[1], s[2]), mb = max3f(s[3], s[4], s[5]);
+      float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 6; c < 62; c += 4) {
-        ma = max3f(ma, s[c], s[c + 1]);
-        mb = max3f(mb, s[c + 2], s[c + 3]);
-      }
-      const float mt = max3f(ma, mb, fmaxf(s[62], s[63])) * sl2;  // log2 units
-      if (k == 0) {
+      for (int c = 4; c < KT; c += 8)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = max3f(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;  // log2 units
+      if (j == 0) {
         m_used = mt;
       } else if (__any_sync(0xffffffffu, mt > m_used + RESCALE_LOG2)) {
-        // rescale the group's O in TMEM once its previous PV has finished (S(j) being
-        // here means PV(j - 4), the group's tile before last, has finished, so the
+        // rescale O in TMEM once P(j - 1) V(j - 1) has finished (S(j) being here means
+        // P(j - 1 - NBUF) V(j - 1 - NBUF), the previous use of that buffer, has, so the
         // phase waited for is the latest one or the next)
-        ok = wait_or_abort(&o_done[sg], (k - 1) & 1, err, abort_flag);
+        const int pb = (j - 1) % NBUF;
+        ok = wait_or_abort(&s_free[pb], ((j - 1) / NBUF) & 1, err, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -433,34 +419,33 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
         m_used = m_new;
       }
       // P row -> bf16 pairs written over this row's S in TMEM (column c holds keys
-      // 2c, 2c + 1, the K-major A layout of the PV MMA); P_lo 32 columns further on.
+      // 2c, 2c + 1, the K-major A layout of the PV MMA); P_lo P_LO_COL columns on.
       // p = 2^(s * log2(e)/sqrt(D) - m): one packed FMA per pair and one ex2 each.
-      // A row may have no visible key yet in this group's tiles (its first tile
-      // lies past the row's position): m_used is then -inf and every score is
-      // -inf, so p = 2^(-inf - 0) = 0 instead of 2^(-inf + inf)
+      // (Key 0 is visible to every row, so m_used is finite from the first tile;
+      // the guard keeps 2^(-inf - m) = 0 meaningful all the same.)
       const float m_ref = m_used == -INFINITY ? 0.f : m_used;
       const uint64_t negm2 = f2(-m_ref, -m_ref);
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-      float ph[KT / 2], plo[SPLIT_P ? KT / 2 : 1];
 #pragma unroll
-      for (int e = 0; e < KT / 2; ++e) {
-        float t0, t1;
-        f2_split(fma_f2(f2(s[2 * e], s[2 * e + 1]), scale2, negm2), t0, t1);
-        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-        const uint64_t p2 = f2(p0, p1);
-        lsum[e & 1] = add_f2(lsum[e & 1], p2);
-        const uint32_t hi = pack_bf16x2(p0, p1);
-        ph[e] = __uint_as_float(hi);
-        if constexpr (SPLIT_P) {
+      for (int h = 0; h < KT / 64; ++h) {
+        float ph[32], plo[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float t0, t1;
+          f2_split(fma_f2(f2(s[64 * h + 2 * e], s[64 * h + 2 * e + 1]), scale2, negm2), t0, t1);
+          const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+          const uint64_t p2 = f2(p0, p1);
+          lsum[e & 1] = add_f2(lsum[e & 1], p2);
+          const uint32_t hi = pack_bf16x2(p0, p1);
+          ph[e] = __uint_as_float(hi);
           // lo = bf16(p - hi), the remainder taken as one packed subtraction
           float r0, r1;
           f2_split(sub_f2(p2, f2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u))), r0, r1);
           plo[e] = __uint_as_float(pack_bf16x2(r0, r1));
         }
+        tmem_st_32cols(s_cols + 32 * h, ph);
+        tmem_st_32cols(s_cols + Cfg::P_LO_COL + 32 * h, plo);
       }
-      const uint32_t p_cols = lane_base + sb * KT;
-      tmem_st_32cols(p_cols, ph);
-      if constexpr (SPLIT_P) tmem_st_32cols(p_cols + Cfg::P_LO_COL, plo);
       {
         float a0, a1, b0, b1;
         f2_split(lsum[0], a0, a1);
@@ -472,46 +457,24 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
       mbar_arrive(&p_full[sb]);
     }
     // every MMA of the CTA has finished (the MMA thread commits `drained` once,
-    // after its last PV): both groups' O are complete. A wait on o_done could not
-    // tell here whether one or two of the group's PVs are still running.
+    // after its last PV), so O is complete
     if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(drained, 0, err, abort_flag));
-    // (m, l) of both groups for this row (every softmax thread arrives once,
-    // also after a timeout; the wait is bounded all the same)
-    red[(sg * 2) * 128 + r] = m_used;
-    red[(sg * 2 + 1) * 128 + r] = l;
-    mbar_arrive(&fin[quarter]);
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&fin[quarter], 0, err, abort_flag));
     if (ok) {
-      // O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)); group sg
-      // writes columns sg * D/2 .. of the row. A group without tiles has m = -inf and
-      // an O that was never written: its weight is 0 and its columns are not read.
+      // O / l -> bf16
       tc_fence_after();
-      const float m0 = red[0 * 128 + r], l0 = red[1 * 128 + r], m1 = red[2 * 128 + r], l1 = red[3 * 128 + r];
-      const float mm = fmaxf(m0, m1);
-      const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - mm), f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mm);
-      const float inv = 1.f / (l0 * f0 + l1 * f1);
-      const bool has1 = n > 1;  // group 1 had at least one tile
+      const float inv = 1.f / l;
       const bool store = q0 + pos_l < T;
-      bf16* dst = o + ((size_t)(b * T + q0 + pos_l) * H + h0 + hl) * D + sg * (D / 2);
-      const uint32_t oc0 = lane_base + 4 * KT + sg * (D / 2), oc1 = oc0 + D;
+      bf16* dst = o + ((size_t)(b * T + q0 + pos_l) * H + h0 + hl) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 2; c += 32) {
-        float o0[32];
-        tmem_ld_32cols(oc0 + c, o0);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o0[e] *= f0;
-        if (has1) {
-          float o1[32];
-          tmem_ld_32cols(oc1 + c, o1);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o0[e] = fmaf(o1[e], f1, o0[e]);
-        }
+      for (int c = 0; c < D; c += 32) {
+        float ov[32];
+        tmem_ld_32cols(o_cols + c, ov);
         if (store) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             float v8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v8[i] = o0[e + i] * inv;
+            for (int i = 0; i < 8; ++i) v8[i] = ov[e + i] * inv;
             store8(dst + c + e, v8);
           }
         }
@@ -533,25 +496,21 @@ __global__ void __launch_bounds__(ATTN_TC_THREADS, 1)
 // ordered (token, head), the canonical K-major tile of the MMA.
 static bool make_q_map(CUtensorMap* map, const void* q, int tokens, int H, int D, int hpc);
 
-// P enters the PV product as two bf16 parts (hi + lo): about 16 bits of each
-// probability instead of 8, for one more MMA per 16 keys.
-constexpr bool kSplitP = true;
-
 template <int D>
 static cudaError_t prefill_tc_d(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, const int* sp,
                                 int sp_scalar, int B, int T, int H, int Hkv, int S_max, int* err, cudaStream_t st) {
-  using Cfg = AttnTcCfg<D, kSplitP>;
+  using Cfg = AttnTcCfg<D>;
   const int n_rep = H / Hkv;
   const int hpc = prefill_heads_per_cta(n_rep);
   const int BQ = 128 / hpc;
   CUtensorMap mq;
   if (!make_q_map(&mq, q, B * T, H, D, hpc)) return cudaErrorInvalidValue;
   static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(attn_prefill_tc_kernel<D, kSplitP>, Cfg::SMEM, attr);
+  cudaError_t e = ensure_smem(attn_prefill_tc_kernel<D>, Cfg::SMEM, attr);
   if (e != cudaSuccess) return e;
   dim3 grid(B * Hkv * (n_rep / hpc), (T + BQ - 1) / BQ);
   if (grid.y > 65535) return cudaErrorInvalidValue;
-  return launch_pdl(attn_prefill_tc_kernel<D, kSplitP>, grid, dim3(ATTN_TC_THREADS), Cfg::SMEM, st, mq, mk, mv,
+  return launch_pdl(attn_prefill_tc_kernel<D>, grid, dim3(ATTN_TC_THREADS), Cfg::SMEM, st, mq, mk, mv,
                     reinterpret_cast<bf16*>(o), sp, sp_scalar, T, H, Hkv, S_max, hpc, err);
 }
 
