@@ -241,13 +241,24 @@ __global__ void __launch_bounds__(160, 1)
         h0 = hp[0];
         h1 = hp[1];
       }
+      // the partials in slot order; the loads of up to 8 slots are issued before
+      // any of them is added, so a chunk costs one L2 round trip, not one per slot
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int sl = 0; sl < count; ++sl) {
-        const float4* src = reinterpret_cast<const float4*>(part + ((size_t)sl * M + m) * N + n);
-        const float4 a = __ldcg(src), b = __ldcg(src + 1);
-        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+      for (int sl0 = 0; sl0 < count; sl0 += 8) {
+        float4 pa[8], pb[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (sl0 + i < count) {
+            const float4* src = reinterpret_cast<const float4*>(part + ((size_t)(sl0 + i) * M + m) * N + n);
+            pa[i] = __ldcg(src);
+            pb[i] = __ldcg(src + 1);
+          }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (sl0 + i < count) {
+            v[0] += pa[i].x; v[1] += pa[i].y; v[2] += pa[i].z; v[3] += pa[i].w;
+            v[4] += pb[i].x; v[5] += pb[i].y; v[6] += pb[i].z; v[7] += pb[i].w;
+          }
       }
       if (res) {
         hp[0] = make_float4(h0.x + v[0], h0.y + v[1], h0.z + v[2], h0.w + v[3]);
