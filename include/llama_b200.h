@@ -268,9 +268,12 @@ int llama_reset(llama_ctx* ctx);
  *   into the loads of the linears' inputs. Eligible when dtype == LLAMA_BF16,
  *   B <= 32, head_dim == 128, dim % 128 == 0 and ffn % 64 == 0; an ineligible
  *   decode call returns LLAMA_ERR_INVALID_ARGS before any launch. The grid
- *   barriers need all of the launch's CTAs resident at once: on a GPU whose
- *   SMs are partly held by work on other streams or processes a barrier can
- *   wait past its bound, which raises LLAMA_ERR_TIMEOUT on the device flag.
+ *   barriers need all of the launch's CTAs resident at once, so the kernel is
+ *   a cooperative launch (no programmatic overlap with the kernel before it):
+ *   a grid larger than the device can hold returns LLAMA_ERR_INVALID_ARGS
+ *   before any launch, and the driver refuses the launch rather than start a
+ *   grid that cannot all be resident (LLAMA_ERR_CUDA). A barrier that still
+ *   waits past its bound raises LLAMA_ERR_TIMEOUT on the device flag.
  *  LLAMA_DECODE_AUTO (the default): the path measured faster on B200 for
  *   the decode workloads, currently LAYERED for every shape.
  * Returns LLAMA_ERR_INVALID_ARGS for another mode. Not stream-ordered: it

@@ -1011,14 +1011,33 @@ bool check_decode_block_plan(const DecodeBlockPlan& pl, int M, int H, size_t par
   return true;
 }
 
+// A cooperative launch: the grid barriers need every CTA resident at once, and
+// the driver then guarantees it (or refuses the launch). The grid is checked
+// against the kernel's occupancy first, so a grid that cannot be resident is
+// refused before anything runs.
 template <int MB>
 static cudaError_t db_launch(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st) {
   const size_t smem = db_smem(MB);
   static std::atomic<unsigned long long> attr{0};
   cudaError_t e = ensure_smem(decode_block_kernel<MB>, smem, attr);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_block_kernel<MB>, dim3(grid), dim3(160), smem, st, maps[0], maps[1], maps[2], maps[3],
-                    maps[4], maps[5], p);
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_block_kernel<MB>, 160, smem)) != cudaSuccess)
+    return e;
+  if ((long long)per_sm * sms < grid) return cudaErrorCooperativeLaunchTooLarge;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(160);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeCooperative;
+  la[0].val.cooperative = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_block_kernel<MB>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
 }
 
 cudaError_t launch_decode_block(const CUtensorMap* maps, const DecodeBlockParams& p, int grid, cudaStream_t st) {

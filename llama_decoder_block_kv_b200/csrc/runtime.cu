@@ -260,7 +260,10 @@ int run_block_persistent(llama_ctx* c, int layer, float* h, int B, const int* sp
   p.max_chunks = pl.max_chunks;
   p.norm_local = pl.norm_local ? 1 : 0;
   const CUtensorMap maps[6] = {Ly.map_w[0], Ly.map_w[1], Ly.map_w[2], Ly.map_w[3], Ly.map_k, Ly.map_v};
-  return launch_decode_block(maps, p, pl.grid, st) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  const cudaError_t e = launch_decode_block(maps, p, pl.grid, st);
+  // a grid that cannot be resident at once is refused before anything runs
+  if (e == cudaErrorCooperativeLaunchTooLarge) return LLAMA_ERR_INVALID_ARGS;
+  return e == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 // Which decode attention kernel a call runs (both compute the same attention).
