@@ -94,6 +94,28 @@ def test_block_ragged_decode_positions():
         pair.close()
 
 
+@pytest.mark.parametrize("dim,H,Hkv,Bsz", [(1024, 8, 2, 2), (1024, 8, 8, 1)])
+def test_long_prefill_on_cta_pairs(dim, H, Hkv, Bsz):
+    """A prefill long enough for the CTA-pair attention kernel (2048 keys or more),
+    against the oracle: GQA (4 query heads per kv head, 32 positions per block) and
+    MHA (128 positions per block); T = 2080 gives an odd number of query blocks in
+    both (65 and 17), so the last pair's second block lies wholly past the
+    sequence; device start positions put the second sequence 40 positions on."""
+    T = 2080
+    w = _wl(dim, H, Hkv, Bm=Bsz, S=2176)
+    pair = Pair(w)
+    try:
+        sp = np.array([0, 40][:Bsz])
+        h = synth.hidden(w, (Bsz, T, dim), call=0)
+        _run(pair, h, sp, BF16_HIDDEN_ABS)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        for b in range(Bsz):
+            written[b, sp[b]:sp[b] + T] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        pair.close()
+
+
 def test_block_fp32_mode():
     w = _wl(256, 4, 2, act="fp32", S=64)
     pair = Pair(w)
