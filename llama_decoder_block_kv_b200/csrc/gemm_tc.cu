@@ -214,6 +214,199 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------------------
+// The 2-SM form: a CTA pair (cluster of two) computes 256 x 256 tiles of C with
+// tcgen05.mma.cta_group::2 (M = 256). Each CTA loads its 128 rows of A and one
+// 128-row block of B (the library's tile layout: blocks 2 nb and 2 nb + 1 of
+// the tile's 256 columns) into its own ring; the copies of both complete on
+// rank 0's ring barriers (primed with both CTAs' bytes). Rank 0, warp 1, lane 0
+// issues every MMA; ring slots and accumulators are released by commits that
+// arrive on both CTAs' barriers. Each CTA's epilogue reads its own 128 rows
+// from its TMEM; the accumulator goes back to the issuer once the epilogue
+// threads of both CTAs have arrived on rank 0's barrier (rank 1's remotely).
+// On B200 a 2-SM MMA with N = 256 costs ~134 cycles against ~168 for the 1-SM
+// form with A in shared memory (measured), and each SM reads half of B.
+namespace {
+constexpr int P_BN = 256;
+constexpr int P_STAGES = 6;
+constexpr uint32_t P_A_BYTES = BM * BK * 2;        // this CTA's 128 rows of A
+constexpr uint32_t P_B_BYTES = 128 * BK * 2;       // this CTA's 128 rows of B
+constexpr size_t P_SMEM = 1024 + (size_t)P_STAGES * (P_A_BYTES + P_B_BYTES) + 256;
+}  // namespace
+
+template <typename T>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M,
+                        int N, int K, EpiParams ep) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base;
+  uint8_t* sB = base + P_STAGES * P_A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + P_STAGES * P_B_BYTES);  // [P_STAGES] rank 0's: both CTAs' copies
+  uint64_t* empty = full + P_STAGES;                                          // [P_STAGES] ring slot consumed
+  uint64_t* tfull = empty + P_STAGES;   // [2] accumulator complete
+  uint64_t* tempty = tfull + 2;         // [2] rank 0's: both CTAs' epilogues have read it
+  uint64_t* drained = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_m = (M + 255) / 256, num_n = (N + P_BN - 1) / P_BN;
+  const int num_tiles = num_m * num_n;
+  const int num_k = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P_STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 2 * 128);
+    }
+    mbar_init(drained, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&map_a);
+    prefetch_tensormap(&map_b);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(2 * P_BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any copy or commit reaches them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const TileCoord tc = tile_coord(tile, num_m, num_n);
+        for (int kb = 0; kb < num_k; ++kb, ++it) {
+          const int stage = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!wait_or_abort(&empty[stage], ph ^ 1, ep.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (P_A_BYTES + P_B_BYTES));
+          const uint32_t bar = mbar_cluster_addr(&full[stage], 0);
+          tma_load_2d_pair(sA + stage * P_A_BYTES, &map_a, bar, kb * BK, tc.mb * 256 + (int)rank * 128);
+          // B in 128-row x 64-k tiles, tile (rb, kb) at rows (rb * num_k + kb) * 128 of the map
+          tma_load_2d_pair(sB + stage * P_B_BYTES, &map_b, bar, 0, ((tc.nb * 2 + (int)rank) * num_k + kb) * 128);
+        }
+      }
+      if (rank == 0) {
+        // every copy of either CTA lands before the pair can retire (bounded): rank
+        // 0's barriers count both CTAs' bytes, and rank 1 does not pass the final
+        // cluster barrier before rank 0 has waited for them
+        const int first = it > P_STAGES ? it - P_STAGES : 0;
+        for (int j = first; j < it; ++j) {
+          uint64_t* bar = &full[j % P_STAGES];
+          const uint32_t ph = (j / P_STAGES) & 1;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar, ph) && global_timer_ns() - t0 < LLAMA_WAIT_LIMIT_NS) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (rank 0)
+      constexpr uint32_t idesc = idesc2_bf16(256, P_BN, false);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!wait_cluster_or_abort(&tempty[acc], aph ^ 1, ep.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * P_BN;
+        for (int kb = 0; kb < num_k; ++kb, ++it) {
+          const int stage = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!wait_or_abort(&full[stage], ph, ep.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * P_A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * P_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma2_ss(d, make_sw128_desc(a_addr + kk * 32), make_sw128_desc(b_addr + kk * 32), idesc,
+                    (kb | kk) != 0 ? 1u : 0u);
+          commit2(&empty[stage]);
+        }
+        if (!ok) break;
+        commit2(&tfull[acc]);
+      }
+      // all MMAs have finished before TMEM is released
+      commit2(drained);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drained, 0) && global_timer_ns() - t0 < LLAMA_WAIT_LIMIT_NS) {
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    int local = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
+      const TileCoord tc = tile_coord(tile, num_m, num_n);
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      const bool ok = wait_or_abort(&tfull[acc], aph, ep.err, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is warp-collective
+      tc_fence_after();
+      const int m = tc.mb * 256 + (int)rank * 128 + row;
+#pragma unroll 1
+      for (int c = 0; c < P_BN / 32; ++c) {
+        float v[32];
+        tmem_ld_32cols(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + c * 32, v);
+        if (m < M) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int n = tc.nb * P_BN + c * 32 + j * 8;
+            if (n < N) epilogue8<T>(ep, m, n, v + j * 8);
+          }
+        }
+      }
+      tc_fence_before();
+      // the reads above have completed (tcgen05.ld waits), so rank 1's arrival can be relaxed
+      if (rank == 0) mbar_arrive(&tempty[acc]);
+      else mbar_arrive_remote_relaxed(&tempty[acc], 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // the other CTA's shared memory and TMEM are used by the pair's MMAs until
+  // `drained`; neither CTA frees its TMEM or retires before both get here
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * P_BN) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
 // signature of the driver's cuTensorMapEncodeTiled (cuda.h), fetched at run
@@ -292,17 +485,44 @@ static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, i
                     ep);
 }
 
-// BN = 256 unless that leaves the last wave badly filled.
+// CTA pairs over 256 x 256 tiles; B is the library's tiled weights (its map, 128-row boxes)
+static cudaError_t launch_tc_pair(const void* A, const CUtensorMap& mb, int M, int N, int K, const EpiParams& ep,
+                                  int num_sms, cudaStream_t st) {
+  CUtensorMap ma;
+  if (!make_tmap_bf16(&ma, A, M, K, BM)) return cudaErrorInvalidValue;
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(gemm_tc_pair_kernel<bf16>, P_SMEM, attr);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + 255) / 256) * ((N + P_BN - 1) / P_BN);
+  const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  return launch_pdl(gemm_tc_pair_kernel<bf16>, dim3(2 * pairs), dim3(192), P_SMEM, st, ma, mb, M, N, K, ep);
+}
+
+// The tile shape with the smallest estimate of waves x tile time, in units of a
+// 1-SM 128 x 256 tile: 1-SM 128 x 128 tiles 0.5, 128 x 256 tiles 1, CTA-pair
+// 256 x 256 tiles 0.8 (two SMs, ~134 against ~168 cycles per N = 256 MMA step,
+// measured); the pair form for weights in the library's tile layout only.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
                            int num_sms, cudaStream_t st, const CUtensorMap* bmap) {
   const int num_m = (M + BM - 1) / BM;
   const int t256 = num_m * ((N + 255) / 256);
   const int t128 = num_m * ((N + 127) / 128);
-  auto eff = [&](int tiles, double cost) {
-    const int waves = (tiles + num_sms - 1) / num_sms;
+  const int tpair = ((M + 255) / 256) * ((N + 255) / 256);
+  auto eff = [](int tiles, int slots, double cost) {
+    const int waves = (tiles + slots - 1) / slots;
     return (double)waves * cost;  // time ~ waves x per-tile cost
   };
-  const bool use256 = (N % 256 == 0) && eff(t256, 2.0) <= eff(t128, 1.0) * 1.05;
+  const double e128 = eff(t128, num_sms, 0.5), e256 = eff(t256, num_sms, 1.0);
+  const double epair = eff(tpair, num_sms / 2, 0.8);
+  if (b_tiled && N % 256 == 0 && num_sms >= 2 && epair < e128 && epair < e256) {
+    CUtensorMap mb;
+    if (bmap)
+      mb = *bmap;  // the library's weights: encoded once when they were set
+    else if (!make_tmap_weights(&mb, B, 1, N, K, 128))
+      return cudaErrorInvalidValue;
+    return launch_tc_pair(A, mb, M, N, K, ep, num_sms, st);
+  }
+  const bool use256 = (N % 256 == 0) && e256 <= e128 * 1.05;
   return use256 ? launch_tc<256>(A, B, b_tiled, M, N, K, ep, num_sms, st, bmap)
                 : launch_tc<128>(A, B, b_tiled, M, N, K, ep, num_sms, st, bmap);
 }

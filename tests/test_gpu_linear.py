@@ -34,6 +34,21 @@ def test_tcgen05_gemm(M, N, K):
     _check(x, w, y)
 
 
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 1024), (1000, 22016, 4096), (8192, 6144, 4096)])
+def test_tcgen05_gemm_on_cta_pairs(M, N, K):
+    """Shapes large enough for the CTA-pair GEMM (2-SM MMAs over 256 x 256 tiles),
+    which takes weights in the library's tile layout: against a float64 matmul of
+    the same bf16 inputs, including a ragged M (1000 rows: the last pair tile holds
+    rows past the matrix). Row-major weights of the same shapes run the single-CTA
+    kernel; the two agree to the GEMM tolerance, not necessarily to the bit."""
+    x, w = _inputs(M, N, K, torch.bfloat16, 13)
+    wt = B.llama_tile_weights(w)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    B.llama_linear(x, wt, y, B.LLAMA_PATH_TCGEN05 | B.LLAMA_WEIGHTS_TILED, n=N)
+    torch.cuda.synchronize()
+    _check(x, w, y)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 128, 256), (5, 384, 4096), (8, 4096, 4096), (16, 12288, 4096),
                                    (17, 256, 11008), (32, 4096, 14336), (32, 28672, 4096), (3, 136, 192), (9, 8, 128)])
 def test_gemv_split_k(M, N, K):
@@ -61,7 +76,9 @@ def test_simt_gemm(M, N, K, dt):
 def test_tiled_weights_give_identical_results(path, M, N, K):
     """The tile layout only changes where a 128 x 64 stage is read from: the
     shared-memory image, hence every MMA and every sum, is the same as with
-    row-major weights, so the outputs are bit-identical."""
+    row-major weights, so the outputs are bit-identical (for shapes that run the
+    same kernel with both layouts, as these do: the CTA-pair GEMM takes only
+    tiled weights, test_tcgen05_gemm_on_cta_pairs)."""
     x, w = _inputs(M, N, K, torch.bfloat16, 41)
     wt = B.llama_tile_weights(w)
     assert wt.numel() == (N + 127) // 128 * 128 * K
