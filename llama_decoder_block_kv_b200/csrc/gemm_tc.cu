@@ -500,8 +500,9 @@ static cudaError_t launch_tc_pair(const void* A, const CUtensorMap& mb, int M, i
 
 // The tile shape with the smallest estimate of waves x tile time, in units of a
 // 1-SM 128 x 256 tile: 1-SM 128 x 128 tiles 0.5, 128 x 256 tiles 1, CTA-pair
-// 256 x 256 tiles 0.8 (two SMs, ~134 against ~168 cycles per N = 256 MMA step,
-// measured); the pair form for weights in the library's tile layout only.
+// 256 x 256 tiles 0.7 (two SMs; the MMA step alone is ~134 against ~168 cycles,
+// and whole GEMMs measured 0.69-0.75 of the single-CTA time); the pair form for
+// weights in the library's tile layout only.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
                            int num_sms, cudaStream_t st, const CUtensorMap* bmap) {
   const int num_m = (M + BM - 1) / BM;
@@ -513,7 +514,7 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int
     return (double)waves * cost;  // time ~ waves x per-tile cost
   };
   const double e128 = eff(t128, num_sms, 0.5), e256 = eff(t256, num_sms, 1.0);
-  const double epair = eff(tpair, num_sms / 2, 0.8);
+  const double epair = eff(tpair, num_sms / 2, 0.7);
   if (b_tiled && N % 256 == 0 && num_sms >= 2 && epair < e128 && epair < e256) {
     CUtensorMap mb;
     if (bmap)
