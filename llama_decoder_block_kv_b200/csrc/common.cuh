@@ -406,9 +406,10 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // arrive on the barrier at the same shared-memory offset in CTA `rank` of the
-// cluster, relaxed (no release fence): used where what the arrival announces is
-// already complete when it is made (tensor-memory stores the arriving threads
-// have waited for with tcgen05.wait::st), so only the signal has to travel.
+// cluster, relaxed (no release fence): for arrivals that announce work already
+// complete when they are made (tensor-memory stores or loads the arriving
+// threads have waited for with tcgen05.wait::st / ::ld), so only the signal has
+// to travel.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint64_t* bar, uint32_t rank) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
@@ -460,7 +461,7 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
-// the 3-D form of the same (the Q tile)
+// the 3-D form of the same
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {
   asm volatile(
