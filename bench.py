@@ -221,6 +221,17 @@ def job_throughput(tokens_per_step_per_rank: int, steps: int, max_ms: float, wor
 
 # ----------------------------------------------------------------------------- single-layer workloads
 
+def decode_launches_per_block(w, tokens: int) -> int:
+    """Kernels of one block's decode step of `tokens` tokens: one persistent launch (bf16, when
+    chosen); else gemv, attention (chunk merge fused), gemv, gemv, gemv and the two RMSNorms, which
+    run inside the GEMVs that read them for bf16 calls of at most 4 tokens at dim <= 4096."""
+    if w.act != "bf16":
+        return 7
+    if DECODE_KERNEL == "persistent":
+        return 1
+    return 5 if (tokens <= 4 and w.dim <= 4096 and w.dim % 64 == 0) else 7
+
+
 class LayerBench:
     """Prefill + decode of one decoder layer (llama7b-layer) or decode only (llama70b-layer)."""
 
@@ -276,9 +287,7 @@ class LayerBench:
 
     def kernels_per_step(self):
         pre = 7 if self.P else 0  # rmsnorm, gemm x2, attention, rmsnorm, gemm x2 (the QKV and wo GEMMs: 4 in all)
-        # decode: rmsnorm, gemv, attention (chunk merge fused), gemv, rmsnorm, gemv, gemv; or one persistent launch
-        dec = 1 if DECODE_KERNEL == "persistent" else 7
-        return pre + self.ND * dec
+        return pre + self.ND * decode_launches_per_block(self.w, self.Bsz)
 
     def decode_gemms(self):
         """(x, w) pairs of the decode linears, same shapes and kernel as the decode path."""
@@ -695,7 +704,7 @@ class ModelBench:
         enh = synth.embed_norm_head(w, device="cuda")
         B.llama_set_embed_norm_head(ctx, enh["tok_embeddings"], enh["norm"], enh["output"])
         del enh
-        per_block = 1 if DECODE_KERNEL == "persistent" else 7
+        per_block = decode_launches_per_block(w, w.batch)
         if w.ragged_hi:                      # ragged decode from prefilled caches
             self.kind = "ragged-decode"
             self.lens = synth.ragged_lengths(w, "cuda")
@@ -724,7 +733,7 @@ class ModelBench:
             B.llama_reserve(ctx, w.batch * P)
             self.tokens_per_step = w.batch * (P + ND)
             blocks = 1 + w.n_layers * 7 + 2
-            self.launches_per_step = blocks + ND * (1 + w.n_layers * (per_block if w.act == "bf16" else 7) + 2)
+            self.launches_per_step = blocks + ND * (1 + w.n_layers * per_block + 2)
             self.inputs = [self.toks]
         else:                                # one long prefill, last-position logits
             self.kind = "prefill"

@@ -22,6 +22,18 @@
 // sums the partials in a fixed order (deterministic) and runs the epilogue,
 // then re-zeroes the counter, so the workspace needs no clearing between
 // launches. A row block inside one range goes straight to the epilogue.
+//
+// For decode calls of at most NORM_MAX_M tokens with K <= NORM_MAX_K the
+// kernel can also compute its input X = RMSNorm(h) itself (the notes'
+// RMSNorm.forward: fp32 statistics, the normalised value rounded to bf16,
+// times the weight, rounded again), which takes the RMSNorm launch and the X
+// round trip through memory off the decode step. The producer copies the norm
+// weight into shared memory ahead of the ring's first weight tiles (plain
+// loads issued beside those copies waited behind them for microseconds) and
+// fetches only NORM_PREFETCH stages before the dependency wait; after it the
+// consumer warps load all of their share of h at once, reduce the sums of
+// squares across the CTA and keep the M normalised rows resident in shared
+// memory for the whole K; the ring carries weight tiles only.
 #include "kernels.cuh"
 
 #include <algorithm>
@@ -44,6 +56,27 @@ __host__ __device__ constexpr int stages(int mb) { return (int)(RING_BUDGET / st
 __host__ __device__ constexpr size_t gemv_smem(int mb) {
   return 1024 + (size_t)stages(mb) * stage_bytes(mb) + (size_t)8 * mb * OS * 4 + 2 * stages(mb) * 8 + 16;
 }
+
+constexpr int NORM_MAX_M = 4;
+constexpr int NORM_MAX_K = 4096;
+constexpr int NORM_CHUNKS = NORM_MAX_K / (128 * 4);  // float4 chunks of one row per consumer thread
+// resident row stride in bytes: 16 bytes past a multiple of 128, so the rows
+// an ldmatrix reads together sit in different banks
+constexpr uint32_t NORM_XS = NORM_MAX_K * 2 + 16;
+constexpr int NORM_STAGES = (int)(RING_BUDGET / W_BYTES);
+// Ring stages fetched before the dependency wait in the fused-norm form. With
+// the whole ring in flight, the loads of h after the wait queued behind those
+// misses; measured on the LLaMA-7B layer's decode (per token): 11 stages
+// 86.9 us, 8 86.1, 7 85.8, 6 85.8, 4 85.9. The plain form keeps its whole
+// ring (its X tiles share the stages' barriers; 5 / 7 / 9 of 10 were slower).
+constexpr int NORM_PREFETCH = 6;
+// ring, resident rows, a 16-byte zero block (the MMA rows past M), the norm
+// weight, output staging, barriers (ring + the weight's)
+__host__ __device__ constexpr size_t gemv_norm_smem() {
+  return 1024 + (size_t)NORM_STAGES * W_BYTES + (size_t)NORM_MAX_M * NORM_XS + 16 + (size_t)NORM_MAX_K * 2 +
+         (size_t)8 * OS * 4 + 2 * NORM_STAGES * 8 + 8 + 16;
+}
+static_assert(gemv_norm_smem() <= 232448, "fused-norm GEMV shared memory");
 }  // namespace
 
 // swizzled byte address of (row, col) in a tile of 128-byte rows written by TMA
@@ -65,20 +98,28 @@ __host__ __device__ __forceinline__ int sk_owner(int x, int total, int grid) {
   return c;
 }
 
-template <int MB>
+// NORM (MB == 1, M <= NORM_MAX_M, K <= NORM_MAX_K): X = RMSNorm(h_norm) with
+// weight w_norm and eps, computed here; map_x is not read.
+template <int MB, bool NORM>
 __global__ void __launch_bounds__(160, 1)
     llama_decode_linear_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, int M,
                      int N, int nk, int total, int tiled, float* __restrict__ part, int* __restrict__ counters,
-                     EpiParams ep) {
-  constexpr int STAGES = stages(MB);
-  constexpr uint32_t SB = stage_bytes(MB);
+                     EpiParams ep, const float* __restrict__ h_norm, const bf16* __restrict__ w_norm, float eps) {
+  static_assert(!NORM || MB == 1, "the fused norm serves one 8-token block");
+  constexpr int STAGES = NORM ? NORM_STAGES : stages(MB);
+  constexpr uint32_t SB = NORM ? W_BYTES : stage_bytes(MB);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* os = reinterpret_cast<float*>(base + STAGES * SB);
+  uint8_t* xres = base + STAGES * SB;  // NORM: the M normalised rows, a zero block, the norm weight
+  uint8_t* xzero = xres + NORM_MAX_M * NORM_XS;
+  uint8_t* wsm = xzero + 16;
+  float* os = reinterpret_cast<float*>(NORM ? wsm + NORM_MAX_K * 2 : xres);
   uint64_t* full = reinterpret_cast<uint64_t*>(os + 8 * MB * OS);
   uint64_t* empty = full + STAGES;
+  uint64_t* wbar = empty + STAGES;  // NORM: the norm weight landed
   __shared__ int s_last;
   __shared__ int s_abort;
+  __shared__ float s_ss[4][NORM_MAX_M];  // NORM: per-warp sums of squares of each row
   volatile int* abort_flag = &s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -91,6 +132,7 @@ __global__ void __launch_bounds__(160, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);
     }
+    if (NORM) mbar_init(wbar, 1);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -103,7 +145,11 @@ __global__ void __launch_bounds__(160, 1)
       prefetch_tensormap(&map_x);
       // The weights do not depend on the previous kernel: fill the ring with
       // weight tiles first, then wait for the producer of X and add X tiles.
-      const int pre = min(STAGES, send - sbeg);
+      if constexpr (NORM) {
+        mbar_arrive_expect_tx(wbar, (uint32_t)(nk * KB * 2));
+        bulk_load(wsm, w_norm, (uint32_t)(nk * KB * 2), wbar);
+      }
+      const int pre = min(NORM ? NORM_PREFETCH : STAGES, send - sbeg);
       for (int i = 0; i < pre; ++i) {
         const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
         mbar_arrive_expect_tx(&full[i], SB);
@@ -111,9 +157,11 @@ __global__ void __launch_bounds__(160, 1)
       }
       pdl_wait();
       pdl_trigger();
-      for (int i = 0; i < pre; ++i) {
-        const int x = sbeg + i, ks = x - (x / nk) * nk;
-        tma_load_2d(base + i * SB + W_BYTES, &map_x, &full[i], ks * KB, 0);
+      if constexpr (!NORM) {
+        for (int i = 0; i < pre; ++i) {
+          const int x = sbeg + i, ks = x - (x / nk) * nk;
+          tma_load_2d(base + i * SB + W_BYTES, &map_x, &full[i], ks * KB, 0);
+        }
       }
       int j = pre;
       for (int x = sbeg + pre; x < send; ++x, ++j) {
@@ -123,17 +171,67 @@ __global__ void __launch_bounds__(160, 1)
         uint8_t* dst = base + st * SB;
         mbar_arrive_expect_tx(&full[st], SB);
         tma_load_2d(dst, &map_w, &full[st], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
-        tma_load_2d(dst + W_BYTES, &map_x, &full[st], ks * KB, 0);
+        if constexpr (!NORM) tma_load_2d(dst + W_BYTES, &map_x, &full[st], ks * KB, 0);
       }
       // the CTA must not retire while a copy into its shared memory is in flight
       for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, ep.err);
+      if constexpr (NORM) mbar_wait(wbar, 0, ep.err);
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  const int K = nk * KB;
   pdl_wait();
   pdl_trigger();
+  if constexpr (NORM) {
+    // every load of this thread's share of the M rows is issued before any is used
+    float4 hv[NORM_MAX_M][NORM_CHUNKS];
+#pragma unroll
+    for (int m = 0; m < NORM_MAX_M; ++m)
+#pragma unroll
+      for (int i = 0; i < NORM_CHUNKS; ++i) {
+        const int c4 = (tid + 128 * i) * 4;
+        hv[m][i] = (m < M && c4 < K) ? *reinterpret_cast<const float4*>(h_norm + (size_t)m * K + c4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int m = 0; m < NORM_MAX_M; ++m) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < NORM_CHUNKS; ++i)
+        ss += hv[m][i].x * hv[m][i].x + hv[m][i].y * hv[m][i].y + hv[m][i].z * hv[m][i].z + hv[m][i].w * hv[m][i].w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) s_ss[warp][m] = ss;
+    }
+    if (tid == 0) *reinterpret_cast<uint4*>(xzero) = make_uint4(0u, 0u, 0u, 0u);
+    wait_or_abort(wbar, 0, ep.err, abort_flag);
+    uint2 wn[NORM_CHUNKS];
+#pragma unroll
+    for (int i = 0; i < NORM_CHUNKS; ++i) {
+      const int c4 = (tid + 128 * i) * 4;
+      wn[i] = c4 < K ? *reinterpret_cast<const uint2*>(wsm + c4 * 2) : make_uint2(0u, 0u);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+    for (int m = 0; m < NORM_MAX_M; ++m) {
+      if (m >= M) break;
+      const float inv = rsqrtf((s_ss[0][m] + s_ss[1][m] + s_ss[2][m] + s_ss[3][m]) / (float)K + eps);
+#pragma unroll
+      for (int i = 0; i < NORM_CHUNKS; ++i) {
+        const int c4 = (tid + 128 * i) * 4;
+        if (c4 < K) {
+          const float2 w0 = unpack_bf16x2(wn[i].x), w1 = unpack_bf16x2(wn[i].y);
+          uint2 u;
+          u.x = pack_bf16x2(round_to<bf16>(hv[m][i].x * inv) * w0.x, round_to<bf16>(hv[m][i].y * inv) * w0.y);
+          u.y = pack_bf16x2(round_to<bf16>(hv[m][i].z * inv) * w1.x, round_to<bf16>(hv[m][i].w * inv) * w1.y);
+          *reinterpret_cast<uint2*>(xres + m * NORM_XS + c4 * 2) = u;
+        }
+      }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
   const int a_row = warp * 32 + (lane & 7) + 8 * ((lane >> 3) & 1);  // + 16 t
   const int a_col = 8 * (lane >> 4);                                 // + 16 kk
   int j = 0;
@@ -159,9 +257,15 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
         for (int kk2 = 0; kk2 < 2; ++kk2) {
           uint32_t xf[MB][4];
+          if constexpr (NORM) {
+            // resident rows (plain row-major); rows past M read the zero block
+            const int row = lane & 7, k0 = (x - rb * nk) * KB + kk2 * 32 + 8 * (lane >> 3);
+            ldmatrix_x4(xf[0], row < M ? smem_u32(xres) + row * NORM_XS + k0 * 2 : smem_u32(xzero));
+          } else {
 #pragma unroll
-          for (int mb = 0; mb < MB; ++mb)
-            ldmatrix_x4(xf[mb], sw128(xb, mb * 8 + (lane & 7), kk2 * 32 + 8 * (lane >> 3)));
+            for (int mb = 0; mb < MB; ++mb)
+              ldmatrix_x4(xf[mb], sw128(xb, mb * 8 + (lane & 7), kk2 * 32 + 8 * (lane >> 3)));
+          }
 #pragma unroll
           for (int s2 = 0; s2 < 2; ++s2) {
             const int kk = kk2 * 2 + s2;
@@ -333,20 +437,23 @@ bool check_gemv_plan(int M, int N, int K, int num_sms) {
   return true;
 }
 
-template <int MB>
+template <int MB, bool NORM = false>
 static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
-                             int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
-  constexpr size_t smem = gemv_smem(MB);
+                             int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st,
+                             const float* h_norm = nullptr, const bf16* w_norm = nullptr, float eps = 0.f) {
+  constexpr size_t smem = NORM ? gemv_norm_smem() : gemv_smem(MB);
   static std::atomic<unsigned long long> attr{0};
-  cudaError_t e = ensure_smem(llama_decode_linear_kernel<MB>, smem, attr);
+  cudaError_t e = ensure_smem(llama_decode_linear_kernel<MB, NORM>, smem, attr);
   if (e != cudaSuccess) return e;
-  return launch_pdl(llama_decode_linear_kernel<MB>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk, p.total, tiled, part,
-                    counters, ep);
+  return launch_pdl(llama_decode_linear_kernel<MB, NORM>, dim3(p.grid), dim3(160), smem, st, mw, mx, M, N, p.nk,
+                    p.total, tiled, part, counters, ep, h_norm, w_norm, eps);
 }
+
+bool gemv_can_fuse_norm(int M, int K) { return M >= 1 && M <= NORM_MAX_M && K % KB == 0 && K <= NORM_MAX_K; }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
                              float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
-                             const CUtensorMap* wmap) {
+                             const CUtensorMap* wmap, const float* h_norm, const void* w_norm, float eps) {
   (void)num_sms;
   const int MB = (M + 7) / 8;
   CUtensorMap mw, mx;
@@ -354,6 +461,14 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int
     mw = *wmap;  // the library's weights: encoded once when they were set
   else if (!make_tmap_weights(&mw, W, tiled, N, K, RPC))
     return cudaErrorInvalidValue;
+  if (h_norm) {  // X = RMSNorm(h_norm), computed by the kernel
+    // the weight is bulk-copied (16-byte aligned); h is read as float4
+    if (!w_norm || !gemv_can_fuse_norm(M, K) || (reinterpret_cast<uintptr_t>(w_norm) & 15) ||
+        (reinterpret_cast<uintptr_t>(h_norm) & 15))
+      return cudaErrorInvalidValue;
+    return launch_mb<1, true>(mw, mw, M, N, p, tiled, part, counters, ep, st, h_norm,
+                              reinterpret_cast<const bf16*>(w_norm), eps);
+  }
   if (!make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
   switch (MB) {
     case 1: return launch_mb<1>(mw, mx, M, N, p, tiled, part, counters, ep, st);

@@ -72,9 +72,13 @@ GemvPlan plan_gemv(int M, int N, int K, int num_sms);
 bool check_gemv_plan(int M, int N, int K, int num_sms);  // host walk of a plan (see gemv.cu)
 // W: [N][K] row-major (tiled = 0) or the library's weight tiles (tiled = 1, tile_weights)
 // wmap (optional): a tensor map of W encoded once by the caller (tiled layout, 128-row boxes); else encoded here
+// h_norm (optional): X is not read; the kernel computes X = RMSNorm(h_norm) itself, h_norm [M][K] fp32 rows,
+// w_norm [K] bf16, eps (the RMSNorm kernel's arithmetic); only where gemv_can_fuse_norm(M, K)
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
                              float* part, int* counters, const EpiParams& ep, int num_sms, cudaStream_t st,
-                             const CUtensorMap* wmap = nullptr);
+                             const CUtensorMap* wmap = nullptr, const float* h_norm = nullptr,
+                             const void* w_norm = nullptr, float eps = 0.f);
+bool gemv_can_fuse_norm(int M, int K);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -12,7 +12,9 @@
 //   xn * W13^T -> silu(a) * b -> g                                       (SwiGLU epilogue)
 //   h += g * W2^T                                                        (residual epilogue)
 // Whole-model calls add the embedding gather before and the final RMSNorm
-// plus the LM head after ("... notes", Transformer.forward).
+// plus the LM head after ("... notes", Transformer.forward). A decode call of
+// at most 4 tokens at dim <= 4096 computes each rmsnorm inside the GEMV that
+// reads xn (same arithmetic, no launch of its own).
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
@@ -200,21 +202,29 @@ EpiParams epi_base(llama_ctx* c, int kind, int M, int N) {
 // W is one of the library's weight matrices: row-major fp32 in fp32 mode,
 // 128 x 64 bf16 tiles (tile_weights) in bf16 mode.
 // wmap: W's tensor map (tiled layout, 128-row boxes), encoded when the weights were set.
+// h_norm / w_norm (decode GEMV only, fuse_norm): A = RMSNorm(h_norm) computed by the GEMV itself.
+bool gemm_is_gemv(const llama_ctx* c, int M, int K) { return c->bf16 && M <= 32 && K % 64 == 0; }
 int gemm(llama_ctx* c, const void* A, const void* W, const CUtensorMap* wmap, int M, int N, int K, const EpiParams& ep,
-         cudaStream_t st) {
+         cudaStream_t st, const float* h_norm = nullptr, const void* w_norm = nullptr) {
+  if (h_norm && !gemm_is_gemv(c, M, K)) return LLAMA_ERR_INVALID_ARGS;
   if (!c->bf16) {
     launch_gemm_simt<float>(A, W, M, N, K, ep, st);
     return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
   }
-  if (M <= 32 && K % 64 == 0) {
+  if (gemm_is_gemv(c, M, K)) {
     GemvPlan p = plan_gemv(M, N, K, c->num_sms);
     if (p.part_floats > c->part_floats || p.row_blocks > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
-    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st, wmap) == cudaSuccess
+    return launch_gemv_bf16(A, W, 1, M, N, K, p, c->part, c->counters, ep, c->num_sms, st, wmap, h_norm, w_norm,
+                            c->a.norm_eps) == cudaSuccess
                ? LLAMA_OK
                : LLAMA_ERR_CUDA;
   }
   return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st, wmap) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
+
+// A decode call of a few tokens (bf16, dim <= 4096) computes both RMSNorms
+// inside the GEMVs that read them: no RMSNorm launch, no xn round trip.
+bool fuse_norm(const llama_ctx* c, int M) { return gemm_is_gemv(c, M, c->dim) && gemv_can_fuse_norm(M, c->dim); }
 
 // elements of one stored weight matrix [N][K]: tiles in bf16 mode, row-major in fp32 mode
 size_t weight_elems(const llama_ctx* c, size_t N, size_t K) { return c->bf16 ? tiled_weight_elems(N, K) : N * K; }
@@ -290,8 +300,10 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
     r = run_block_persistent(c, layer, h, B, sp_dev, sp_host, st);
     return r == 1 ? LLAMA_ERR_INVALID_ARGS : r;
   }
-  if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
-               : launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
+  const bool fnorm = fuse_norm(c, M);
+  if (!fnorm && (c->bf16 ? launch_rmsnorm<bf16>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
+                         : launch_rmsnorm<float>(h, Ly.attn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) !=
+                    cudaSuccess)
     return LLAMA_ERR_CUDA;
 
   EpiParams e = epi_base(c, EPI_QKV_ROPE, M, c->n_qkv);
@@ -306,7 +318,9 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.Hkv = c->Hkv;
   e.D = c->D;
   e.S_max = c->S;
-  if ((r = gemm(c, c->xn, Ly.wqkv, &Ly.map_w[0], M, c->n_qkv, c->dim, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.wqkv, &Ly.map_w[0], M, c->n_qkv, c->dim, e, st, fnorm ? h : nullptr,
+                fnorm ? Ly.attn_norm : nullptr)))
+    return r;
 
   cudaError_t ce;
   if (!c->bf16) {
@@ -338,13 +352,16 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   e.ld_out = c->dim;
   if ((r = gemm(c, c->o, Ly.wo, &Ly.map_w[1], M, c->dim, HD, e, st))) return r;
 
-  if ((c->bf16 ? launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
-               : launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) != cudaSuccess)
+  if (!fnorm && (c->bf16 ? launch_rmsnorm<bf16>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)
+                         : launch_rmsnorm<float>(h, Ly.ffn_norm, c->xn, M, c->dim, c->a.norm_eps, 1, 0, st)) !=
+                    cudaSuccess)
     return LLAMA_ERR_CUDA;
 
   e = epi_base(c, EPI_SWIGLU, M, 2 * c->F);
   e.g_out = c->g;
-  if ((r = gemm(c, c->xn, Ly.w13, &Ly.map_w[2], M, 2 * c->F, c->dim, e, st))) return r;
+  if ((r = gemm(c, c->xn, Ly.w13, &Ly.map_w[2], M, 2 * c->F, c->dim, e, st, fnorm ? h : nullptr,
+                fnorm ? Ly.ffn_norm : nullptr)))
+    return r;
 
   e = epi_base(c, EPI_RESIDUAL, M, c->dim);
   e.out = h;

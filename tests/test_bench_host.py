@@ -61,3 +61,28 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 3
+
+
+def test_decode_launch_count_per_block():
+    """The `gpu_launches` claim: 5 kernels per block and decode step where the
+    GEMVs compute the RMSNorms (bf16, at most 4 tokens, dim <= 4096), 7 where the
+    RMSNorms are launches of their own, 1 for the persistent decode kernel."""
+    import bench
+    from llama_decoder_block_kv_b200 import synth
+    w7 = synth.WORKLOADS["llama7b-layer"]
+    w70 = synth.WORKLOADS["llama70b-layer"]
+    w8 = synth.WORKLOADS["llama3-8b-decode"]
+    wt = synth.WORKLOADS["tiny-fp32"]
+    assert bench.decode_launches_per_block(w7, 1) == 5
+    assert bench.decode_launches_per_block(w7, 4) == 5
+    assert bench.decode_launches_per_block(w7, 5) == 7
+    assert bench.decode_launches_per_block(w70, 16) == 7    # dim 8192
+    assert bench.decode_launches_per_block(w8, 32) == 7     # 32 tokens
+    assert bench.decode_launches_per_block(wt, 1) == 7      # fp32: the SIMT path
+    saved = bench.DECODE_KERNEL
+    try:
+        bench.DECODE_KERNEL = "persistent"
+        assert bench.decode_launches_per_block(w7, 1) == 1
+        assert bench.decode_launches_per_block(wt, 1) == 7
+    finally:
+        bench.DECODE_KERNEL = saved

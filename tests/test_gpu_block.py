@@ -66,6 +66,30 @@ def test_block_prefill_chunk_and_decode(dim, H, Hkv):
         pair.close()
 
 
+@pytest.mark.parametrize("dim,H,Hkv,Bsz", [(1024, 8, 2, 1), (1024, 8, 2, 4), (1024, 8, 2, 5), (2048, 16, 16, 1),
+                                           (2048, 16, 4, 3), (192, 3, 1, 2)])
+def test_decode_rmsnorm_inside_the_gemv(dim, H, Hkv, Bsz):
+    """Decode calls of at most 4 tokens at dim <= 4096 compute both RMSNorms
+    inside the GEMVs that read them (the norm weight copied into shared memory,
+    the normalised rows kept resident); 5 tokens take the RMSNorm launches.
+    Both against the oracle over a few steps with per-sequence positions and
+    random norm weights, including dim 192 (K of 3 stages, most consumer
+    threads holding no chunk of the row). dim 4096, the largest fused K, is
+    the 7B-layer workload test (test_gpu_workloads.py, batch-1 decode under
+    the full-size bound)."""
+    w = _wl(dim, H, Hkv, Bm=Bsz, S=128)
+    pair = Pair(w)
+    try:
+        h = synth.hidden(w, (Bsz, 21, dim), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        pos = np.full(Bsz, 21) if Bsz > 1 else 21  # device positions for batches, a scalar for one
+        for i in range(3):
+            h = synth.hidden(w, (Bsz, 1, dim), call=1 + i)
+            _run(pair, h, pos + i, BF16_HIDDEN_ABS)
+    finally:
+        pair.close()
+
+
 def test_block_ragged_decode_positions():
     w = _wl(512, 4, 2, Bm=4, S=512)
     pair = Pair(w)
