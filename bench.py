@@ -916,6 +916,8 @@ def main():
     ap.add_argument("--clock-log", default=None, help="directory for the per-rank clock sample CSV")
     ap.add_argument("--decode-kernel", default="auto", choices=sorted(DECODE_KERNELS),
                     help="decode-step launch structure (llama_set_decode_kernel)")
+    ap.add_argument("--gemv-mma", default="auto", choices=["auto", "warp", "tcgen05"],
+                    help="product of the 9..32-token decode GEMV (llama_set_decode_linear_mma)")
     ap.add_argument("--decode-attention", default="auto", choices=sorted(DECODE_ATTENTIONS),
                     help="decode attention kernel of the per-step launches (llama_set_decode_attention)")
     args = ap.parse_args()
@@ -933,6 +935,8 @@ def main():
         if out is not None:
             print(json.dumps(out), flush=True)
         return
+    B.llama_set_decode_linear_mma({"auto": B.LLAMA_GEMV_MMA_AUTO, "warp": B.LLAMA_GEMV_MMA_WARP,
+                                   "tcgen05": B.LLAMA_GEMV_MMA_TCGEN05}[args.gemv_mma])
     world, rank, local = dist_setup()
     out = run_ours(args, world, rank, local)
     if rank == 0:

@@ -84,6 +84,11 @@ extern "C" {
 #define LLAMA_ATTN_CHUNKED 1 /* a CTA per (sequence, kv head group, chunk of keys) */
 #define LLAMA_ATTN_STREAMK 2 /* the key tiles of all sequences dealt out evenly over two CTAs per SM */
 
+/* Product of the batched decode GEMV (9..32 tokens), llama_set_decode_linear_mma */
+#define LLAMA_GEMV_MMA_AUTO 0    /* the library's choice: currently WARP (measured as fast or faster) */
+#define LLAMA_GEMV_MMA_WARP 1    /* warp-level mma.sync, weights and tokens through ldmatrix */
+#define LLAMA_GEMV_MMA_TCGEN05 2 /* tcgen05.mma from shared memory, accumulators in tensor memory */
+
 /*
  * ModelArgs of the notes' section 3 code plus rope_theta ("灵哥讲llama3(中)",
  * Transformer class) and the storage type.
@@ -304,6 +309,19 @@ int llama_set_decode_kernel(llama_ctx* ctx, int mode);
  * applies to calls made after it.
  */
 int llama_set_decode_attention(llama_ctx* ctx, int mode);
+
+/*
+ * Choose how the decode GEMV (the weight-streaming kernel of linears with 9 to
+ * 32 tokens: every decode linear of a batch of 9..32 sequences, and
+ * llama_linear's LLAMA_PATH_GEMV) forms its products (LLAMA_GEMV_MMA_*). Both
+ * compute y = x W^T of the notes' Attention and FeedForward linears with fp32
+ * accumulation; they differ only in the order of fp32 sums within a 64-wide
+ * k stage. The pages have no counterpart: this is a kernel switch of the
+ * library. Process-wide (every context and llama_linear); calls of up to 8
+ * tokens always take the warp-level form. Returns LLAMA_ERR_INVALID_ARGS for
+ * another mode. Not stream-ordered: it applies to launches made after it.
+ */
+int llama_set_decode_linear_mma(int mode);
 
 /*
  * Synchronise the device, then return and clear the device flags: LLAMA_OK,

@@ -32,13 +32,14 @@ LLAMA_PATH_AUTO, LLAMA_PATH_TCGEN05, LLAMA_PATH_GEMV, LLAMA_PATH_SIMT = 0, 1, 2,
 LLAMA_WEIGHTS_TILED = 16
 LLAMA_DECODE_AUTO, LLAMA_DECODE_LAYERED, LLAMA_DECODE_PERSISTENT = 0, 1, 2
 LLAMA_ATTN_AUTO, LLAMA_ATTN_CHUNKED, LLAMA_ATTN_STREAMK = 0, 1, 2
+LLAMA_GEMV_MMA_AUTO, LLAMA_GEMV_MMA_WARP, LLAMA_GEMV_MMA_TCGEN05 = 0, 1, 2
 
 # every symbol the header declares (checked by the CPU test suite)
 EXPORTED = ("llama_ffn_hidden", "llama_create", "llama_destroy", "llama_set_layer", "llama_set_embed_norm_head",
             "llama_reserve", "llama_forward", "llama_forward_ragged", "llama_block_forward", "llama_kv_read",
             "llama_kv_write", "llama_reset", "llama_get_error", "llama_strerror", "llama_linear",
             "llama_linear_noalloc", "llama_linear_noalloc_status", "llama_sample", "llama_generate", "llama_set_decode_kernel",
-            "llama_set_decode_attention", "llama_tile_weights",
+            "llama_set_decode_attention", "llama_set_decode_linear_mma", "llama_tile_weights",
             "llama_selftest_bounded_wait", "llama_set_alloc_limit", "llama_allocated_bytes",
             "llama_selfcheck_plans")
 
@@ -92,6 +93,7 @@ def lib() -> ctypes.CDLL:
         L.llama_generate.argtypes = [vp, vp, vp, i, i, i, f, f, vp, vp]
         L.llama_set_decode_kernel.argtypes = [vp, i]
         L.llama_set_decode_attention.argtypes = [vp, i]
+        L.llama_set_decode_linear_mma.argtypes = [i]
         L.llama_tile_weights.argtypes = [vp, vp, i, i, vp]
         L.llama_selftest_bounded_wait.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_double)]
         L.llama_set_alloc_limit.argtypes = [ctypes.c_uint64]
@@ -224,6 +226,11 @@ def llama_reset(ctx) -> None:
 
 def llama_set_decode_kernel(ctx, mode: int) -> None:
     _check(lib().llama_set_decode_kernel(ctx, int(mode)), "llama_set_decode_kernel")
+
+
+def llama_set_decode_linear_mma(mode: int) -> None:
+    """Product of the 9..32-token decode GEMV (LLAMA_GEMV_MMA_*), process-wide."""
+    _check(lib().llama_set_decode_linear_mma(int(mode)), "llama_set_decode_linear_mma")
 
 
 def llama_set_decode_attention(ctx, mode: int) -> None:

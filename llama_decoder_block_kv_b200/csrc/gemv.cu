@@ -375,6 +375,236 @@ __global__ void __launch_bounds__(160, 1)
   }
 }
 
+// tcgen05 form of the same kernel for 9..32 tokens (MB = 2 or 4; 17..24 tokens
+// run as MB = 4, the X box's rows past M filled with zeros by the copy). The
+// ring, the stream-K ranges, the partial workspace and the epilogue are those
+// of llama_decode_linear_kernel; only the product changes: a sixth warp's
+// elected thread issues tcgen05.mma with the stage's 128 weight rows as A
+// (M = 128) and its 8 MB token rows as B (N = 8 MB), 4 MMAs of 16 k per stage,
+// accumulating in tensor memory (two 32-column buffers, alternating between
+// the row-block segments of the CTA's range), and frees the stage with a
+// commit. The tensor core reads each stage once, where the warp-level form
+// issues 32 mma.sync and 16 ldmatrix per warp and stage at 32 tokens (32 KB of
+// shared-memory reads per 20 KB stage); measured, the two run at the same
+// speed (see g_gemv_mma), so the warp-level form stays the default and this
+// one is selected with llama_set_decode_linear_mma. The four epilogue warps read
+// their 32 rows of the accumulator with tcgen05.ld (lane = weight row, column
+// = token) into the same [token][row] staging tile.
+template <int MB>
+__global__ void __launch_bounds__(192, 1)
+    llama_decode_linear_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                                  int M, int N, int nk, int total, int tiled, float* __restrict__ part,
+                                  int* __restrict__ counters, EpiParams ep) {
+  static_assert(MB == 2 || MB == 4, "N = 8 MB must be a multiple of 16 for M = 128");
+  constexpr int STAGES = stages(MB);
+  constexpr uint32_t SB = stage_bytes(MB);
+  constexpr uint32_t IDESC = make_idesc_bf16(RPC, 8 * MB);
+  constexpr uint32_t TMEM_COLS = 64;  // two accumulator buffers of 32 columns
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* os = reinterpret_cast<float*>(base + STAGES * SB);
+  uint64_t* full = reinterpret_cast<uint64_t*>(os + 8 * MB * OS);
+  uint64_t* empty = full + STAGES;
+  uint64_t* afull = empty + STAGES;  // [2] accumulator buffer complete
+  uint64_t* aempty = afull + 2;      // [2] accumulator buffer read by the four epilogue warps
+  uint64_t* drained = aempty + 2;    // every MMA of the CTA finished
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_last;
+  __shared__ int s_abort;
+  volatile int* abort_flag = &s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grid = gridDim.x, cta = blockIdx.x;
+  const int sbeg = sk_begin(cta, total, grid), send = sk_begin(cta + 1, total, grid);
+
+  if (tid == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&afull[i], 1);
+      mbar_init(&aempty[i], 4);
+    }
+    mbar_init(drained, 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&s_tmem, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tensormap(&map_w);
+      prefetch_tensormap(&map_x);
+      const int pre = min(STAGES, send - sbeg);
+      for (int i = 0; i < pre; ++i) {
+        const int x = sbeg + i, rb = x / nk, ks = x - rb * nk;
+        mbar_arrive_expect_tx(&full[i], SB);
+        tma_load_2d(base + i * SB, &map_w, &full[i], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
+      }
+      pdl_wait();
+      pdl_trigger();
+      for (int i = 0; i < pre; ++i) {
+        const int x = sbeg + i, ks = x - (x / nk) * nk;
+        tma_load_2d(base + i * SB + W_BYTES, &map_x, &full[i], ks * KB, 0);
+      }
+      int j = pre;
+      for (int x = sbeg + pre; x < send; ++x, ++j) {
+        const int st = j % STAGES;
+        if (!wait_or_abort(&empty[st], ((j / STAGES) & 1) ^ 1, ep.err, abort_flag)) break;
+        const int rb = x / nk, ks = x - rb * nk;
+        uint8_t* dst = base + st * SB;
+        mbar_arrive_expect_tx(&full[st], SB);
+        tma_load_2d(dst, &map_w, &full[st], tiled ? 0 : ks * KB, tiled ? (rb * nk + ks) * RPC : rb * RPC);
+        tma_load_2d(dst + W_BYTES, &map_x, &full[st], ks * KB, 0);
+      }
+      // the CTA must not retire while a copy into its shared memory is in flight
+      for (int i = (j > STAGES ? j - STAGES : 0); i < j; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, ep.err);
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA issuer
+    pdl_trigger();
+    if (lane == 0) {
+      int j = 0, seg = 0;
+      bool ok = true;
+      for (int x = sbeg; x < send && ok; ++seg) {
+        const int rb = x / nk, seg_end = min(send, (rb + 1) * nk);
+        const int buf = seg & 1;
+        if (!wait_or_abort(&aempty[buf], ((seg >> 1) & 1) ^ 1, ep.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * 32;
+        for (bool first = true; x < seg_end; ++x, ++j, first = false) {
+          const int st = j % STAGES;
+          if (!wait_or_abort(&full[st], (j / STAGES) & 1, ep.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t wa = smem_u32(base + st * SB), xa = wa + W_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk)
+            tc_mma_bf16(d, make_sw128_desc(wa + kk * 32), make_sw128_desc(xa + kk * 32), IDESC,
+                        (first && kk == 0) ? 0u : 1u);
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(&afull[buf]);
+      }
+      // every MMA of this thread has finished before the tensor memory is released
+      tc_commit(drained);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drained, 0) && global_timer_ns() - t0 < LLAMA_WAIT_LIMIT_NS) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------- epilogue warps 0-3
+    pdl_wait();
+    pdl_trigger();
+    const int row = warp * 32 + lane;  // weight row of the row block = TMEM lane
+    int seg = 0;
+    for (int x = sbeg; x < send; ++seg) {
+      const int rb = x / nk;
+      const int seg_beg = x, seg_end = min(send, (rb + 1) * nk);
+      x = seg_end;
+      const int buf = seg & 1;
+      const bool ok = wait_or_abort(&afull[buf], (seg >> 1) & 1, ep.err, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is warp-collective
+      tc_fence_after();
+      float v[32];
+      tmem_ld_32cols(tmem + ((uint32_t)(warp * 32) << 16) + buf * 32, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aempty[buf]);
+
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+      for (int m = 0; m < 8 * MB; ++m) os[m * OS + row] = v[m];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+
+      const int nbase = rb * RPC;
+      if (seg_beg == rb * nk && seg_end == (rb + 1) * nk) {
+        for (int c = tid; c < M * (RPC / 8); c += 128) {
+          const int m = c / (RPC / 8), jc = c - m * (RPC / 8);
+          const int n = nbase + jc * 8;
+          if (n < N) {
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = os[m * OS + jc * 8 + e];
+            epilogue8<bf16>(ep, m, n, o);
+          }
+        }
+        continue;
+      }
+      const int c_first = sk_owner(rb * nk, total, grid);
+      const int c_last = sk_owner((rb + 1) * nk - 1, total, grid);
+      const int count = c_last - c_first + 1, slot = cta - c_first;
+      for (int e = tid; e < M * (RPC / 4); e += 128) {
+        const int m = e / (RPC / 4), jc = e - m * (RPC / 4);
+        const int n = nbase + jc * 4;
+        if (n < N) {
+          const float4 o = make_float4(os[m * OS + jc * 4], os[m * OS + jc * 4 + 1], os[m * OS + jc * 4 + 2],
+                                       os[m * OS + jc * 4 + 3]);
+          __stcg(reinterpret_cast<float4*>(part + ((size_t)slot * M + m) * N + n), o);
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (tid == 0) s_last = (atomic_add_acq_rel(&counters[rb], 1) == count - 1);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!s_last) continue;
+      for (int c = tid; c < M * (RPC / 8); c += 128) {
+        const int m = c / (RPC / 8), jc = c - m * (RPC / 8);
+        const int n = nbase + jc * 8;
+        if (n >= N) continue;
+        const bool res = ep.kind == EPI_RESIDUAL;
+        float4* hp = res ? reinterpret_cast<float4*>(ep.out + (size_t)m * ep.ld_out + n) : nullptr;
+        float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0;
+        if (res) {
+          h0 = hp[0];
+          h1 = hp[1];
+        }
+        float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int sl0 = 0; sl0 < count; sl0 += 8) {
+          float4 pa[8], pb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (sl0 + i < count) {
+              const float4* src = reinterpret_cast<const float4*>(part + ((size_t)(sl0 + i) * M + m) * N + n);
+              pa[i] = __ldcg(src);
+              pb[i] = __ldcg(src + 1);
+            }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (sl0 + i < count) {
+              o[0] += pa[i].x; o[1] += pa[i].y; o[2] += pa[i].z; o[3] += pa[i].w;
+              o[4] += pb[i].x; o[5] += pb[i].y; o[6] += pb[i].z; o[7] += pb[i].w;
+            }
+        }
+        if (res) {
+          hp[0] = make_float4(h0.x + o[0], h0.y + o[1], h0.z + o[2], h0.w + o[3]);
+          hp[1] = make_float4(h1.x + o[4], h1.y + o[5], h1.z + o[6], h1.w + o[7]);
+        } else {
+          epilogue8<bf16>(ep, m, n, o);
+        }
+      }
+      if (tid == 0) counters[rb] = 0;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 // grid = one CTA per SM (fewer if there are fewer stages than SMs); the
 // partial workspace holds one [M][N] slice per contributor of the most-split
 // row block.
@@ -449,6 +679,34 @@ static cudaError_t launch_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M
                     p.total, tiled, part, counters, ep, h_norm, w_norm, eps);
 }
 
+template <int MB>
+static cudaError_t launch_tc_mb(const CUtensorMap& mw, const CUtensorMap& mx, int M, int N, const GemvPlan& p,
+                                int tiled, float* part, int* counters, const EpiParams& ep, cudaStream_t st) {
+  constexpr size_t smem = gemv_smem(MB) + 64;
+  static_assert(gemv_smem(MB) + 64 <= 232448, "tcgen05 decode GEMV shared memory");
+  static std::atomic<unsigned long long> attr{0};
+  cudaError_t e = ensure_smem(llama_decode_linear_tc_kernel<MB>, smem, attr);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(llama_decode_linear_tc_kernel<MB>, dim3(p.grid), dim3(192), smem, st, mw, mx, M, N, p.nk,
+                    p.total, tiled, part, counters, ep);
+}
+
+// Product of the batched (9..32-token) calls: LLAMA_GEMV_MMA_* (process-wide).
+// AUTO takes the warp-level form: measured on B200 (CUDA graph of back-to-back
+// launches, tiled weights, us per launch, warp-level against tcgen05): 32
+// tokens x [28672 x 4096] 44.2 / 45.4, [4096 x 14336] 27.0 / 27.2, [6144 x
+// 4096] 17.1 / 17.5, [4096 x 4096] 15.6 / 16.1; 16 tokens x [57344 x 8192]
+// 148.2 / 150.8, [8192 x 28672] 75.5 / 76.1; 24 tokens x [6144 x 4096] 15.5 /
+// 16.5. The product is not what bounds these calls (the 32-token weight
+// stream runs at the same speed either way).
+static std::atomic<int> g_gemv_mma{LLAMA_GEMV_MMA_AUTO};
+
+int set_gemv_mma(int mode) {
+  if (mode < LLAMA_GEMV_MMA_AUTO || mode > LLAMA_GEMV_MMA_TCGEN05) return -1;
+  g_gemv_mma.store(mode, std::memory_order_relaxed);
+  return 0;
+}
+
 bool gemv_can_fuse_norm(int M, int K) { return M >= 1 && M <= NORM_MAX_M && K % KB == 0 && K <= NORM_MAX_K; }
 
 cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int N, int K, const GemvPlan& p,
@@ -468,6 +726,13 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int
       return cudaErrorInvalidValue;
     return launch_mb<1, true>(mw, mw, M, N, p, tiled, part, counters, ep, st, h_norm,
                               reinterpret_cast<const bf16*>(w_norm), eps);
+  }
+  if (MB >= 2 && g_gemv_mma.load(std::memory_order_relaxed) == LLAMA_GEMV_MMA_TCGEN05) {
+    // 17..24 tokens take the 32-row box (rows past M read as zeros)
+    const int mbt = MB == 2 ? 2 : 4;
+    if (!make_tmap_bf16(&mx, X, M, K, 8 * mbt)) return cudaErrorInvalidValue;
+    return mbt == 2 ? launch_tc_mb<2>(mw, mx, M, N, p, tiled, part, counters, ep, st)
+                    : launch_tc_mb<4>(mw, mx, M, N, p, tiled, part, counters, ep, st);
   }
   if (!make_tmap_bf16(&mx, X, M, K, 8 * MB)) return cudaErrorInvalidValue;
   switch (MB) {

@@ -79,6 +79,8 @@ cudaError_t launch_gemv_bf16(const void* X, const void* W, int tiled, int M, int
                              const CUtensorMap* wmap = nullptr, const float* h_norm = nullptr,
                              const void* w_norm = nullptr, float eps = 0.f);
 bool gemv_can_fuse_norm(int M, int K);
+// LLAMA_GEMV_MMA_* for the 9..32-token calls (process-wide); -1 for another mode
+int set_gemv_mma(int mode);
 
 // gemm_tc.cu
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

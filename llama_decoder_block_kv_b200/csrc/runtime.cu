@@ -837,6 +837,10 @@ int llama_set_decode_attention(llama_ctx* c, int mode) {
   return LLAMA_OK;
 }
 
+int llama_set_decode_linear_mma(int mode) {
+  return set_gemv_mma(mode) == 0 ? LLAMA_OK : LLAMA_ERR_INVALID_ARGS;
+}
+
 int llama_set_decode_kernel(llama_ctx* c, int mode) {
   if (!c || mode < LLAMA_DECODE_AUTO || mode > LLAMA_DECODE_PERSISTENT) return LLAMA_ERR_INVALID_ARGS;
   c->decode_mode = mode;

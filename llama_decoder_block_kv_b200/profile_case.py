@@ -32,10 +32,14 @@ def main():
     ap.add_argument("--shape", default="7b", choices=["7b", "8b"],
                     help="prefill-attn: the LLaMA-7B layer (MHA) or the LLaMA-3-8B layer (GQA 32/8)")
     ap.add_argument("--batch", type=int, default=1, help="prefill-attn: sequences of T tokens")
+    ap.add_argument("--gemv-mma", default="auto", choices=["auto", "warp", "tcgen05"],
+                    help="gemv: the product of 9..32-token calls (llama_set_decode_linear_mma)")
     ap.add_argument("--row-major", action="store_true",
                     help="gemv / tc: pass the weights row-major instead of in the library's tile layout")
     a = ap.parse_args()
     torch.cuda.set_device(0)
+    B.llama_set_decode_linear_mma({"auto": B.LLAMA_GEMV_MMA_AUTO, "warp": B.LLAMA_GEMV_MMA_WARP,
+                                   "tcgen05": B.LLAMA_GEMV_MMA_TCGEN05}[a.gemv_mma])
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if a.kind in ("gemv", "tc", "simt"):

@@ -60,6 +60,31 @@ def test_gemv_split_k(M, N, K):
     _check(x, w, y)
 
 
+@pytest.mark.parametrize("mode", [B.LLAMA_GEMV_MMA_WARP, B.LLAMA_GEMV_MMA_TCGEN05])
+@pytest.mark.parametrize("M,N,K", [(9, 8, 128), (16, 12288, 4096), (17, 256, 11008), (24, 6144, 4096),
+                                   (32, 4096, 14336), (32, 28672, 4096), (13, 1000, 640)])
+def test_gemv_batched_both_products(mode, M, N, K):
+    """The 9..32-token decode GEMV with either product (warp-level mma.sync, or
+    tcgen05.mma into tensor memory with 17..24 tokens padded to a 32-row box):
+    against a float64 matmul, twice in a row (counters re-armed), including row
+    blocks that end inside one CTA's range and ragged N."""
+    x, w = _inputs(M, N, K, torch.bfloat16, 23)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    B.llama_set_decode_linear_mma(mode)
+    try:
+        for _ in range(2):
+            B.llama_linear(x, w, y, B.LLAMA_PATH_GEMV)
+        torch.cuda.synchronize()
+    finally:
+        B.llama_set_decode_linear_mma(B.LLAMA_GEMV_MMA_AUTO)
+    _check(x, w, y)
+
+
+def test_decode_linear_mma_mode_is_checked():
+    with pytest.raises(Exception):
+        B.llama_set_decode_linear_mma(3)
+
+
 @pytest.mark.parametrize("M,N,K,dt", [(33, 136, 200, torch.float32), (64, 64, 64, torch.float32),
                                       (5, 256, 96, torch.bfloat16)])
 def test_simt_gemm(M, N, K, dt):
