@@ -121,8 +121,79 @@ size_t simt_smem_bytes() {
   return ring > ctile ? ring : ctile;
 }
 
+// fp32 decode GEMV for a few tokens (M <= 8, K <= 1024, K % 4 == 0, N % 8 ==
+// 0): in the tiled kernel above a call of one token fills one row of a 64-row
+// tile and walks K in 16-wide steps, one dependent round trip per ring stage,
+// so a decode step of a small fp32 model is a chain of latencies. Here a CTA
+// of 8 warps computes 8 consecutive output columns for all M tokens, warp w
+// column n0 + w: each lane loads its K / 128 float4 of that weight row before
+// the dependency wait (the weights do not depend on the previous kernel), the
+// token rows are staged in shared memory after it, each sum is a warp
+// reduction, and M threads hand the 8 columns of their token to the shared
+// epilogue.
+namespace {
+constexpr int GV_KMAX = 1024, GV_MMAX = 8;
+}
+
+__global__ void __launch_bounds__(256)
+    gemv_f32_kernel(const float* __restrict__ A, const float* __restrict__ W, int M, int N, int K, EpiParams ep) {
+  __shared__ float4 xs[GV_MMAX * GV_KMAX / 4];  // the M token rows, GV_KMAX floats apart
+  __shared__ float res[GV_MMAX][8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * 8, n = n0 + warp;
+  const int K4 = K >> 2;
+  float4 wv[GV_KMAX / 128];
+#pragma unroll
+  for (int i = 0; i < GV_KMAX / 128; ++i) {
+    const int k4 = lane + 32 * i;
+    wv[i] = (n < N && k4 < K4) ? __ldg(reinterpret_cast<const float4*>(W + (size_t)n * K) + k4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  pdl_wait();
+  for (int i = tid; i < M * K4; i += 256) {
+    const int m = i / K4;
+    xs[m * (GV_KMAX / 4) + (i - m * K4)] = reinterpret_cast<const float4*>(A)[i];
+  }
+  __syncthreads();
+  pdl_trigger();
+#pragma unroll
+  for (int m = 0; m < GV_MMAX; ++m) {
+    if (m >= M) break;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < GV_KMAX / 128; ++i) {
+      const int k4 = lane + 32 * i;
+      if (k4 < K4) {
+        const float4 x = xs[m * (GV_KMAX / 4) + k4];
+        acc = fmaf(wv[i].x, x.x, acc);
+        acc = fmaf(wv[i].y, x.y, acc);
+        acc = fmaf(wv[i].z, x.z, acc);
+        acc = fmaf(wv[i].w, x.w, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) res[m][warp] = acc;
+  }
+  __syncthreads();
+  if (tid < M) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = res[tid][e];
+    epilogue8<float>(ep, tid, n0, v);
+  }
+}
+
 template <typename T>
 void launch_gemm_simt(const void* A, const void* W, int M, int N, int K, const EpiParams& ep, cudaStream_t st) {
+  if constexpr (sizeof(T) == 4) {
+    if (M >= 1 && M <= GV_MMAX && K <= GV_KMAX && K % 4 == 0 && N % 8 == 0 &&
+        !(reinterpret_cast<uintptr_t>(A) & 15) && !(reinterpret_cast<uintptr_t>(W) & 15)) {
+      launch_pdl(gemv_f32_kernel, dim3(N / 8), dim3(256), 0, st, reinterpret_cast<const float*>(A),
+                 reinterpret_cast<const float*>(W), M, N, K, ep);
+      return;
+    }
+  }
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
   launch_pdl(gemm_simt_kernel<T>, grid, dim3(THREADS), simt_smem_bytes<T>(), st, reinterpret_cast<const T*>(A),
              reinterpret_cast<const T*>(W), M, N, K, ep);

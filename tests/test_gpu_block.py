@@ -230,3 +230,31 @@ def test_chunked_prefill_with_per_sequence_positions(dim, H, Hkv):
         assert_cache_matches(pair, 0, written, 2e-2)
     finally:
         pair.close()
+
+
+@pytest.mark.parametrize("mma", [B.LLAMA_GEMV_MMA_WARP, B.LLAMA_GEMV_MMA_TCGEN05])
+@pytest.mark.parametrize("Bsz", [16, 19, 32])
+def test_batched_decode_with_either_gemv_product(mma, Bsz):
+    """Decode steps of 16, 19 and 32 sequences run the batched decode GEMV with
+    every epilogue (RoPE and the cache append on wqkv, the residual add on wo
+    and w2, SiLU times the gate on w1|w3); either product of that kernel
+    (warp-level mma.sync, or tcgen05.mma into tensor memory with 19 tokens in
+    a 32-row box) against the oracle, with per-sequence positions, and the
+    cache slots written."""
+    w = _wl(1024, 8, 2, Bm=Bsz, S=64)
+    pair = Pair(w)
+    B.llama_set_decode_linear_mma(mma)
+    try:
+        h = synth.hidden(w, (Bsz, 9, 1024), call=0)
+        _run(pair, h, 0, BF16_HIDDEN_ABS)
+        pos = 9 + (np.arange(Bsz) % 5)
+        written = np.zeros((w.max_batch_size, w.max_seq_len), dtype=bool)
+        written[:Bsz, :9] = True
+        for i in range(3):
+            h = synth.hidden(w, (Bsz, 1, 1024), call=1 + i)
+            _run(pair, h, pos + i, BF16_HIDDEN_ABS)
+            written[np.arange(Bsz), pos + i] = True
+        assert_cache_matches(pair, 0, written, 2e-2)
+    finally:
+        B.llama_set_decode_linear_mma(B.LLAMA_GEMV_MMA_AUTO)
+        pair.close()

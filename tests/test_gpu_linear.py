@@ -86,7 +86,11 @@ def test_decode_linear_mma_mode_is_checked():
 
 
 @pytest.mark.parametrize("M,N,K,dt", [(33, 136, 200, torch.float32), (64, 64, 64, torch.float32),
-                                      (5, 256, 96, torch.bfloat16)])
+                                      (5, 256, 96, torch.bfloat16),
+                                      # fp32 calls of up to 8 tokens take the warp-per-column GEMV
+                                      (1, 1000, 256, torch.float32), (8, 1536, 768, torch.float32),
+                                      (3, 136, 200, torch.float32), (7, 64, 1024, torch.float32),
+                                      (9, 1536, 768, torch.float32), (2, 512, 1032, torch.float32)])
 def test_simt_gemm(M, N, K, dt):
     x, w = _inputs(M, N, K, dt, 31)
     y = torch.full((M, N), float("nan"), device="cuda")
