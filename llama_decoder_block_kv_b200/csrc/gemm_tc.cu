@@ -236,7 +236,7 @@ constexpr size_t P_SMEM = 1024 + (size_t)P_STAGES * (P_A_BYTES + P_B_BYTES) + 25
 template <typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, int M,
-                        int N, int K, EpiParams ep) {
+                        int N, int K, EpiParams ep, int splits, float* __restrict__ ws, int* __restrict__ sync) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base;
@@ -255,6 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const int num_m = (M + 255) / 256, num_n = (N + P_BN - 1) / P_BN;
   const int num_tiles = num_m * num_n;
   const int num_k = (K + BK - 1) / BK;
+  const int units = num_tiles * splits;  // (tile, k half) work units, the halves of a tile adjacent
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P_STAGES; ++i) {
@@ -292,9 +293,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       // ------------------------------------------------------------ producer (both CTAs)
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+      for (int u = pair; u < units && ok; u += npairs) {
+        const int tile = u / splits, s = u - tile * splits;
         const TileCoord tc = tile_coord(tile, num_m, num_n);
-        for (int kb = 0; kb < num_k; ++kb, ++it) {
+        for (int kb = s * num_k / splits; kb < (s + 1) * num_k / splits; ++kb, ++it) {
           const int stage = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
           if (!wait_or_abort(&empty[stage], ph ^ 1, ep.err, abort_flag)) {
@@ -328,7 +330,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       constexpr uint32_t idesc = idesc2_bf16(256, P_BN, false);
       int it = 0, local = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++local) {
+      for (int u = pair; u < units && ok; u += npairs, ++local) {
+        const int s = u % splits;
+        const int kb0 = s * num_k / splits, kb1 = (s + 1) * num_k / splits;
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
         if (!wait_cluster_or_abort(&tempty[acc], aph ^ 1, ep.err, abort_flag)) {
@@ -337,7 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + acc * P_BN;
-        for (int kb = 0; kb < num_k; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int stage = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
           if (!wait_or_abort(&full[stage], ph, ep.err, abort_flag)) {
@@ -350,7 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             mma2_ss(d, make_sw128_desc(a_addr + kk * 32), make_sw128_desc(b_addr + kk * 32), idesc,
-                    (kb | kk) != 0 ? 1u : 0u);
+                    (kb != kb0 || kk != 0) ? 1u : 0u);
           commit2(&empty[stage]);
         }
         if (!ok) break;
@@ -367,7 +371,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     int local = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
+    for (int u = pair; u < units; u += npairs, ++local) {
+      const int tile = u / splits;
       const TileCoord tc = tile_coord(tile, num_m, num_n);
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
@@ -375,10 +380,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is warp-collective
       tc_fence_after();
       const int m = tc.mb * 256 + (int)rank * 128 + row;
+      const uint32_t tacc = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
+      // Split tiles: the warp's 32 rows of the two k halves meet here. The
+      // first half to finish stores its sums ([column][row], 32 KB per warp)
+      // and raises a flag; the second adds them to its own and runs the
+      // epilogue (p0 + p1 = p1 + p0 in fp32, so the bits do not depend on
+      // which finished first), then re-arms the counter and the flag.
+      bool first = false, merge = false;
+      float* wp = nullptr;
+      int* cnt = nullptr;
+      if (splits > 1) {
+        const int slot = (tile * 2 + (int)rank) * 4 + quarter;
+        cnt = sync + 2 * slot;
+        wp = ws + (size_t)slot * (P_BN * 32);
+        int f = 0;
+        if (lane == 0) f = atomic_add_acq_rel(cnt, 1) == 0;
+        first = __shfl_sync(0xffffffffu, f, 0) != 0;
+        if (!first) {
+          int got = 1;
+          if (lane == 0) {
+            const uint64_t t0 = global_timer_ns();
+            while (!(got = ld_acquire_gpu(cnt + 1)) && global_timer_ns() - t0 < LLAMA_WAIT_LIMIT_NS) {
+            }
+            if (!got) atomicOr(ep.err, LLAMA_DEV_TIMEOUT);
+          }
+          merge = __shfl_sync(0xffffffffu, got, 0) != 0;
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < P_BN / 32; ++c) {
         float v[32];
-        tmem_ld_32cols(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + c * 32, v);
+        tmem_ld_32cols(tacc + c * 32, v);
+        if (first) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) __stcg(wp + (c * 32 + j) * 32 + lane, v[j]);
+          continue;
+        }
+        if (merge) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] += __ldcg(wp + (c * 32 + j) * 32 + lane);
+        }
         if (m < M) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -386,6 +427,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             if (n < N) epilogue8<T>(ep, m, n, v + j * 8);
           }
         }
+      }
+      if (first) {
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          st_release_gpu(cnt + 1, 1);
+        }
+      } else if (splits > 1 && lane == 0) {
+        cnt[0] = 0;
+        cnt[1] = 0;
       }
       tc_fence_before();
       // the reads above have completed (tcgen05.ld waits), so rank 1's arrival can be relaxed
@@ -487,16 +538,21 @@ static cudaError_t launch_tc(const void* A, const void* B, int b_tiled, int M, i
 
 // CTA pairs over 256 x 256 tiles; B is the library's tiled weights (its map, 128-row boxes)
 static cudaError_t launch_tc_pair(const void* A, const CUtensorMap& mb, int M, int N, int K, const EpiParams& ep,
-                                  int num_sms, cudaStream_t st) {
+                                  int num_sms, cudaStream_t st, int splits, float* ws, int* sync) {
   CUtensorMap ma;
   if (!make_tmap_bf16(&ma, A, M, K, BM)) return cudaErrorInvalidValue;
   static std::atomic<unsigned long long> attr{0};
   cudaError_t e = ensure_smem(gemm_tc_pair_kernel<bf16>, P_SMEM, attr);
   if (e != cudaSuccess) return e;
-  const int tiles = ((M + 255) / 256) * ((N + P_BN - 1) / P_BN);
-  const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  return launch_pdl(gemm_tc_pair_kernel<bf16>, dim3(2 * pairs), dim3(192), P_SMEM, st, ma, mb, M, N, K, ep);
+  const int units = ((M + 255) / 256) * ((N + P_BN - 1) / P_BN) * splits;
+  const int pairs = units < num_sms / 2 ? units : num_sms / 2;
+  return launch_pdl(gemm_tc_pair_kernel<bf16>, dim3(2 * pairs), dim3(192), P_SMEM, st, ma, mb, M, N, K, ep, splits,
+                    ws, sync);
 }
+
+size_t gemm_split_ws_floats(int tiles) { return (size_t)tiles * 2 * 128 * P_BN; }
+size_t gemm_split_sync_ints(int tiles) { return (size_t)tiles * 2 * 4 * 2; }
+int gemm_split_max_tiles(int num_sms) { return 3 * (num_sms / 2); }
 
 // The tile shape with the smallest estimate of waves x tile time, in units of a
 // 1-SM 128 x 256 tile: 1-SM 128 x 128 tiles 0.5, 128 x 256 tiles 1, CTA-pair
@@ -504,7 +560,7 @@ static cudaError_t launch_tc_pair(const void* A, const CUtensorMap& mb, int M, i
 // and whole GEMMs measured 0.69-0.75 of the single-CTA time); the pair form for
 // weights in the library's tile layout only.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
-                           int num_sms, cudaStream_t st, const CUtensorMap* bmap) {
+                           int num_sms, cudaStream_t st, const CUtensorMap* bmap, const GemmSplitWs* split) {
   const int num_m = (M + BM - 1) / BM;
   const int t256 = num_m * ((N + 255) / 256);
   const int t128 = num_m * ((N + 127) / 128);
@@ -514,14 +570,29 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int
     return (double)waves * cost;  // time ~ waves x per-tile cost
   };
   const double e128 = eff(t128, num_sms, 0.5), e256 = eff(t256, num_sms, 1.0);
-  const double epair = eff(tpair, num_sms / 2, 0.7);
+  double epair = eff(tpair, num_sms / 2, 0.7);
+  // Two k halves per pair tile (run on different pairs; the second to finish
+  // adds the first's partial sums) where that fills pairs a single wave of
+  // whole tiles leaves idle. A half costs 0.35 plus 12 / num_k for the
+  // partial tile's round trip through L2 and the unit's fixed cost, fitted on
+  // B200 at M = 512: N = 4096, K = 11008 took 47.0 us against 61.6 us on
+  // 128 x 128 tiles, while K = 4096 (28.6 against 26.6 us) and the two-wave
+  // shapes N = 12288 and 22016 at K = 4096 (65.7 / 97.5 against 58.6 / 86.5 us
+  // unsplit) were slower.
+  const int num_k = (K + BK - 1) / BK;
+  const bool can_split = split && split->ws && split->sync && tpair <= split->tiles &&
+                         tpair <= gemm_split_max_tiles(num_sms) && num_k >= 8;
+  const double esplit = can_split ? eff(2 * tpair, num_sms / 2, 0.35 + 12.0 / num_k) : 1e30;
+  const int splits = esplit < epair ? 2 : 1;
+  if (splits == 2) epair = esplit;
   if (b_tiled && N % 256 == 0 && num_sms >= 2 && epair < e128 && epair < e256) {
     CUtensorMap mb;
     if (bmap)
       mb = *bmap;  // the library's weights: encoded once when they were set
     else if (!make_tmap_weights(&mb, B, 1, N, K, 128))
       return cudaErrorInvalidValue;
-    return launch_tc_pair(A, mb, M, N, K, ep, num_sms, st);
+    return launch_tc_pair(A, mb, M, N, K, ep, num_sms, st, splits, splits > 1 ? split->ws : nullptr,
+                          splits > 1 ? split->sync : nullptr);
   }
   const bool use256 = (N % 256 == 0) && e256 <= e128 * 1.05;
   return use256 ? launch_tc<256>(A, B, b_tiled, M, N, K, ep, num_sms, st, bmap)

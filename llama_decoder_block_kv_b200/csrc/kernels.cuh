@@ -87,9 +87,22 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                        uint32_t b1, uint32_t b2);
 bool make_tmap_weights(CUtensorMap* map, const void* ptr, int tiled, uint64_t N, uint64_t K, uint32_t box_rows);
+// Scratch of the CTA-pair GEMM's two-way k split, for up to `tiles` 256 x 256
+// tiles: ws gemm_split_ws_floats(tiles) floats, sync gemm_split_sync_ints(tiles)
+// ints, zeroed once (every launch leaves them zeroed).
+struct GemmSplitWs {
+  float* ws = nullptr;
+  int* sync = nullptr;
+  int tiles = 0;
+};
+size_t gemm_split_ws_floats(int tiles);
+size_t gemm_split_sync_ints(int tiles);
+int gemm_split_max_tiles(int num_sms);  // the largest tile count that can take the split
 // bmap (optional, tiled B only): a tensor map of B encoded once by the caller (128-row boxes)
+// split (optional): scratch that lets small-M calls split each pair tile's k range in two
 cudaError_t launch_gemm_tc(const void* A, const void* B, int b_tiled, int M, int N, int K, const EpiParams& ep,
-                           int num_sms, cudaStream_t st, const CUtensorMap* bmap = nullptr);
+                           int num_sms, cudaStream_t st, const CUtensorMap* bmap = nullptr,
+                           const GemmSplitWs* split = nullptr);
 
 // Query heads one decode-attention CTA serves (one kv head's group of n_rep
 // query heads, split into n_rep / hpc groups; an MMA row block holds 16): all of

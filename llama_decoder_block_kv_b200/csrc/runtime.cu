@@ -73,6 +73,7 @@ struct llama_ctx {
   size_t part_floats = 0;
   int* counters = nullptr;
   int counters_n = 0;
+  GemmSplitWs split;  // the CTA-pair GEMM's two-way k split (prefill calls of few tiles), sized by reserve
   // persistent decode kernel: grid-barrier words and per-128-column sums of squares of h
   unsigned* gbar = nullptr;
   float* ssq = nullptr;
@@ -182,6 +183,25 @@ int reserve(llama_ctx* c, int tokens) {
   if ((r = alloc(&c->q, round256(T * c->H * c->D * c->esz)))) return r;
   if ((r = alloc(&c->o, round256(T * c->H * c->D * c->esz)))) return r;
   if ((r = alloc(&c->g, round256(T * c->F * c->esz)))) return r;
+  if (c->bf16) {
+    // the split serves calls of at most gemm_split_max_tiles pair tiles: size it
+    // for the most tiles one of the model's linears has at this many tokens
+    const int Ns[5] = {c->n_qkv, c->dim, 2 * c->F, c->dim, c->V};
+    int tiles = 0;
+    for (int i = 0; i < 5; ++i)
+      if (Ns[i] > 0) tiles = std::max(tiles, (int)((T + 255) / 256) * ((Ns[i] + 255) / 256));
+    tiles = std::min(tiles, gemm_split_max_tiles(c->num_sms));
+    if (tiles > c->split.tiles) {
+      release(reinterpret_cast<void*&>(c->split.ws));
+      release(reinterpret_cast<void*&>(c->split.sync));
+      c->split.tiles = 0;
+      if ((r = alloc(reinterpret_cast<void**>(&c->split.ws), gemm_split_ws_floats(tiles) * sizeof(float)))) return r;
+      if ((r = alloc(reinterpret_cast<void**>(&c->split.sync), gemm_split_sync_ints(tiles) * sizeof(int)))) return r;
+      if (cudaMemset(c->split.sync, 0, gemm_split_sync_ints(tiles) * sizeof(int)) != cudaSuccess)
+        return LLAMA_ERR_CUDA;
+      c->split.tiles = tiles;
+    }
+  }
   c->ws_tokens = tokens;
   return LLAMA_OK;
 }
@@ -219,7 +239,8 @@ int gemm(llama_ctx* c, const void* A, const void* W, const CUtensorMap* wmap, in
                ? LLAMA_OK
                : LLAMA_ERR_CUDA;
   }
-  return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st, wmap) == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  return launch_gemm_tc(A, W, 1, M, N, K, ep, c->num_sms, st, wmap, &c->split) == cudaSuccess ? LLAMA_OK
+                                                                                             : LLAMA_ERR_CUDA;
 }
 
 // A decode call of a few tokens (bf16, dim <= 4096) computes both RMSNorms
@@ -413,6 +434,7 @@ size_t g_lin_part_floats = 0;
 int* g_lin_counters = nullptr;
 int g_lin_counters_n = 0;
 int* g_lin_err = nullptr;
+GemmSplitWs g_lin_split;  // the CTA-pair GEMM's k-split scratch (grown to the call's tiles)
 int g_lin_dev = -1;  // device of the private workspace (the first call's)
 
 }  // namespace
@@ -580,6 +602,8 @@ void llama_destroy(llama_ctx* c) {
   release(c->o);
   release(c->g);
   release(reinterpret_cast<void*&>(c->part));
+  release(reinterpret_cast<void*&>(c->split.ws));
+  release(reinterpret_cast<void*&>(c->split.sync));
   release(reinterpret_cast<void*&>(c->counters));
   release(reinterpret_cast<void*&>(c->gbar));
   release(reinterpret_cast<void*&>(c->ssq));
@@ -1061,9 +1085,25 @@ int llama_linear(const void* x, const void* w, float* y, int M, int N, int K, in
       break;
     }
     case LLAMA_PATH_TCGEN05:
+    {
       if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARGS;
-      if (launch_gemm_tc(x, w, tiled, M, N, K, e, sms, st) != cudaSuccess) return LLAMA_ERR_CUDA;
+      const int tiles = std::min(((M + 255) / 256) * ((N + 255) / 256), gemm_split_max_tiles(sms));
+      if (tiled && tiles > g_lin_split.tiles) {
+        cudaDeviceSynchronize();
+        release(reinterpret_cast<void*&>(g_lin_split.ws));
+        release(reinterpret_cast<void*&>(g_lin_split.sync));
+        g_lin_split.tiles = 0;
+        if (alloc(reinterpret_cast<void**>(&g_lin_split.ws), gemm_split_ws_floats(tiles) * sizeof(float)))
+          return LLAMA_ERR_OOM;
+        if (alloc(reinterpret_cast<void**>(&g_lin_split.sync), gemm_split_sync_ints(tiles) * sizeof(int)))
+          return LLAMA_ERR_OOM;
+        cudaMemset(g_lin_split.sync, 0, gemm_split_sync_ints(tiles) * sizeof(int));
+        g_lin_split.tiles = tiles;
+      }
+      if (launch_gemm_tc(x, w, tiled, M, N, K, e, sms, st, nullptr, &g_lin_split) != cudaSuccess)
+        return LLAMA_ERR_CUDA;
       break;
+    }
     default:
       return LLAMA_ERR_INVALID_ARGS;
   }

@@ -49,6 +49,25 @@ def test_tcgen05_gemm_on_cta_pairs(M, N, K):
     _check(x, w, y)
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 4096, 11008), (300, 4096, 11008), (40, 512, 8192), (40, 512, 8256),
+                                   (512, 12288, 4096), (512, 22016, 4096)])
+def test_tcgen05_gemm_on_cta_pairs_with_k_halves(M, N, K):
+    """Calls whose whole pair tiles fill less than one wave, with long k ranges
+    (the LLaMA-7B layer's w2 at 512 tokens, a ragged 300 and 40, an odd number
+    of 64-wide k steps), split each pair tile's k range in two, run on
+    different pairs; the second half to finish adds the first's partial sums.
+    The 7B layer's wqkv and w1|w3 at 512 tokens stay whole. Against a float64
+    matmul, three calls in a row (the arrival counters and flags re-arm
+    themselves)."""
+    x, w = _inputs(M, N, K, torch.bfloat16, 17)
+    wt = B.llama_tile_weights(w)
+    for _ in range(3):
+        y = torch.full((M, N), float("nan"), device="cuda")
+        B.llama_linear(x, wt, y, B.LLAMA_PATH_TCGEN05 | B.LLAMA_WEIGHTS_TILED, n=N)
+        torch.cuda.synchronize()
+        _check(x, w, y)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 128, 256), (5, 384, 4096), (8, 4096, 4096), (16, 12288, 4096),
                                    (17, 256, 11008), (32, 4096, 14336), (32, 28672, 4096), (3, 136, 192), (9, 8, 128)])
 def test_gemv_split_k(M, N, K):
@@ -100,14 +119,15 @@ def test_simt_gemm(M, N, K, dt):
 
 
 @pytest.mark.parametrize("path,M,N,K", [(B.LLAMA_PATH_GEMV, 1, 12288, 4096), (B.LLAMA_PATH_GEMV, 9, 136, 192),
-                                        (B.LLAMA_PATH_GEMV, 32, 4096, 11008), (B.LLAMA_PATH_TCGEN05, 300, 1024, 1024),
-                                        (B.LLAMA_PATH_TCGEN05, 512, 12288, 4096), (B.LLAMA_PATH_TCGEN05, 77, 384, 448)])
+                                        (B.LLAMA_PATH_GEMV, 32, 4096, 11008), (B.LLAMA_PATH_TCGEN05, 300, 1152, 1024),
+                                        (B.LLAMA_PATH_TCGEN05, 512, 12160, 4096), (B.LLAMA_PATH_TCGEN05, 77, 384, 448)])
 def test_tiled_weights_give_identical_results(path, M, N, K):
     """The tile layout only changes where a 128 x 64 stage is read from: the
     shared-memory image, hence every MMA and every sum, is the same as with
     row-major weights, so the outputs are bit-identical (for shapes that run the
     same kernel with both layouts, as these do: the CTA-pair GEMM takes only
-    tiled weights, test_tcgen05_gemm_on_cta_pairs)."""
+    tiled weights with N a multiple of 256, test_tcgen05_gemm_on_cta_pairs, so
+    the tcgen05 shapes here have N = 128 mod 256)."""
     x, w = _inputs(M, N, K, torch.bfloat16, 41)
     wt = B.llama_tile_weights(w)
     assert wt.numel() == (N + 127) // 128 * 128 * K
