@@ -171,9 +171,9 @@ int llama_set_embed_norm_head(llama_ctx* ctx, const void* tok_embeddings_dev, co
 
 /*
  * Size the workspace for calls of up to max_tokens tokens (B*T): the
- * activation buffers, and in bf16 mode the prefill GEMM's k-split scratch
- * (256 KB per 256 x 256 output tile of the model's widest linear at that many
- * tokens, at most 3 x (SMs / 2) tiles). Calls with more tokens grow it on
+ * activation buffers, and in bf16 mode, above 32 tokens, the prefill GEMM's
+ * k-split scratch (256 KB per 256 x 256 output tile of the model's widest
+ * linear at that many tokens, at most 3 x (SMs / 2) tiles). Calls with more tokens grow it on
  * demand, which allocates and therefore cannot be captured in a CUDA graph;
  * call this first to capture.
  */

@@ -183,7 +183,7 @@ int reserve(llama_ctx* c, int tokens) {
   if ((r = alloc(&c->q, round256(T * c->H * c->D * c->esz)))) return r;
   if ((r = alloc(&c->o, round256(T * c->H * c->D * c->esz)))) return r;
   if ((r = alloc(&c->g, round256(T * c->F * c->esz)))) return r;
-  if (c->bf16) {
+  if (c->bf16 && tokens > 32) {  // calls of up to 32 tokens run the GEMV, not the GEMM
     // the split serves calls of at most gemm_split_max_tiles pair tiles: size it
     // for the most tiles one of the model's linears has at this many tokens
     const int Ns[5] = {c->n_qkv, c->dim, 2 * c->F, c->dim, c->V};
