@@ -608,12 +608,26 @@ __global__ void __launch_bounds__(192, 1)
 // grid = one CTA per SM (fewer if there are fewer stages than SMs); the
 // partial workspace holds one [M][N] slice per contributor of the most-split
 // row block.
+//
+// Where a whole number c >= 2 of CTAs per row block still keeps at least 85 %
+// of the SMs streaming, the grid is row_blocks x c instead: every range then
+// lies inside one row block (each CTA has one segment, one partial tile and at
+// most one merge, and every row block exactly c contributors), rather than
+// most CTAs straddling two row blocks. Measured on B200 (graphs of back-to-back
+// launches, us): one token x [4096 x 4096] 10.7 -> 9.1 and [4096 x 11008]
+// 17.9 -> 17.1; 16 tokens x [8192 x 8192] 25.5 -> 24.9; 32 tokens x [4096 x
+// 4096] 15.5 -> 13.8 and [6144 x 4096] 17.1 -> 15.9; the 7B-layer decode step
+// 85.9 -> 84.0 us per token.
 GemvPlan plan_gemv(int M, int N, int K, int num_sms) {
   GemvPlan p;
   p.row_blocks = (N + RPC - 1) / RPC;
   p.nk = K / KB;
   p.total = p.row_blocks * p.nk;
   p.grid = p.total < num_sms ? p.total : num_sms;
+  if (p.row_blocks <= num_sms) {
+    const int c = num_sms / p.row_blocks;
+    if (c >= 2 && p.row_blocks * c * 100 >= num_sms * 85 && p.nk >= c) p.grid = p.row_blocks * c;
+  }
   int smax = 1;
   for (int rb = 0; rb < p.row_blocks; ++rb) {
     const int c = sk_owner((rb + 1) * p.nk - 1, p.total, p.grid) - sk_owner(rb * p.nk, p.total, p.grid) + 1;
