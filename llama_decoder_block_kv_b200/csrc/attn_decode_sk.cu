@@ -532,6 +532,20 @@ DecodeSkPlan plan_decode_sk(int B, int H, int Hkv, int D, int max_len, int num_s
   return p;
 }
 
+// One position for the whole batch: every unit has the same number of key
+// tiles, so a grid of a whole number of CTAs per unit (where that keeps at
+// least 85 % of the two-per-SM slots) puts each CTA's range inside one unit.
+// Measured on B200, the 70B layer at batch 16 x 4096: 0.3318 -> 0.3292 ms per
+// step (256 CTAs instead of 296). Only ever shrinks the grid, so the
+// workspace sized for plan_decode_sk's grid still holds the partials.
+void align_decode_sk_uniform(DecodeSkPlan& p, int len, int num_sms) {
+  if (!p.ok) return;
+  const int cap = 2 * num_sms, n_t = (len + SKT - 1) / SKT;
+  if (p.units > cap) return;
+  const int cc = cap / p.units;
+  if (p.units * cc * 100 >= cap * 85 && n_t >= cc && p.units * cc < p.grid) p.grid = p.units * cc;
+}
+
 static size_t sk_smem(int D, int B) {
   return 1024 + (size_t)SK_STAGES * 2 * SKT * D * 2 + 2 * SK_STAGES * 8 + (size_t)(2 * B + 1) * 4;
 }

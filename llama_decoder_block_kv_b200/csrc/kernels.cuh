@@ -145,6 +145,8 @@ struct DecodeSkPlan {
   size_t part_floats = 0;
 };
 DecodeSkPlan plan_decode_sk(int B, int H, int Hkv, int D, int max_len, int num_sms);
+// calls whose sequences all hold `len` keys: a grid of whole CTAs per unit where it pays (shrinks only)
+void align_decode_sk_uniform(DecodeSkPlan& p, int len, int num_sms);
 cudaError_t launch_attn_decode_sk(const CUtensorMap& mk, const CUtensorMap& mv, const void* q, void* o, float* part,
                                   int* counters, const int* sp, int sp_scalar, int B, int H, int Hkv, int D, int S_max,
                                   const DecodeSkPlan& p, int* err, cudaStream_t st);

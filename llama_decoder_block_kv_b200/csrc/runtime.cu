@@ -350,18 +350,7 @@ int run_block(llama_ctx* c, int layer, float* h, int B, int T, const int* sp_dev
   } else if (T == 1) {
     const int max_len = sp_dev ? c->S : sp_host + 1;
     DecodeSkPlan sk = plan_decode_sk(B, c->H, c->Hkv, c->D, max_len, c->num_sms);
-    // One position for the whole batch: every unit has the same number of key
-    // tiles, so a grid of a whole number of CTAs per unit (where that keeps at
-    // least 85 % of the two-per-SM slots) puts each CTA's range inside one unit.
-    // Measured on B200, the 70B layer at batch 16 x 4096: 0.3318 -> 0.3292 ms
-    // per step (256 CTAs instead of 296).
-    if (!sp_dev && sk.ok) {
-      const int cap = 2 * c->num_sms, n_t = (max_len + 63) / 64;
-      if (sk.units <= cap) {
-        const int cc = cap / sk.units;
-        if (sk.units * cc * 100 >= cap * 85 && n_t >= cc && sk.units * cc < sk.grid) sk.grid = sk.units * cc;
-      }
-    }
+    if (!sp_dev) align_decode_sk_uniform(sk, max_len, c->num_sms);
     if (c->attn_mode == LLAMA_ATTN_STREAMK && !sk.ok) return LLAMA_ERR_INVALID_ARGS;
     if (sk.ok && use_stream_k(c->attn_mode, sk, max_len, c->num_sms)) {
       if (sk.part_floats > c->part_floats || sk.units > c->counters_n) return LLAMA_ERR_INVALID_ARGS;
@@ -989,6 +978,8 @@ int llama_selfcheck_plans(int M, int dim, int n_heads, int n_kv_heads, int ffn, 
   for (int sp : sps) {
     DecodeSkPlan p1 = plan_decode_sk(M, n_heads, n_kv_heads, D, sp + 1, num_sms);
     std::fill(pos.begin(), pos.end(), sp);
+    if (!check_decode_sk(p1, pos.data(), M, n_heads, n_kv_heads, D, S)) return LLAMA_ERR_INTERNAL;
+    align_decode_sk_uniform(p1, sp + 1, num_sms);  // the grid such calls launch
     if (!check_decode_sk(p1, pos.data(), M, n_heads, n_kv_heads, D, S)) return LLAMA_ERR_INTERNAL;
   }
   return LLAMA_OK;
