@@ -5,8 +5,9 @@
 // (the KV-cache section of "LLaMa-1/2/3 原理+源码——拆解" makes the same
 // point: with the cache the bottleneck becomes memory access).
 //
-// Persistent stream-K kernel, one CTA per SM: the weight stages of all row
-// blocks (128 rows x 64 k each) are dealt out as equal contiguous ranges. A
+// Persistent stream-K kernel, at most one CTA per SM (see plan_gemv for the
+// grid): the weight stages of all row blocks (128 rows x 64 k each) are dealt
+// out as equal contiguous ranges. A
 // producer warp streams its range's weight tiles together with the matching
 // X tiles (8*MB tokens x 64 bf16) through a deep shared-memory ring with TMA
 // (128-byte swizzle, no multicast), never pausing at row-block edges. The
