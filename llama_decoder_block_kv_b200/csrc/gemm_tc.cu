@@ -405,6 +405,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             if (!got) atomicOr(ep.err, LLAMA_DEV_TIMEOUT);
           }
           merge = __shfl_sync(0xffffffffu, got, 0) != 0;
+          __syncwarp();  // orders the other lanes' loads of the partial sums after lane 0's acquire
         }
       }
 #pragma unroll 1
