@@ -136,7 +136,7 @@ constexpr int GV_KMAX = 1024, GV_MMAX = 8;
 }
 
 __global__ void __launch_bounds__(256)
-    gemv_f32_kernel(const float* __restrict__ A, const float* __restrict__ W, int M, int N, int K, EpiParams ep) {
+    llama_decode_linear_f32_kernel(const float* __restrict__ A, const float* __restrict__ W, int M, int N, int K, EpiParams ep) {
   __shared__ float4 xs[GV_MMAX * GV_KMAX / 4];  // the M token rows, GV_KMAX floats apart
   __shared__ float res[GV_MMAX][8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -189,7 +189,7 @@ void launch_gemm_simt(const void* A, const void* W, int M, int N, int K, const E
   if constexpr (sizeof(T) == 4) {
     if (M >= 1 && M <= GV_MMAX && K <= GV_KMAX && K % 4 == 0 && N % 8 == 0 &&
         !(reinterpret_cast<uintptr_t>(A) & 15) && !(reinterpret_cast<uintptr_t>(W) & 15)) {
-      launch_pdl(gemv_f32_kernel, dim3(N / 8), dim3(256), 0, st, reinterpret_cast<const float*>(A),
+      launch_pdl(llama_decode_linear_f32_kernel, dim3(N / 8), dim3(256), 0, st, reinterpret_cast<const float*>(A),
                  reinterpret_cast<const float*>(W), M, N, K, ep);
       return;
     }
